@@ -1,0 +1,245 @@
+/*
+ * symnmf.h -- C ABI of libsymnmf.so, the B200 (sm_100a) SymNMF clustering path.
+ *
+ * The method (sources cited by page title and section):
+ *   [CaS] "GPU-Accelerated Clustering for Financial Instruments at Scale",
+ *         NVIDIA technical blog: sections "Factorization at scale",
+ *         "Choosing the rank k", "Factorizing with SymNMF", "Why this solver",
+ *         "Tracking stability through time with the Rand index".
+ *   [SMI] "GPU-Accelerated SymNMF Clustering Scales to a Million Financial
+ *         Instruments" (English copy of the same post): AdaGrad update in
+ *         LaTeX form and the AdaptGrow algorithm sketch.
+ *   [LRD] abstract of "Low-Rank Dependence Decomposition via Accelerated
+ *         Symmetric Non-negative Matrix Factorization": trace identity,
+ *         Block-SVRG AdaptGrow.
+ *
+ * A dependence matrix S (n x n, |Pearson correlation| or TPDM of a T x n
+ * returns window) is factorised as S ~ H H^T with H >= 0 (n x k) by
+ * projected diagonal AdaGrad on f(H) = ||S||^2 - 2 tr(H^T S H) + ||H^T H||^2,
+ * one pass over S per full-batch iteration; the row-wise argmax of H is the
+ * hard cluster label.
+ *
+ * Conventions shared by every entry point
+ *  - Pointers named S, R, H, G, X, Y, labels and ws are DEVICE pointers on the
+ *    current CUDA device; pointers documented as "host" are host memory.
+ *  - All matrices are row-major.  S is n x n with leading dimension lds >= n
+ *    and FULL symmetric storage (both triangles hold the values; the library
+ *    may read either one).  R is T x n (row = day) with leading dimension
+ *    ldr >= n.  H, G, X, Y are n x k dense (leading dimension k).
+ *  - Alignment: S and R must be 16-byte aligned and lds, ldr multiples of 4
+ *    (16-byte rows), else SYMNMF_ERR_INVALID_ARG.  H, G, X, Y need 4-byte
+ *    alignment.
+ *  - Ownership: the caller allocates and frees everything.  The library
+ *    allocates no device memory: entry points that need scratch take a
+ *    caller-provided workspace `ws` of `ws_bytes` bytes (256-byte aligned),
+ *    sized by symnmf_workspace_size(); too small gives SYMNMF_ERR_WORKSPACE.
+ *  - Streams: work is issued on `stream` (NULL = the legacy default stream).
+ *    Builders, symnmf_sh, symnmf_stats and symnmf_labels are asynchronous.
+ *    symnmf_fit and symnmf_spectral_probe write host outputs and synchronise
+ *    `stream` before they return.
+ *  - Errors: every call returns a symnmf_status; SYMNMF_OK = 0.  A failing
+ *    call leaves a description in symnmf_last_error() (per host thread).
+ *    Not converging within the budget is SYMNMF_OK with stats.converged = 0.
+ *    Sizes: 1 <= n, n*lds and T*ldr below 2^62; 1 <= k <= 64.
+ */
+#ifndef SYMNMF_H
+#define SYMNMF_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define SYMNMF_API __attribute__((visibility("default")))
+#else
+#define SYMNMF_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t / CUstream. */
+typedef struct CUstream_st* symnmf_stream_t;
+
+typedef enum {
+    SYMNMF_OK = 0,
+    SYMNMF_ERR_INVALID_ARG = 1,   /* bad size, pointer, alignment or parameter */
+    SYMNMF_ERR_NONFINITE = 2,     /* S holds NaN/Inf, or the loss became non-finite */
+    SYMNMF_ERR_WORKSPACE = 3,     /* ws_bytes smaller than symnmf_workspace_size() */
+    SYMNMF_ERR_CUDA = 4,          /* a CUDA runtime/driver call failed */
+    SYMNMF_ERR_TIMEOUT = 5,       /* a bounded device-side wait gave up */
+    SYMNMF_ERR_NOT_SUPPORTED = 6  /* no sm_100 device, or option not available */
+} symnmf_status;
+
+enum { SYMNMF_SOLVER_ADAGRAD = 0, SYMNMF_SOLVER_BLOCK_SVRG = 1, SYMNMF_SOLVER_AUTO = 2 };
+enum { SYMNMF_INIT_SEEDED = 0, SYMNMF_INIT_USER = 1 };
+enum {
+    SYMNMF_OP_BUILD_CORR = 0,
+    SYMNMF_OP_BUILD_TPDM = 1,
+    SYMNMF_OP_SPECTRAL_PROBE = 2,
+    SYMNMF_OP_FIT = 3,
+    SYMNMF_OP_SH = 4,
+    SYMNMF_OP_STATS = 5
+};
+
+/*
+ * Parameters of symnmf_fit ([SMI] AdaptGrow sketch: adaptgrow(S, k, lr, phi,
+ * steps, eps)).  Fill with symnmf_fit_params_default() and override.
+ */
+typedef struct {
+    int solver;              /* SYMNMF_SOLVER_*; default ADAGRAD */
+    int init;                /* SYMNMF_INIT_SEEDED (H0 = scale-matched seeded draw) or _USER (H holds H0) */
+    uint64_t seed;           /* init stream seed and Block-SVRG permutation seed; default 0 */
+    float lr;                /* AdaGrad step eta; default 0.1 */
+    float eps;               /* AdaGrad epsilon (outside the root); default 1e-10 */
+    int max_iters;           /* full-batch updates (ADAGRAD) or epochs (BLOCK_SVRG); default 2000 */
+    double rel_tol;          /* stop when |f_t - f_{t-1}| / f_{t-1} < rel_tol; 0 = off; default 1e-5 */
+    int64_t block_rows;      /* Block-SVRG block b; 0 = power of two nearest n/10 */
+    int grow;                /* AdaptGrow: double b when an epoch stalls; default 1 */
+    double stall_tol;        /* stall = relative snapshot-loss decrease below this; default 1e-4 */
+    double gap_threshold;    /* AUTO: gamma_{k+1} >= this selects full batch; default 5.0 */
+    int upper_only;          /* reserved; must be 0 */
+    float* G_inout;          /* optional device n*k: AdaGrad accumulator in (resume) and out; NULL = start at 0 */
+    double* loss_history;    /* optional host array: f(H_t) of every evaluation (snapshots for Block-SVRG) */
+    int loss_history_len;    /* capacity of loss_history */
+    const double* eigvals;   /* optional host, descending: AUTO uses these instead of running the probe */
+    int n_eigvals;           /* length of eigvals (>= k+2 to be used) */
+    int probe_block;         /* AUTO probe block size; default 16 */
+    int probe_max_iter;      /* AUTO probe Lanczos block steps; default 40 */
+    double probe_tol;        /* AUTO probe Ritz tolerance; default 1e-6 */
+    int check_every;         /* host reads the stop flag every this many iterations; default 16 */
+    int timing;              /* 1 = record CUDA-event time of the S-stream kernels in stats */
+} symnmf_fit_params;
+
+typedef struct {
+    int iters;               /* full-batch updates applied to reach the returned H */
+    int epochs;              /* Block-SVRG epochs run */
+    int converged;           /* 1 when rel_tol stopped the run */
+    int solver_used;         /* SYMNMF_SOLVER_ADAGRAD or _BLOCK_SVRG (possibly grown to full batch) */
+    int64_t block_final;     /* Block-SVRG block at exit (n when grown to full batch) */
+    double loss;             /* f(H) of the returned H (trace identity, fp64) */
+    double rel_change;       /* last relative loss change */
+    double gamma;            /* post-rank gap ratio (AUTO), else NaN */
+    double s_mean;           /* sum(S) / n^2 */
+    double s_sqnorm;         /* ||S||_F^2 */
+    int evaluations;         /* passes over S that evaluated the loss (loss_history entries written) */
+    int stream_launches;     /* with timing = 1: S-stream kernel launches timed */
+    double stream_ms;        /* with timing = 1: their summed CUDA-event time, ms */
+    double loop_ms;          /* with timing = 1: CUDA-event time of the iteration loop, ms */
+    int kernel_launches;     /* kernels this call launched */
+} symnmf_fit_stats;
+
+/* Defaults listed in symnmf_fit_params. */
+SYMNMF_API void symnmf_fit_params_default(symnmf_fit_params* params);
+
+/* Static string for a status code. */
+SYMNMF_API const char* symnmf_status_string(int status);
+
+/* Detail of the last failing call on this host thread ("" if none). */
+SYMNMF_API const char* symnmf_last_error(void);
+
+/* Library ABI version (major * 10000 + minor * 100 + patch). */
+SYMNMF_API int symnmf_version(void);
+
+/*
+ * Workspace bytes needed by `op` (SYMNMF_OP_*) for the given sizes.
+ * k: rank (FIT, SH) or n_eig (SPECTRAL_PROBE); T: days (builders);
+ * params: FIT options (may be NULL = defaults) -- for SPECTRAL_PROBE only
+ * probe_block and probe_max_iter are read.  Writes *bytes.
+ */
+SYMNMF_API int symnmf_workspace_size(int op, int64_t n, int k, int64_t T,
+                          const symnmf_fit_params* params, size_t* bytes);
+
+/*
+ * S = |corr(R)|: absolute Pearson correlation of the n columns of the T x n
+ * returns window R ([CaS] "Tracking stability through time...": correlation
+ * captures co-movement over the body of the distribution).
+ * S_ij = |sum_t z_ti z_tj| / sqrt(sum_t z_ti^2 sum_t z_tj^2) with z the
+ * column-centred returns; S_ii = 1; a zero-variance column gives a zero row
+ * and column apart from S_ii = 1.  Column means and norms in fp64.
+ * Requires T >= 2.  Asynchronous.
+ */
+SYMNMF_API int symnmf_build_corr(const float* R, int64_t T, int64_t n, int64_t ldr,
+                      float* S, int64_t lds, void* ws, size_t ws_bytes,
+                      symnmf_stream_t stream);
+
+/*
+ * S = TPDM(R): tail pairwise dependence matrix ([CaS] "Tracking stability
+ * through time...": co-movement conditional on extreme events).
+ *   r_ti  = rank of tail_sign*R_ti within column i (1..T; ties -> earlier day)
+ *   x_ti  = (-ln(r_ti/(T+1)))^(-1/2)         (Frechet, alpha = 2, fp64)
+ *   rho_t = ||x_t||_2                         (fp64)
+ *   E     = the N = max(1, floor(tail_frac*T)) days of largest rho (ties -> earlier day)
+ *   S_ij  = (n/N) sum_{t in E} (x_ti/rho_t)(x_tj/rho_t)
+ * tail_frac in (0, 1]; tail_sign = +1 or -1.  R must be finite.  Asynchronous.
+ */
+SYMNMF_API int symnmf_build_tpdm(const float* R, int64_t T, int64_t n, int64_t ldr,
+                      double tail_frac, int tail_sign, float* S, int64_t lds,
+                      void* ws, size_t ws_bytes, symnmf_stream_t stream);
+
+/*
+ * Statistics pre-pass: out_dev[0] = sum S_ij, out_dev[1] = ||S||_F^2 (fp64,
+ * non-finite entries skipped), out_dev[2] = count of non-finite entries (as a
+ * double).  out_dev is a device array of 3 doubles.  Asynchronous.
+ * ([CaS] "Factorization at scale": ||S||^2 is the constant of the trace loss.)
+ */
+SYMNMF_API int symnmf_stats(const float* S, int64_t n, int64_t lds, double* out_dev,
+                 void* ws, size_t ws_bytes, symnmf_stream_t stream);
+
+/*
+ * Y = S X: one pass of the S-stream ([CaS] "Factorization at scale": the
+ * dominant S H products) for X, Y n x k (1 <= k <= 64).  Asynchronous.
+ */
+SYMNMF_API int symnmf_sh(const float* S, int64_t n, int64_t lds, const float* X, int k,
+              float* Y, void* ws, size_t ws_bytes, symnmf_stream_t stream);
+
+/*
+ * Leading eigenvalues of S by block Lanczos with full reorthogonalisation on
+ * the S-stream ([CaS] "Choosing the rank k": inspect the leading eigenvalues
+ * and pick k at the clearest gap; "Why this solver": gamma_{k+1}).
+ * Writes the n_eig algebraically largest Ritz values, descending, into the
+ * host array eigvals_host.  block (1..64) vectors per step, at most max_iter
+ * block steps (basis <= block*max_iter <= n); stops when every wanted Ritz
+ * residual is <= tol * |lambda_1|.  Start block from the splitmix64 counter
+ * stream of `seed`.  Synchronises `stream`.
+ */
+SYMNMF_API int symnmf_spectral_probe(const float* S, int64_t n, int64_t lds, int n_eig,
+                          int block, int max_iter, double tol, uint64_t seed,
+                          double* eigvals_host, void* ws, size_t ws_bytes,
+                          symnmf_stream_t stream);
+
+/*
+ * Factorise S ~ H H^T, H >= 0 ([SMI] AdaptGrow sketch; [CaS] "Factorizing
+ * with SymNMF": G <- G + g*g, H <- max(H - lr g/(sqrt(G)+eps), 0)).
+ *   ADAGRAD:    g = 4 (H (H^T H) - S H), one S pass per iteration; the pass
+ *               that forms S H_t also evaluates f(H_t) and takes the update.
+ *               Evaluation t = 0..max_iters; stops at the first t > 0 with
+ *               relative loss change < rel_tol, or at t = max_iters, and
+ *               returns H_t.
+ *   BLOCK_SVRG: per epoch a snapshot pass (S H~, f(H~)), then one SVRG step
+ *               per row block of b rows in a seeded order,
+ *               g = 4 (H H^T H - S H~ - m S[:,B] (H_B - H~_B)), m = ceil(n/b);
+ *               stalled epochs double b; at b = n it continues as ADAGRAD.
+ *   AUTO:       gamma_{k+1} = lambda_{k+1}/|lambda_{k+2}| >= gap_threshold
+ *               selects ADAGRAD, else BLOCK_SVRG.
+ * H (n x k, device): output; with INIT_USER also the input H0.
+ * stats_host may be NULL.  Synchronises `stream`.
+ */
+SYMNMF_API int symnmf_fit(const float* S, int64_t n, int64_t lds, int k,
+               const symnmf_fit_params* params, float* H,
+               symnmf_fit_stats* stats_host, void* ws, size_t ws_bytes,
+               symnmf_stream_t stream);
+
+/*
+ * labels[i] = argmax_j H_ij, lowest j on ties ([CaS] "Factorizing with
+ * SymNMF": the row-wise argmax is the hard cluster label).  H n x k, labels
+ * n int32 (device).  Needs no workspace.  Asynchronous.
+ */
+SYMNMF_API int symnmf_labels(const float* H, int64_t n, int k, int32_t* labels,
+                  symnmf_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SYMNMF_H */

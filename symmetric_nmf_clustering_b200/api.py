@@ -1,0 +1,201 @@
+"""Python binding of libsymnmf.so: argument marshalling only.
+
+PyTorch provides device memory and the current CUDA stream; every step of the
+SymNMF path runs in the library's kernels.  Function names follow the C ABI
+(include/symnmf.h) without the ``symnmf_`` prefix.
+"""
+from __future__ import annotations
+
+import ctypes as C
+
+import numpy as np
+import torch
+
+from . import _lib as L
+
+__all__ = ["alloc_S", "workspace", "build_corr", "build_tpdm", "stats", "sh",
+           "spectral_probe", "fit", "labels", "fit_params", "FitParams", "FitStats"]
+
+FitParams = L.FitParams
+FitStats = L.FitStats
+_SOLVERS = {"adagrad": L.SOLVER_ADAGRAD, "block_svrg": L.SOLVER_BLOCK_SVRG, "auto": L.SOLVER_AUTO}
+
+
+def _lib():
+    return L.load()
+
+
+def _stream(device) -> int:
+    return torch.cuda.current_stream(device).cuda_stream
+
+
+def _check_cuda(t: torch.Tensor, name: str, dtype=torch.float32):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise TypeError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+
+
+def _dense(t: torch.Tensor, name: str):
+    _check_cuda(t, name)
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous (row-major)")
+
+
+def _matrix(t: torch.Tensor, name: str):
+    """(rows, cols, leading dimension) of a row-major matrix with unit column stride."""
+    _check_cuda(t, name)
+    if t.dim() != 2 or t.stride(1) != 1:
+        raise ValueError(f"{name} must be a 2-D row-major matrix (unit column stride)")
+    return t.shape[0], t.shape[1], t.stride(0)
+
+
+def alloc_S(n: int, device=None) -> torch.Tensor:
+    """An n x n float32 matrix whose rows are padded to a multiple of 4 floats."""
+    lds = (n + 3) // 4 * 4
+    return torch.empty((n, lds), dtype=torch.float32, device=device)[:, :n]
+
+
+def workspace(op: int, n: int, k: int = 0, T: int = 0, params: FitParams | None = None,
+              device=None) -> torch.Tensor:
+    size = C.c_size_t(0)
+    L.check("symnmf_workspace_size",
+            _lib().symnmf_workspace_size(op, n, k, T, C.byref(params) if params is not None else None,
+                                         C.byref(size)))
+    return torch.empty(max(int(size.value), 256), dtype=torch.uint8, device=device)
+
+
+def build_corr(R: torch.Tensor, out: torch.Tensor | None = None, ws: torch.Tensor | None = None):
+    """S = |Pearson correlation| of the columns of the T x n window R."""
+    T, n, ldr = _matrix(R, "R")
+    S = alloc_S(n, R.device) if out is None else out
+    nS, nS2, lds = _matrix(S, "out")
+    if (nS, nS2) != (n, n):
+        raise ValueError("out must be n x n")
+    ws = workspace(L.OP_BUILD_CORR, n, 0, T, device=R.device) if ws is None else ws
+    L.check("symnmf_build_corr", _lib().symnmf_build_corr(
+        R.data_ptr(), T, n, ldr, S.data_ptr(), lds, ws.data_ptr(), ws.numel(), _stream(R.device)))
+    return S
+
+
+def build_tpdm(R: torch.Tensor, tail_frac: float = 0.05, tail_sign: int = 1,
+               out: torch.Tensor | None = None, ws: torch.Tensor | None = None):
+    """S = TPDM of the T x n window R (top tail_frac of days by radius, scaled by n)."""
+    T, n, ldr = _matrix(R, "R")
+    S = alloc_S(n, R.device) if out is None else out
+    nS, nS2, lds = _matrix(S, "out")
+    if (nS, nS2) != (n, n):
+        raise ValueError("out must be n x n")
+    ws = workspace(L.OP_BUILD_TPDM, n, 0, T, device=R.device) if ws is None else ws
+    L.check("symnmf_build_tpdm", _lib().symnmf_build_tpdm(
+        R.data_ptr(), T, n, ldr, float(tail_frac), int(tail_sign), S.data_ptr(), lds,
+        ws.data_ptr(), ws.numel(), _stream(R.device)))
+    return S
+
+
+def stats(S: torch.Tensor, ws: torch.Tensor | None = None) -> torch.Tensor:
+    """Device tensor [sum S, ||S||_F^2, non-finite count] (float64)."""
+    n, _, lds = _matrix(S, "S")
+    out = torch.empty(3, dtype=torch.float64, device=S.device)
+    ws = workspace(L.OP_STATS, n, device=S.device) if ws is None else ws
+    L.check("symnmf_stats", _lib().symnmf_stats(S.data_ptr(), n, lds, out.data_ptr(),
+                                                ws.data_ptr(), ws.numel(), _stream(S.device)))
+    return out
+
+
+def sh(S: torch.Tensor, X: torch.Tensor, ws: torch.Tensor | None = None) -> torch.Tensor:
+    """Y = S X for an n x k block X (one pass over S)."""
+    n, _, lds = _matrix(S, "S")
+    _dense(X, "X")
+    k = X.shape[1]
+    Y = torch.empty_like(X)
+    ws = workspace(L.OP_SH, n, k, device=S.device) if ws is None else ws
+    L.check("symnmf_sh", _lib().symnmf_sh(S.data_ptr(), n, lds, X.data_ptr(), k, Y.data_ptr(),
+                                          ws.data_ptr(), ws.numel(), _stream(S.device)))
+    return Y
+
+
+def spectral_probe(S: torch.Tensor, n_eig: int, block: int = 16, max_iter: int = 40,
+                   tol: float = 1e-6, seed: int = 0, ws: torch.Tensor | None = None) -> np.ndarray:
+    """The n_eig leading eigenvalues of S (descending) by block Lanczos."""
+    n, _, lds = _matrix(S, "S")
+    p = fit_params(probe_block=block, probe_max_iter=max_iter)
+    ws = workspace(L.OP_SPECTRAL_PROBE, n, n_eig, params=p, device=S.device) if ws is None else ws
+    out = (C.c_double * n_eig)()
+    L.check("symnmf_spectral_probe", _lib().symnmf_spectral_probe(
+        S.data_ptr(), n, lds, n_eig, block, max_iter, float(tol), int(seed) & (2**64 - 1), out,
+        ws.data_ptr(), ws.numel(), _stream(S.device)))
+    return np.array(out[:], dtype=np.float64)
+
+
+def fit_params(**kw) -> FitParams:
+    p = FitParams()
+    _lib().symnmf_fit_params_default(C.byref(p))
+    for key, val in kw.items():
+        if key == "solver" and isinstance(val, str):
+            val = _SOLVERS[val]
+        setattr(p, key, val)
+    return p
+
+
+def fit(S: torch.Tensor, k: int, *, H0: torch.Tensor | None = None, G: torch.Tensor | None = None,
+        solver: str = "adagrad", seed: int = 0, lr: float = 0.1, eps: float = 1e-10,
+        max_iters: int = 2000, rel_tol: float = 1e-5, block_rows: int = 0, grow: bool = True,
+        stall_tol: float = 1e-4, gap_threshold: float = 5.0, eigvals=None,
+        probe_block: int = 16, probe_max_iter: int = 40, probe_tol: float = 1e-6,
+        check_every: int = 16, timing: bool = False, history: bool = False,
+        out: torch.Tensor | None = None, ws: torch.Tensor | None = None):
+    """Factorise S ~ H H^T with H >= 0.  Returns (H, stats dict).
+
+    H0 given: INIT_USER from a copy of H0 (or in place when ``out is H0``);
+    otherwise the scale-matched seeded init.  G (n x k float32) is the AdaGrad
+    accumulator, read and updated in place.  With ``history`` the per-
+    evaluation losses are returned in stats["history"].
+    """
+    n, _, lds = _matrix(S, "S")
+    if H0 is not None:
+        _dense(H0, "H0")
+        H = H0 if out is H0 else H0.clone()
+    else:
+        H = torch.empty((n, k), dtype=torch.float32, device=S.device) if out is None else out
+    _dense(H, "H")
+    if tuple(H.shape) != (n, k):
+        raise ValueError("H must be n x k")
+    p = fit_params(solver=solver, init=L.INIT_USER if H0 is not None else L.INIT_SEEDED,
+                   seed=int(seed) & (2**64 - 1), lr=lr, eps=eps, max_iters=max_iters,
+                   rel_tol=rel_tol, block_rows=block_rows, grow=int(grow), stall_tol=stall_tol,
+                   gap_threshold=gap_threshold, probe_block=probe_block,
+                   probe_max_iter=probe_max_iter, probe_tol=probe_tol, check_every=check_every,
+                   timing=int(timing))
+    if G is not None:
+        _dense(G, "G")
+        p.G_inout = G.data_ptr()
+    hist = None
+    if history:
+        hist = (C.c_double * (max_iters + 1))()
+        p.loss_history = C.cast(hist, C.POINTER(C.c_double))
+        p.loss_history_len = max_iters + 1
+    ev = None
+    if eigvals is not None:
+        ev = (C.c_double * len(eigvals))(*[float(x) for x in eigvals])
+        p.eigvals = C.cast(ev, C.POINTER(C.c_double))
+        p.n_eigvals = len(eigvals)
+    ws = workspace(L.OP_FIT, n, k, params=p, device=S.device) if ws is None else ws
+    st = FitStats()
+    L.check("symnmf_fit", _lib().symnmf_fit(S.data_ptr(), n, lds, k, C.byref(p), H.data_ptr(),
+                                            C.byref(st), ws.data_ptr(), ws.numel(),
+                                            _stream(S.device)))
+    d = st.as_dict()
+    if hist is not None:
+        d["history"] = np.array(hist[:st.evaluations], dtype=np.float64)
+    return H, d
+
+
+def labels(H: torch.Tensor) -> torch.Tensor:
+    """Hard labels: row-wise argmax of H (lowest index on ties), int32."""
+    _dense(H, "H")
+    n, k = H.shape
+    out = torch.empty(n, dtype=torch.int32, device=H.device)
+    L.check("symnmf_labels", _lib().symnmf_labels(H.data_ptr(), n, k, out.data_ptr(),
+                                                  _stream(H.device)))
+    return out

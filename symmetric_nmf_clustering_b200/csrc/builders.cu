@@ -1,0 +1,335 @@
+// Dependence-matrix builders from a T x n returns window ([CaS] "Tracking
+// stability through time with the Rand index": |Pearson correlation| for the
+// body of the distribution, TPDM for co-movement in the tails).
+//
+// Both end in a symmetric Gram S = c * op(Z^T Z) over the day index, computed
+// by one tiled kernel with the builder's epilogue (abs + unit diagonal for
+// correlation, the n/N scale for TPDM).
+#include "common.cuh"
+
+namespace symnmf {
+
+constexpr int GB = 128;   // Gram output tile (GB x GB)
+constexpr int GK = 16;    // day-slab per stage
+constexpr int GT = 256;   // threads, 8 x 8 outputs each
+
+enum GramMode { GRAM_CORR = 0, GRAM_TPDM = 1 };
+
+static int64_t round_up(int64_t a, int64_t b) { return (a + b - 1) / b * b; }
+
+// S[i][j] = epi(sum_t Z[t][i] Z[t][j]) for the tile (blockIdx.y, blockIdx.x).
+// Z is Kp x ldz (Kp multiple of GK, ldz multiple of GB, zero padded).
+__global__ void __launch_bounds__(GT)
+gram_kernel(const float* __restrict__ Z, int64_t ldz, int Kp, int64_t n,
+            float* __restrict__ S, int64_t lds, int mode, float scale) {
+    __shared__ __align__(16) float As[2][GK][GB];
+    __shared__ __align__(16) float Bs[2][GK][GB];
+    const int tid = threadIdx.x;
+    const int64_t I0 = (int64_t)blockIdx.y * GB, J0 = (int64_t)blockIdx.x * GB;
+    const int tx = tid % 16, ty = tid / 16;
+
+    float acc[8][8];
+#pragma unroll
+    for (int a = 0; a < 8; ++a)
+#pragma unroll
+        for (int b = 0; b < 8; ++b) acc[a][b] = 0.f;
+
+    // each thread moves 2 float4 of each operand per stage
+    float4 ra[2], rb[2];
+    auto load = [&](int k0) {
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+            const int e = tid + q * GT;
+            const int row = e / 32, c4 = e % 32;
+            const float* base = Z + (int64_t)(k0 + row) * ldz;
+            ra[q] = *reinterpret_cast<const float4*>(base + I0 + c4 * 4);
+            rb[q] = *reinterpret_cast<const float4*>(base + J0 + c4 * 4);
+        }
+    };
+    auto store = [&](int buf) {
+#pragma unroll
+        for (int q = 0; q < 2; ++q) {
+            const int e = tid + q * GT;
+            const int row = e / 32, c4 = e % 32;
+            *reinterpret_cast<float4*>(&As[buf][row][c4 * 4]) = ra[q];
+            *reinterpret_cast<float4*>(&Bs[buf][row][c4 * 4]) = rb[q];
+        }
+    };
+
+    load(0);
+    store(0);
+    __syncthreads();
+    int buf = 0;
+    for (int k0 = 0; k0 < Kp; k0 += GK) {
+        const bool more = k0 + GK < Kp;
+        if (more) load(k0 + GK);
+#pragma unroll
+        for (int kk = 0; kk < GK; ++kk) {
+            const float4 a0 = *reinterpret_cast<const float4*>(&As[buf][kk][ty * 4]);
+            const float4 a1 = *reinterpret_cast<const float4*>(&As[buf][kk][64 + ty * 4]);
+            const float4 b0 = *reinterpret_cast<const float4*>(&Bs[buf][kk][tx * 4]);
+            const float4 b1 = *reinterpret_cast<const float4*>(&Bs[buf][kk][64 + tx * 4]);
+            const float a[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+            const float b[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+#pragma unroll
+            for (int r = 0; r < 8; ++r)
+#pragma unroll
+                for (int c = 0; c < 8; ++c) acc[r][c] = fmaf(a[r], b[c], acc[r][c]);
+        }
+        if (more) {
+            store(buf ^ 1);
+            __syncthreads();
+            buf ^= 1;
+        }
+    }
+
+#pragma unroll
+    for (int r = 0; r < 8; ++r) {
+        const int64_t i = I0 + (r < 4 ? ty * 4 + r : 64 + ty * 4 + (r - 4));
+        if (i >= n) continue;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+            const int64_t j = J0 + h * 64 + tx * 4;
+            float v[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                float x = acc[r][h * 4 + u];
+                if (mode == GRAM_CORR) {
+                    x = fabsf(x);
+                    if (i == j + u) x = 1.f;
+                } else {
+                    x *= scale;
+                }
+                v[u] = x;
+            }
+            float* dst = S + i * lds + j;
+            if (j + 3 < n) {
+                *reinterpret_cast<float4*>(dst) = make_float4(v[0], v[1], v[2], v[3]);
+            } else {
+                for (int u = 0; u < 4; ++u)
+                    if (j + u < n) dst[u] = v[u];
+            }
+        }
+    }
+}
+
+static int launch_gram(const float* Z, int64_t ldz, int Kp, int64_t n, float* S, int64_t lds,
+                       int mode, float scale, cudaStream_t s) {
+    const int64_t tiles = (n + GB - 1) / GB;
+    if (tiles > 65535) {
+        set_error("n = %lld too large for the Gram tile grid", (long long)n);
+        return SYMNMF_ERR_INVALID_ARG;
+    }
+    dim3 grid((unsigned)tiles, (unsigned)tiles);
+    gram_kernel<<<grid, GT, 0, s>>>(Z, ldz, Kp, n, S, lds, mode, scale);
+    SYMNMF_LAUNCH_CHECK();
+    return SYMNMF_OK;
+}
+
+// ----------------------------------------------------------------------------
+// |Pearson correlation|
+// ----------------------------------------------------------------------------
+int corr_plan(Arena& a, int64_t T, int64_t n, double** mu, double** inv, float** Z,
+              int64_t* ldz) {
+    *ldz = round_up(n, GB);
+    const int64_t Kp = round_up(T, GK);
+    *mu = a.take<double>(n);
+    *inv = a.take<double>(n);
+    *Z = a.take<float>((size_t)Kp * *ldz);
+    return SYMNMF_OK;
+}
+
+// Column means and inverse norms of the centred columns, fp64 two-pass.
+__global__ void colstats_kernel(const float* __restrict__ R, int64_t T, int64_t n,
+                                int64_t ldr, double* __restrict__ mu,
+                                double* __restrict__ inv) {
+    const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= n) return;
+    double s = 0.0;
+    for (int64_t t = 0; t < T; ++t) s += (double)R[t * ldr + i];
+    const double m = s / (double)T;
+    double ss = 0.0;
+    for (int64_t t = 0; t < T; ++t) {
+        const double d = (double)R[t * ldr + i] - m;
+        ss = fma(d, d, ss);
+    }
+    mu[i] = m;
+    inv[i] = ss > 0.0 ? 1.0 / sqrt(ss) : 0.0;   // zero-variance column -> zero row of Z
+}
+
+// Z[t][i] = (R[t][i] - mu_i) / ||R_i - mu_i||, zero in the padding.
+__global__ void normalize_kernel(const float* __restrict__ R, int64_t T, int64_t n,
+                                 int64_t ldr, const double* __restrict__ mu,
+                                 const double* __restrict__ inv, float* __restrict__ Z,
+                                 int64_t ldz, int64_t Kp) {
+    const int64_t total = Kp * ldz;
+    for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < total;
+         e += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t t = e / ldz, i = e % ldz;
+        float z = 0.f;
+        if (t < T && i < n) z = (float)(((double)R[t * ldr + i] - mu[i]) * inv[i]);
+        Z[e] = z;
+    }
+}
+
+int launch_corr(const float* R, int64_t T, int64_t n, int64_t ldr, float* S,
+                int64_t lds, double* mu, double* inv, float* Z, int64_t ldz,
+                cudaStream_t s) {
+    const int64_t Kp = round_up(T, GK);
+    colstats_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(R, T, n, ldr, mu, inv);
+    SYMNMF_LAUNCH_CHECK();
+    const int64_t total = Kp * ldz;
+    const int64_t blocks = min64((total + 255) / 256, 8192);
+    normalize_kernel<<<(unsigned)blocks, 256, 0, s>>>(R, T, n, ldr, mu, inv, Z, ldz, Kp);
+    SYMNMF_LAUNCH_CHECK();
+    return launch_gram(Z, ldz, (int)Kp, n, S, lds, GRAM_CORR, 1.f, s);
+}
+
+// ----------------------------------------------------------------------------
+// TPDM
+// ----------------------------------------------------------------------------
+int tpdm_plan(Arena& a, int64_t T, int64_t n, int N, int32_t** ranks, double** phi,
+              double** rho, int32_t** days, float** W, int64_t* ldw) {
+    *ldw = round_up(n, GB);
+    *ranks = a.take<int32_t>((size_t)T * n);
+    *phi = a.take<double>((size_t)T + 1);
+    *rho = a.take<double>((size_t)T);
+    *days = a.take<int32_t>((size_t)N);
+    *W = a.take<float>((size_t)round_up(N, GK) * *ldw);
+    return SYMNMF_OK;
+}
+
+constexpr int RK_COLS = 32;                       // columns per block (one per lane)
+constexpr int RK_THREADS = 256;
+constexpr int64_t RK_SMEM_MAX = 200 * 1024;       // stage the columns in smem up to this
+
+// r_ti = 1 + #{s : x_s < x_t} + #{s < t : x_s == x_t}, x = tail_sign * R[:, i]
+template <bool SMEM>
+__global__ void __launch_bounds__(RK_THREADS)
+rank_kernel(const float* __restrict__ R, int64_t T, int64_t n, int64_t ldr, float sign,
+            int32_t* __restrict__ ranks) {
+    extern __shared__ float xs[];  // [T][32] when SMEM
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+    const int64_t i = (int64_t)blockIdx.x * RK_COLS + lane;
+    const bool valid = i < n;
+    const int64_t ic = valid ? i : 0;
+    if (SMEM) {
+        for (int64_t t = w; t < T; t += RK_THREADS / 32)
+            xs[t * RK_COLS + lane] = valid ? sign * R[t * ldr + ic] : 0.f;
+        __syncthreads();
+    }
+    auto val = [&](int64_t t) -> float {
+        return SMEM ? xs[t * RK_COLS + lane] : sign * __ldg(R + t * ldr + ic);
+    };
+    for (int64_t base = (int64_t)w * 4; base < T; base += 4 * (RK_THREADS / 32)) {
+        float x[4];
+        int cnt[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            x[q] = base + q < T ? val(base + q) : 0.f;
+            cnt[q] = 0;
+        }
+        for (int64_t s2 = 0; s2 < T; ++s2) {
+            const float v = val(s2);
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+                cnt[q] += (v < x[q]) | ((v == x[q]) & (s2 < base + q));
+        }
+        if (valid) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+                if (base + q < T) ranks[(base + q) * n + i] = cnt[q] + 1;
+        }
+    }
+}
+
+// phi[r] = (-ln(r / (T+1)))^(-1/2): Frechet (alpha = 2) margin of rank r, fp64.
+__global__ void phi_kernel(double* __restrict__ phi, int64_t T) {
+    const int64_t r = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (r > T) return;
+    phi[r] = r == 0 ? 0.0 : 1.0 / sqrt(-log((double)r / (double)(T + 1)));
+}
+
+// rho_t = sqrt(sum_i phi[r_ti]^2), one block per day, fixed reduction order.
+__global__ void rho_kernel(const int32_t* __restrict__ ranks, const double* __restrict__ phi,
+                           int64_t n, double* __restrict__ rho) {
+    __shared__ double red[256];
+    const int64_t t = blockIdx.x;
+    double s = 0.0;
+    for (int64_t i = threadIdx.x; i < n; i += blockDim.x) {
+        const double x = phi[ranks[t * n + i]];
+        s = fma(x, x, s);
+    }
+    red[threadIdx.x] = s;
+    __syncthreads();
+    for (int o = 128; o > 0; o >>= 1) {
+        if ((int)threadIdx.x < o) red[threadIdx.x] += red[threadIdx.x + o];
+        __syncthreads();
+    }
+    if (threadIdx.x == 0) rho[t] = sqrt(red[0]);
+}
+
+// days[p] = the day of position p when days are ordered by decreasing rho,
+// ties to the earlier day; only positions p < N are written.
+__global__ void select_kernel(const double* __restrict__ rho, int64_t T, int N,
+                              int32_t* __restrict__ days) {
+    const int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (t >= T) return;
+    const double r = rho[t];
+    int64_t pos = 0;
+    for (int64_t s2 = 0; s2 < T; ++s2) {
+        const double q = rho[s2];
+        pos += (q > r) | ((q == r) & (s2 < t));
+    }
+    if (pos < N) days[pos] = (int32_t)t;
+}
+
+// W[p][i] = phi[r_{days[p], i}] / rho_{days[p]}; zero padding to Np x ldw.
+__global__ void gather_w_kernel(const int32_t* __restrict__ ranks, const double* __restrict__ phi,
+                                const double* __restrict__ rho, const int32_t* __restrict__ days,
+                                int N, int64_t n, float* __restrict__ W, int64_t ldw,
+                                int64_t Np) {
+    const int64_t total = Np * ldw;
+    for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < total;
+         e += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t p = e / ldw, i = e % ldw;
+        float v = 0.f;
+        if (p < N && i < n) {
+            const int64_t t = days[p];
+            v = (float)(phi[ranks[t * n + i]] / rho[t]);
+        }
+        W[e] = v;
+    }
+}
+
+int launch_tpdm(const float* R, int64_t T, int64_t n, int64_t ldr, int N,
+                int tail_sign, float* S, int64_t lds, int32_t* ranks, double* phi,
+                double* rho, int32_t* days, float* W, int64_t ldw, cudaStream_t s) {
+    const unsigned rblocks = (unsigned)((n + RK_COLS - 1) / RK_COLS);
+    const int64_t smem = T * RK_COLS * (int64_t)sizeof(float);
+    const float sign = tail_sign < 0 ? -1.f : 1.f;
+    if (smem <= RK_SMEM_MAX) {
+        SYMNMF_CUDA_TRY(cudaFuncSetAttribute(rank_kernel<true>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)RK_SMEM_MAX));
+        rank_kernel<true><<<rblocks, RK_THREADS, (size_t)smem, s>>>(R, T, n, ldr, sign, ranks);
+    } else {
+        rank_kernel<false><<<rblocks, RK_THREADS, 0, s>>>(R, T, n, ldr, sign, ranks);
+    }
+    SYMNMF_LAUNCH_CHECK();
+    phi_kernel<<<(unsigned)((T + 1 + 255) / 256), 256, 0, s>>>(phi, T);
+    SYMNMF_LAUNCH_CHECK();
+    rho_kernel<<<(unsigned)T, 256, 0, s>>>(ranks, phi, n, rho);
+    SYMNMF_LAUNCH_CHECK();
+    select_kernel<<<(unsigned)((T + 255) / 256), 256, 0, s>>>(rho, T, N, days);
+    SYMNMF_LAUNCH_CHECK();
+    const int64_t Np = round_up(N, GK);
+    const int64_t total = Np * ldw;
+    const int64_t blocks = min64((total + 255) / 256, 8192);
+    gather_w_kernel<<<(unsigned)blocks, 256, 0, s>>>(ranks, phi, rho, days, N, n, W, ldw, Np);
+    SYMNMF_LAUNCH_CHECK();
+    const float scale = (float)((double)n / (double)N);
+    return launch_gram(W, ldw, (int)Np, n, S, lds, GRAM_TPDM, scale, s);
+}
+
+}  // namespace symnmf

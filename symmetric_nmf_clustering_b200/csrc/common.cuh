@@ -1,0 +1,166 @@
+// Internal declarations shared by the libsymnmf translation units.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <algorithm>
+#include <cstdio>
+#include <string>
+
+#include "symnmf.h"
+
+namespace symnmf {
+
+__host__ __device__ __forceinline__ int64_t min64(int64_t a, int64_t b) { return a < b ? a : b; }
+__host__ __device__ __forceinline__ int64_t max64(int64_t a, int64_t b) { return a > b ? a : b; }
+
+// ---------------------------------------------------------------- errors
+void set_error(const char* fmt, ...);
+void clear_error();
+
+struct Status {
+    int code = SYMNMF_OK;
+};
+
+#define SYMNMF_CUDA_TRY(expr)                                                     \
+    do {                                                                          \
+        cudaError_t e_ = (expr);                                                  \
+        if (e_ != cudaSuccess) {                                                  \
+            ::symnmf::set_error("%s failed: %s (%s:%d)", #expr,                   \
+                                cudaGetErrorString(e_), __FILE__, __LINE__);      \
+            return SYMNMF_ERR_CUDA;                                               \
+        }                                                                         \
+    } while (0)
+
+// Kernels launched by the calling host thread (reset by the entry points).
+void note_launch();
+int launches();
+void reset_launches();
+
+#define SYMNMF_LAUNCH_CHECK()                                                     \
+    do {                                                                          \
+        ::symnmf::note_launch();                                                  \
+        cudaError_t e_ = cudaGetLastError();                                      \
+        if (e_ != cudaSuccess) {                                                  \
+            ::symnmf::set_error("kernel launch failed: %s (%s:%d)",               \
+                                cudaGetErrorString(e_), __FILE__, __LINE__);      \
+            return SYMNMF_ERR_CUDA;                                               \
+        }                                                                         \
+    } while (0)
+
+#define SYMNMF_TRY(expr)                                                          \
+    do {                                                                          \
+        int s_ = (expr);                                                          \
+        if (s_ != SYMNMF_OK) return s_;                                           \
+    } while (0)
+
+// ---------------------------------------------------------------- workspace
+// A bump allocator over the caller's workspace; every block 256-byte aligned.
+struct Arena {
+    char* base = nullptr;
+    size_t cap = 0;
+    size_t used = 0;
+    bool dry = false;  // sizing pass: no base pointer
+    template <class T>
+    T* take(size_t count) {
+        size_t off = (used + 255) & ~size_t(255);
+        used = off + count * sizeof(T);
+        if (dry || used > cap) return nullptr;
+        return reinterpret_cast<T*>(base + off);
+    }
+    bool ok() const { return dry || used <= cap; }
+};
+
+// ---------------------------------------------------------------- device state
+// Loop state of a fit, kept in the workspace and updated by the finalise kernel.
+constexpr int KMAX = 64;
+struct FitState {
+    double s_sum, s_sqnorm, s_bad;     // statistics pre-pass
+    double loss, loss_prev, rel;       // last evaluation
+    double A64[KMAX * KMAX];           // Gram H^T H of the current iterate (fp64)
+    float A32[KMAX * KMAX];            // same, rounded to fp32 for the epilogue
+    int t;                             // evaluations done
+    int t_stop;                        // evaluation index of the returned iterate
+    int done;                          // 1: stop issued (no further work)
+    int converged;
+    int nonfinite;
+    int pad_;
+};
+
+// Epilogue / finalise modes.
+enum Mode : int {
+    MODE_FULL = 0,        // evaluate f(H_t), full-gradient AdaGrad step, Gram of H_{t+1}
+    MODE_SNAPSHOT = 1,    // Block-SVRG snapshot: store P~ = S H, evaluate f(H), no step
+    MODE_SVRG_INNER = 2,  // Block-SVRG inner step: P = P~ + m Y, AdaGrad step, Gram
+    MODE_GRAM = 3,        // Gram of the given H only
+    MODE_PRODUCT = 4,     // store Y = S X
+    MODE_STEP_SNAP = 5    // full-gradient step from the stored P~ (no S pass), Gram
+};
+
+// ---------------------------------------------------------------- kernels (launchers)
+struct Dev {
+    int sms = 148;
+    int cc_major = 10;
+};
+int device_info(Dev* d);
+
+// S-stream partial products part[s] = S[J_s, :]^T X[J_s, :] (see stream.cu)
+struct StreamPlan {
+    int64_t n;        // rows of the output (instruments)
+    int k;            // columns of X
+    int64_t j0, j1;   // contraction range (rows of S read, by symmetry)
+    int splits;       // contraction splits
+    int kp;           // padded column count of one pass (8, 16, 24, 32)
+    int groups;       // column groups (k > 32)
+};
+StreamPlan plan_stream(const Dev& d, int64_t n, int k, int64_t j0, int64_t j1);
+size_t stream_partial_floats(const StreamPlan& p);
+int launch_stream_partial(const StreamPlan& p, const float* S, int64_t lds,
+                          const float* Xa, const float* Xb, int64_t ldx, float* part,
+                          const FitState* st, cudaStream_t s);
+size_t fit_state_bytes();
+
+int epilogue_blocks(int64_t n);
+int launch_epilogue(int mode, int64_t n, int k, const float* part, int splits,
+                    const float* H, const float* G, float* Hn, float* Gn,
+                    float* Psnap, float m_scale, float lr, float eps,
+                    double* tr_part, double* gram_part, float* Y,
+                    const FitState* st, cudaStream_t s);
+int launch_finalize(int mode, int nblk, int k, const double* tr_part,
+                    const double* gram_part, FitState* st, double rel_tol,
+                    int max_evals, double* history, int history_cap,
+                    cudaStream_t s);
+
+int launch_stats(const float* S, int64_t n, int64_t lds, double* part, int nblk,
+                 double* out3, cudaStream_t s);
+int stats_blocks();
+int launch_init(float* H, int64_t n, int k, uint64_t seed, const FitState* st,
+                cudaStream_t s);
+int launch_labels(const float* H, int64_t n, int k, int32_t* labels, cudaStream_t s);
+
+// builders
+int corr_plan(Arena& a, int64_t T, int64_t n, double** mu, double** inv, float** Z,
+              int64_t* ldz);
+int launch_corr(const float* R, int64_t T, int64_t n, int64_t ldr, float* S,
+                int64_t lds, double* mu, double* inv, float* Z, int64_t ldz,
+                cudaStream_t s);
+int tpdm_plan(Arena& a, int64_t T, int64_t n, int N, int32_t** ranks, double** phi,
+              double** rho, int32_t** days, float** W, int64_t* ldw);
+int launch_tpdm(const float* R, int64_t T, int64_t n, int64_t ldr, int N,
+                int tail_sign, float* S, int64_t lds, int32_t* ranks, double* phi,
+                double* rho, int32_t* days, float* W, int64_t ldw, cudaStream_t s);
+
+// small dense helpers for the spectral probe
+int launch_uniform_fill(float* X, int64_t count, uint64_t seed, float offset,
+                        cudaStream_t s);
+int launch_gemm_tn(const float* V, int64_t n, int64_t ldv, int cv, const float* W,
+                   int64_t ldw, int cw, double* C, double* part, int nblk,
+                   cudaStream_t s);
+int gemm_tn_blocks(int64_t n);
+int launch_gemm_nn_sub(float* W, int64_t n, int64_t ldw, int cw, const float* V,
+                       int64_t ldv, int cv, const float* C, cudaStream_t s);
+int launch_trsm_right(float* W, int64_t n, int64_t ldw, int cw, const float* Rinv,
+                      cudaStream_t s);
+
+}  // namespace symnmf
