@@ -4,6 +4,7 @@
 // data runs in the kernels of stream.cu, misc.cu and builders.cu.
 #include <cmath>
 #include <cstdarg>
+#include <cstdlib>
 #include <cstring>
 #include <limits>
 #include <vector>
@@ -71,6 +72,40 @@ static int check_S(const float* S, int64_t n, int64_t lds) {
     return SYMNMF_OK;
 }
 
+// ---------------------------------------------------------------- S-stream dispatch
+// The tensor-core kernel is the S-stream; SYMNMF_STREAM=cuda_core selects the
+// CUDA-core kernel instead (same result within fp32 rounding), for comparison.
+static bool use_tc() {
+    static int v = -1;
+    if (v < 0) {
+        const char* e = getenv("SYMNMF_STREAM");
+        v = (e != nullptr && std::strcmp(e, "cuda_core") == 0) ? 0 : 1;
+    }
+    return v == 1;
+}
+
+static size_t stream_partials(const Dev& d, int64_t n, int k, int64_t r0, int64_t r1) {
+    return std::max(stream_partial_floats(plan_stream(d, n, k, r0, r1)),
+                    tc_partial_floats(plan_stream_tc(d, n, k, r0, r1)));
+}
+
+struct StreamArgs {
+    const float* S;
+    int64_t n, lds;
+    int k;
+    float* part;
+    float* XT;     // [X_hi; X_lo] operand buffer (tensor-core path)
+    int64_t ldxt;
+    int* err;
+    const FitState* st;
+};
+
+// part[s] = S[:, r0:r1] X[r0:r1, :] with X = Xa - Xb (Xb may be NULL) on the rows
+// [r0, r1).  xt_ready: XT already holds the split of X (tensor-core path).
+static int stream_product(const Dev& d, const StreamArgs& a, const float* Xa, const float* Xb,
+                          int64_t ldx, int64_t r0, int64_t r1, bool xt_ready, cudaStream_t s,
+                          int* splits, struct Timing* tm);
+
 // ---------------------------------------------------------------- workspace plans
 struct FitLayout {
     FitState* st = nullptr;
@@ -87,6 +122,8 @@ struct FitLayout {
     void* probe_ws = nullptr;
     size_t probe_bytes = 0;
     int hist_cap = 0;
+    float* XT = nullptr;
+    int64_t ldxt = 0;
 };
 
 static int64_t default_block_rows(int64_t n) {
@@ -104,6 +141,9 @@ struct ProbeLayout {
     float* Q = nullptr;      // n x mtot basis, row-major (ld = mtot)
     float* W = nullptr;      // n x b product block
     float* part = nullptr;   // stream partials
+    float* XT = nullptr;     // split operand of the tensor-core stream
+    int64_t ldxt = 0;
+    int* err = nullptr;
     double* tn_part = nullptr;
     double* C64 = nullptr;
     float* C32 = nullptr;
@@ -119,11 +159,13 @@ static int64_t probe_mtot(int64_t n, int block, int max_iter) {
 static size_t probe_workspace(const Dev& d, int64_t n, int block, int max_iter, Arena* a,
                               ProbeLayout* L) {
     const int64_t mtot = std::max<int64_t>(probe_mtot(n, block, max_iter), block);
-    StreamPlan sp = plan_stream(d, n, block, 0, n);
     L->mtot = (int)mtot;
     L->Q = a->take<float>((size_t)n * mtot);
     L->W = a->take<float>((size_t)n * block);
-    L->part = a->take<float>(stream_partial_floats(sp));
+    L->part = a->take<float>(stream_partials(d, n, block, 0, n));
+    L->ldxt = xt_ld(n);
+    L->XT = a->take<float>((size_t)xt_rows(block) * L->ldxt);
+    L->err = a->take<int>(64);
     L->tn_part = a->take<double>((size_t)gemm_tn_blocks(n) * 4096);
     L->C64 = a->take<double>((size_t)mtot * block);
     L->C32 = a->take<float>((size_t)mtot * block);
@@ -137,7 +179,7 @@ static int plan_fit(const Dev& d, Arena& a, int64_t n, int k, const symnmf_fit_p
     L->H1 = a.take<float>((size_t)n * k);
     L->G0 = a.take<float>((size_t)n * k);
     L->G1 = a.take<float>((size_t)n * k);
-    size_t pf = stream_partial_floats(plan_stream(d, n, k, 0, n));
+    size_t pf = stream_partials(d, n, k, 0, n);
     const bool svrg = P.solver != SYMNMF_SOLVER_ADAGRAD;
     int64_t b = 0;
     if (svrg) {
@@ -147,11 +189,13 @@ static int plan_fit(const Dev& d, Arena& a, int64_t n, int k, const symnmf_fit_p
             const int64_t m = (n + bb - 1) / bb;
             for (int64_t blk = 0; blk < m && blk < 2; ++blk) {
                 const int64_t r0 = blk * bb, r1 = std::min(n, r0 + bb);
-                pf = std::max(pf, stream_partial_floats(plan_stream(d, n, k, r0, r1)));
+                pf = std::max(pf, stream_partials(d, n, k, r0, r1));
             }
         }
     }
     L->part = a.take<float>(pf);
+    L->ldxt = xt_ld(n);
+    L->XT = a.take<float>((size_t)xt_rows(k) * L->ldxt);
     const int nb = epilogue_blocks(n);
     L->tr_part = a.take<double>((size_t)nb);
     L->gram_part = a.take<double>((size_t)nb * k * k);
@@ -258,6 +302,27 @@ static int read_state(const FitState* st, HostState* h, cudaStream_t s) {
     return SYMNMF_OK;
 }
 
+static int stream_product(const Dev& d, const StreamArgs& a, const float* Xa, const float* Xb,
+                          int64_t ldx, int64_t r0, int64_t r1, bool xt_ready, cudaStream_t s,
+                          int* splits, Timing* tm) {
+    if (use_tc()) {
+        const TcPlan p = plan_stream_tc(d, a.n, a.k, r0, r1);
+        if (!xt_ready)
+            SYMNMF_TRY(launch_split(Xa, Xb, ldx, a.k, r0, r1, p.j0, p.j1, a.XT, a.ldxt, s));
+        if (tm) SYMNMF_TRY(tm->begin(s));
+        SYMNMF_TRY(launch_stream_tc(p, a.S, a.lds, a.XT, a.ldxt, a.part, a.err, a.st, s));
+        if (tm) SYMNMF_TRY(tm->end(s));
+        *splits = p.splits;
+    } else {
+        const StreamPlan p = plan_stream(d, a.n, a.k, r0, r1);
+        if (tm) SYMNMF_TRY(tm->begin(s));
+        SYMNMF_TRY(launch_stream_partial(p, a.S, a.lds, Xa, Xb, ldx, a.part, a.st, s));
+        if (tm) SYMNMF_TRY(tm->end(s));
+        *splits = p.splits;
+    }
+    return SYMNMF_OK;
+}
+
 struct FitCtx {
     Dev d;
     const float* S;
@@ -272,17 +337,31 @@ struct FitCtx {
     int epochs = 0;
     cudaStream_t s;
     Timing tm;
+    StreamArgs args() const {
+        StreamArgs a;
+        a.S = S;
+        a.n = n;
+        a.lds = lds;
+        a.k = k;
+        a.part = L.part;
+        a.XT = L.XT;
+        a.ldxt = L.ldxt;
+        a.err = &L.st->kerr;
+        a.st = L.st;
+        return a;
+    }
 };
 
 // One S pass + epilogue + finalise in `mode`, reading Hb[cur], writing Hb[cur^1].
-static int full_pass(FitCtx& c, int mode, int max_evals) {
-    StreamPlan sp = plan_stream(c.d, c.n, c.k, 0, c.n);
-    SYMNMF_TRY(c.tm.begin(c.s));
-    SYMNMF_TRY(launch_stream_partial(sp, c.S, c.lds, c.Hb[c.cur], nullptr, c.k, c.L.part, c.L.st, c.s));
-    SYMNMF_TRY(c.tm.end(c.s));
-    SYMNMF_TRY(launch_epilogue(mode, c.n, c.k, c.L.part, sp.splits, c.Hb[c.cur], c.Gb[c.cur],
+// xt_ready: the split operand of Hb[cur] is already in XT (full-batch loop).
+static int full_pass(FitCtx& c, int mode, int max_evals, bool xt_ready) {
+    int splits = 0;
+    SYMNMF_TRY(stream_product(c.d, c.args(), c.Hb[c.cur], nullptr, c.k, 0, c.n, xt_ready, c.s,
+                              &splits, &c.tm));
+    SYMNMF_TRY(launch_epilogue(mode, c.n, c.k, c.L.part, splits, c.Hb[c.cur], c.Gb[c.cur],
                                c.Hb[c.cur ^ 1], c.Gb[c.cur ^ 1], c.L.Psnap, 0.f, c.P->lr,
-                               c.P->eps, c.L.tr_part, c.L.gram_part, nullptr, c.L.st, c.s));
+                               c.P->eps, c.L.tr_part, c.L.gram_part, nullptr, c.L.st, c.s,
+                               c.L.XT, c.L.ldxt));
     return launch_finalize(mode, epilogue_blocks(c.n), c.k, c.L.tr_part, c.L.gram_part, c.L.st,
                            c.P->rel_tol, max_evals, c.L.hist, c.L.hist_cap, c.s);
 }
@@ -296,7 +375,7 @@ static int run_full(FitCtx& c, int max_evals, HostState* hs) {
     const int iters_begin = c.iters;
     const int check = c.P->check_every;
     for (int launched = 0;; ++launched) {
-        SYMNMF_TRY(full_pass(c, MODE_FULL, max_evals));
+        SYMNMF_TRY(full_pass(c, MODE_FULL, max_evals, true));
         c.cur ^= 1;
         if ((launched + 1) % check == 0 || t_begin + launched + 1 >= max_evals) {
             SYMNMF_TRY(read_state(c.L.st, hs, c.s));
@@ -334,7 +413,7 @@ static int run_svrg(FitCtx& c, int max_evals, HostState* hs, int64_t* block_fina
     std::vector<int64_t> perm;
     for (int e = 0;; ++e) {
         // snapshot: P~ = S H~, f(H~), stopping test on consecutive evaluations
-        SYMNMF_TRY(full_pass(c, MODE_SNAPSHOT, max_evals));
+        SYMNMF_TRY(full_pass(c, MODE_SNAPSHOT, max_evals, false));
         SYMNMF_TRY(read_state(c.L.st, hs, c.s));
         SYMNMF_TRY(c.tm.harvest());
         if (hs->nonfinite || hs->converged) break;
@@ -346,7 +425,8 @@ static int run_svrg(FitCtx& c, int max_evals, HostState* hs, int64_t* block_fina
             // grown to the full gradient: take the step from the stored P~, then full batch
             SYMNMF_TRY(launch_epilogue(MODE_STEP_SNAP, n, c.k, nullptr, 0, c.Hb[c.cur], c.Gb[c.cur],
                                        c.Hb[c.cur ^ 1], c.Gb[c.cur ^ 1], c.L.Psnap, 0.f, c.P->lr,
-                                       c.P->eps, c.L.tr_part, c.L.gram_part, nullptr, c.L.st, c.s));
+                                       c.P->eps, c.L.tr_part, c.L.gram_part, nullptr, c.L.st, c.s,
+                                       c.L.XT, c.L.ldxt));
             SYMNMF_TRY(launch_finalize(MODE_STEP_SNAP, epilogue_blocks(n), c.k, c.L.tr_part,
                                        c.L.gram_part, c.L.st, c.P->rel_tol, max_evals, c.L.hist,
                                        c.L.hist_cap, c.s));
@@ -361,12 +441,10 @@ static int run_svrg(FitCtx& c, int max_evals, HostState* hs, int64_t* block_fina
                                         cudaMemcpyDeviceToDevice, c.s));
         for (int64_t q = 0; q < m; ++q) {
             const int64_t r0 = perm[q] * b, r1 = std::min(n, r0 + b);
-            StreamPlan sp = plan_stream(c.d, n, c.k, r0, r1);
-            SYMNMF_TRY(c.tm.begin(c.s));
-            SYMNMF_TRY(launch_stream_partial(sp, c.S, c.lds, c.Hb[c.cur], c.L.Hsnap, c.k, c.L.part,
-                                             c.L.st, c.s));
-            SYMNMF_TRY(c.tm.end(c.s));
-            SYMNMF_TRY(launch_epilogue(MODE_SVRG_INNER, n, c.k, c.L.part, sp.splits, c.Hb[c.cur],
+            int splits = 0;
+            SYMNMF_TRY(stream_product(c.d, c.args(), c.Hb[c.cur], c.L.Hsnap, c.k, r0, r1, false,
+                                      c.s, &splits, &c.tm));
+            SYMNMF_TRY(launch_epilogue(MODE_SVRG_INNER, n, c.k, c.L.part, splits, c.Hb[c.cur],
                                        c.Gb[c.cur], c.Hb[c.cur ^ 1], c.Gb[c.cur ^ 1], c.L.Psnap,
                                        (float)m, c.P->lr, c.P->eps, c.L.tr_part, c.L.gram_part,
                                        nullptr, c.L.st, c.s));
@@ -443,9 +521,11 @@ static int fit_impl(const float* S, int64_t n, int64_t lds, int k, const symnmf_
                                         cudaMemcpyDeviceToDevice, s));
     else
         SYMNMF_CUDA_TRY(cudaMemsetAsync(c.L.G0, 0, (size_t)n * k * sizeof(float), s));
-    // Gram of H0
+    // Gram of H0 (also writes the split operand of H0; its padding rows stay zero)
+    SYMNMF_CUDA_TRY(cudaMemsetAsync(c.L.XT, 0, (size_t)xt_rows(k) * c.L.ldxt * sizeof(float), s));
     SYMNMF_TRY(launch_epilogue(MODE_GRAM, n, k, nullptr, 0, H, nullptr, nullptr, nullptr, nullptr,
-                               0.f, 0.f, 0.f, c.L.tr_part, c.L.gram_part, nullptr, c.L.st, s));
+                               0.f, 0.f, 0.f, c.L.tr_part, c.L.gram_part, nullptr, c.L.st, s,
+                               c.L.XT, c.L.ldxt));
     SYMNMF_TRY(launch_finalize(MODE_GRAM, epilogue_blocks(n), k, c.L.tr_part, c.L.gram_part,
                                c.L.st, P.rel_tol, P.max_iters + 1, c.L.hist, c.L.hist_cap, s));
 
@@ -485,6 +565,14 @@ static int fit_impl(const float* S, int64_t n, int64_t lds, int k, const symnmf_
                                         sizeof(double) * std::min(evals, P.loss_history_len),
                                         cudaMemcpyDeviceToHost, s));
     SYMNMF_CUDA_TRY(cudaStreamSynchronize(s));
+    {
+        int kerr = 0;
+        SYMNMF_CUDA_TRY(cudaMemcpy(&kerr, &c.L.st->kerr, sizeof(int), cudaMemcpyDeviceToHost));
+        if (kerr != 0) {
+            set_error("an S-stream pipeline wait timed out on the device (code %d)", kerr);
+            return SYMNMF_ERR_TIMEOUT;
+        }
+    }
     if (hs.nonfinite) {
         set_error("the loss became non-finite at evaluation %d", hs.t_stop);
         return SYMNMF_ERR_NONFINITE;
@@ -686,7 +774,17 @@ static int probe_impl(const Dev& d, const float* S, int64_t n, int64_t lds, int 
     const int mtot = L.mtot;
     const int64_t ldq = mtot;
     const int steps = mtot / b;  // blocks the basis can hold
-    StreamPlan sp = plan_stream(d, n, b, 0, n);
+    StreamArgs sa;
+    sa.S = S;
+    sa.n = n;
+    sa.lds = lds;
+    sa.k = b;
+    sa.part = L.part;
+    sa.XT = L.XT;
+    sa.ldxt = L.ldxt;
+    sa.err = L.err;
+    sa.st = nullptr;
+    SYMNMF_CUDA_TRY(cudaMemsetAsync(L.err, 0, sizeof(int), s));
     std::vector<double> T((size_t)mtot * mtot, 0.0), B, coef, theta, prev;
     // start block: seeded uniform noise, orthonormalised
     SYMNMF_TRY(launch_uniform_fill(L.W, n * (int64_t)b, seed, -0.5f, s));
@@ -698,9 +796,10 @@ static int probe_impl(const Dev& d, const float* S, int64_t n, int64_t lds, int 
     int have = 0;  // columns of T resolved
     for (int j = 0; j < steps; ++j) {
         // W = S Q_j (one S pass)
-        SYMNMF_TRY(launch_stream_partial(sp, S, lds, L.Q + (size_t)j * b, nullptr, ldq, L.part,
-                                         nullptr, s));
-        SYMNMF_TRY(launch_epilogue(MODE_PRODUCT, n, b, L.part, sp.splits, nullptr, nullptr, nullptr,
+        int splits = 0;
+        SYMNMF_TRY(stream_product(d, sa, L.Q + (size_t)j * b, nullptr, ldq, 0, n, false, s,
+                                  &splits, nullptr));
+        SYMNMF_TRY(launch_epilogue(MODE_PRODUCT, n, b, L.part, splits, nullptr, nullptr, nullptr,
                                    nullptr, nullptr, 0.f, 0.f, 0.f, nullptr, nullptr, L.W, nullptr,
                                    s));
         // full reorthogonalisation against Q_0..Q_j, twice; the Q_j coefficients are A_j
@@ -742,6 +841,15 @@ static int probe_impl(const Dev& d, const float* S, int64_t n, int64_t lds, int 
             }
     }
     (void)have;
+    {
+        int kerr = 0;
+        SYMNMF_CUDA_TRY(cudaMemcpyAsync(&kerr, L.err, sizeof(int), cudaMemcpyDeviceToHost, s));
+        SYMNMF_CUDA_TRY(cudaStreamSynchronize(s));
+        if (kerr != 0) {
+            set_error("an S-stream pipeline wait timed out on the device (code %d)", kerr);
+            return SYMNMF_ERR_TIMEOUT;
+        }
+    }
     if (theta.empty()) {
         set_error("spectral probe: basis of %d vectors is smaller than n_eig = %d", mtot, n_eig);
         return SYMNMF_ERR_INVALID_ARG;
@@ -854,7 +962,9 @@ int symnmf_workspace_size(int op, int64_t n, int k, int64_t T, const symnmf_fit_
         }
         case SYMNMF_OP_SH: {
             SYMNMF_CHECK_ARG(k >= 1 && k <= KMAX, "k must be in [1, 64]");
-            a.take<float>(stream_partial_floats(plan_stream(d, n, k, 0, n)));
+            a.take<float>(stream_partials(d, n, k, 0, n));
+            a.take<float>((size_t)xt_rows(k) * xt_ld(n));
+            a.take<int>(64);
             break;
         }
         case SYMNMF_OP_STATS:
@@ -959,18 +1069,28 @@ int symnmf_sh(const float* S, int64_t n, int64_t lds, const float* X, int k, flo
     SYMNMF_TRY(check_ws(ws, ws_bytes));
     Dev d;
     SYMNMF_TRY(device_info(&d));
-    StreamPlan sp = plan_stream(d, n, k, 0, n);
     Arena a;
     a.base = static_cast<char*>(ws);
     a.cap = ws_bytes;
-    float* part = a.take<float>(stream_partial_floats(sp));
+    StreamArgs sa;
+    sa.S = S;
+    sa.n = n;
+    sa.lds = lds;
+    sa.k = k;
+    sa.part = a.take<float>(stream_partials(d, n, k, 0, n));
+    sa.ldxt = xt_ld(n);
+    sa.XT = a.take<float>((size_t)xt_rows(k) * sa.ldxt);
+    sa.err = a.take<int>(64);
+    sa.st = nullptr;
     if (!a.ok()) {
         set_error("workspace too small: %zu given, %zu needed", ws_bytes, a.used);
         return SYMNMF_ERR_WORKSPACE;
     }
     cudaStream_t s = (cudaStream_t)stream;
-    SYMNMF_TRY(launch_stream_partial(sp, S, lds, X, nullptr, k, part, nullptr, s));
-    return launch_epilogue(MODE_PRODUCT, n, k, part, sp.splits, nullptr, nullptr, nullptr, nullptr,
+    SYMNMF_CUDA_TRY(cudaMemsetAsync(sa.err, 0, sizeof(int), s));
+    int splits = 0;
+    SYMNMF_TRY(stream_product(d, sa, X, nullptr, k, 0, n, false, s, &splits, nullptr));
+    return launch_epilogue(MODE_PRODUCT, n, k, sa.part, splits, nullptr, nullptr, nullptr, nullptr,
                            nullptr, 0.f, 0.f, 0.f, nullptr, nullptr, Y, nullptr, s);
 }
 

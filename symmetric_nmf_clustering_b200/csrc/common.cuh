@@ -85,7 +85,7 @@ struct FitState {
     int done;                          // 1: stop issued (no further work)
     int converged;
     int nonfinite;
-    int pad_;
+    int kerr;                          // device-side error code (bounded wait gave up)
 };
 
 // Epilogue / finalise modes.
@@ -121,12 +121,32 @@ int launch_stream_partial(const StreamPlan& p, const float* S, int64_t lds,
                           const FitState* st, cudaStream_t s);
 size_t fit_state_bytes();
 
+// Tensor-core S-stream (stream_tc.cu): X enters as its exact TF32 split
+// XT = [X_hi; X_lo] stored K-major (2*K16 rows of length ldxt, K16 = k rounded up to 16).
+struct TcPlan {
+    int64_t n;
+    int k, K16;
+    int64_t j0, j1;   // contraction range, j0 a multiple of 32
+    int64_t tiles;    // 128-row tiles of the output
+    int splits;       // contraction splits
+    int64_t jspan;    // columns per split (multiple of 32)
+};
+TcPlan plan_stream_tc(const Dev& d, int64_t n, int k, int64_t j0, int64_t j1);
+size_t tc_partial_floats(const TcPlan& p);
+int launch_stream_tc(const TcPlan& p, const float* S, int64_t lds, const float* XT, int64_t ldxt,
+                     float* part, int* err, const FitState* st, cudaStream_t s);
+int launch_split(const float* Xa, const float* Xb, int64_t ldx, int k, int64_t r0, int64_t r1,
+                 int64_t jlo, int64_t jhi, float* XT, int64_t ldxt, cudaStream_t s);
+inline int64_t xt_ld(int64_t n) { return (n + 31) / 32 * 32; }
+inline int xt_rows(int k) { return 2 * ((k + 15) / 16 * 16); }
+
 int epilogue_blocks(int64_t n);
 int launch_epilogue(int mode, int64_t n, int k, const float* part, int splits,
                     const float* H, const float* G, float* Hn, float* Gn,
                     float* Psnap, float m_scale, float lr, float eps,
                     double* tr_part, double* gram_part, float* Y,
-                    const FitState* st, cudaStream_t s);
+                    const FitState* st, cudaStream_t s, float* XT = nullptr,
+                    int64_t ldxt = 0);
 int launch_finalize(int mode, int nblk, int k, const double* tr_part,
                     const double* gram_part, FitState* st, double rel_tol,
                     int max_evals, double* history, int history_cap,

@@ -195,7 +195,7 @@ epilogue_kernel(int mode, int64_t n, int k, const float* __restrict__ part, int 
                 float* __restrict__ Hn, float* __restrict__ Gn, float* __restrict__ Psnap,
                 float m_scale, float lr, float eps, double* __restrict__ tr_part,
                 double* __restrict__ gram_part, float* __restrict__ Y,
-                const FitState* st) {
+                const FitState* st, float* __restrict__ XT, int64_t ldxt) {
     if (st != nullptr && st->done) return;
     // As (k x k Gram, used by the step) and hs (new rows, used by the Gram
     // partial) are live at different times and share one buffer.
@@ -288,6 +288,19 @@ epilogue_kernel(int mode, int64_t n, int k, const float* __restrict__ part, int 
         for (int c = 0; c < KE; ++c) h[c] = hnew[c];
     }
 
+    // exact TF32 split [h_hi; h_lo] of the rows in h, the next S-stream's operand
+    if (XT != nullptr && valid && (mode == MODE_FULL || mode == MODE_STEP_SNAP || mode == MODE_GRAM)) {
+        const int K16 = (k + 15) / 16 * 16;
+#pragma unroll
+        for (int c = 0; c < KE; ++c) {
+            if (c < k) {
+                const float hb = __uint_as_float(__float_as_uint(h[c]) & 0xFFFFE000u);
+                XT[(int64_t)c * ldxt + i] = hb;
+                XT[(int64_t)(K16 + c) * ldxt + i] = h[c] - hb;
+            }
+        }
+    }
+
     // Gram partial of the rows now in h (new iterate, or the given H for MODE_GRAM)
     __syncthreads();  // every thread is done reading As
 #pragma unroll
@@ -307,12 +320,12 @@ int launch_epilogue(int mode, int64_t n, int k, const float* part, int splits,
                     const float* H, const float* G, float* Hn, float* Gn,
                     float* Psnap, float m_scale, float lr, float eps,
                     double* tr_part, double* gram_part, float* Y,
-                    const FitState* st, cudaStream_t s) {
+                    const FitState* st, cudaStream_t s, float* XT, int64_t ldxt) {
     const int nb = epilogue_blocks(n);
 #define SYMNMF_EP(KE)                                                                 \
     epilogue_kernel<KE><<<nb, EP_ROWS, 0, s>>>(mode, n, k, part, splits, H, G, Hn, Gn, \
                                                Psnap, m_scale, lr, eps, tr_part,       \
-                                               gram_part, Y, st)
+                                               gram_part, Y, st, XT, ldxt)
     if (k <= 8) SYMNMF_EP(8);
     else if (k <= 16) SYMNMF_EP(16);
     else if (k <= 24) SYMNMF_EP(24);

@@ -1,0 +1,362 @@
+// Tensor-core S-stream: part[s] = S[:, J_s] X[J_s, :] on the 5th-generation
+// tensor cores (tcgen05), fp32-accurate through an exact TF32 split.
+//
+// The pages' hot spot is the S H product that streams S once per iteration
+// ([CaS] "Factorization at scale": the dominant S H multiplications).  At
+// k = 24 that is 12 flop per byte of S: more fp32 FMA than the CUDA cores
+// can issue at HBM speed, so the contraction runs on the tensor cores while
+// the kernel stays bound by the HBM read of S.
+//
+// Accuracy.  TF32 keeps 10 explicit mantissa bits.  Every fp32 value is split
+// exactly as x = hi + lo with hi = x with its low 13 mantissa bits cleared and
+// lo = x - hi (exact, at most 13 significant bits), and
+//     S X = S_hi X_hi + S_hi X_lo + S_lo X_hi + O(2^-22 |S| |X|),
+// accumulated in fp32 in TMEM.  hi is a TF32 number, so the product does not
+// depend on how the tensor core converts fp32 operands.
+//
+// Per CTA (256 threads, two CTAs per SM): a 128-row tile of S times the
+// contraction range of its split, in stages of 32 columns (128 bytes):
+//   warp 0      TMA producer: S tile (128 x 32, 128-byte swizzle) and the
+//               matching [X_hi; X_lo] tile (2*K16 x 32, K-major) per stage,
+//               K16 = k rounded up to 16 (an MMA with M = 128 and A in TMEM
+//               needs N to be a multiple of 16)
+//   warp 1      MMA issuer: per 8-column step, D[:, 0:2K16] += S_hi [X_hi;X_lo]
+//               and D[:, 0:K16] += S_lo X_hi, A operands read from TMEM
+//   warp 2      TMEM allocator
+//   warps 4-7   split warps: thread r reads row r of the S tile from shared
+//               memory, stores its hi and lo planes into TMEM lane r, and at
+//               the end reads D back and writes the partial row
+#include <cudaTypedefs.h>
+
+#include "common.cuh"
+#include "sm100.cuh"
+
+namespace symnmf {
+
+constexpr int TC_BM = 128;                  // S rows per tile = TMEM lanes
+constexpr int TC_BK = 32;                   // columns per stage (128 bytes of fp32)
+constexpr int TC_NS = 4;                    // shared-memory stages
+constexpr int TC_NT = 2;                    // TMEM stages of the split S tile
+constexpr int TC_THREADS = 256;
+constexpr uint32_t TC_TMEM_COLS = 256;
+constexpr uint32_t TC_A_BYTES = TC_BM * TC_BK * 4;
+constexpr uint32_t TC_COL_A = 128;          // TMEM column of the first S stage (D below)
+
+template <int K16>
+struct TcCfg {
+    static constexpr int N1 = 2 * K16;                       // [X_hi ; X_lo]
+    static constexpr int N2 = K16;                           // X_hi
+    static constexpr uint32_t B_BYTES = N1 * TC_BK * 4;     // multiple of 1024
+    static constexpr uint32_t STAGE = TC_A_BYTES + B_BYTES;
+    static constexpr uint32_t SMEM = TC_NS * STAGE + 1024;  // + alignment slack
+};
+
+__device__ __forceinline__ void tc_fail(int* err, volatile int* abort_flag, int code) {
+    *abort_flag = 1;
+    if (err != nullptr) atomicExch(err, code);
+}
+
+template <int K16>
+__global__ void __launch_bounds__(TC_THREADS, 1)
+stream_tc_kernel(const __grid_constant__ CUtensorMap mapS, const __grid_constant__ CUtensorMap mapX,
+                 int64_t n, int k, int64_t j0, int64_t j1, int64_t jspan,
+                 float* __restrict__ part, int* __restrict__ err, const FitState* st) {
+    using Cfg = TcCfg<K16>;
+    using namespace sm100;
+    if (st != nullptr && st->done) return;
+
+    extern __shared__ uint8_t tc_smem_raw[];
+    __shared__ __align__(8) uint64_t bar_full[TC_NS], bar_empty[TC_NS];
+    __shared__ __align__(8) uint64_t bar_tfull[TC_NT], bar_tempty[TC_NT], bar_acc;
+    __shared__ uint32_t tmem_base_sh;
+    __shared__ volatile int abort_sh;
+
+    uint8_t* smem = reinterpret_cast<uint8_t*>(
+        (reinterpret_cast<uintptr_t>(tc_smem_raw) + 1023) & ~uintptr_t(1023));
+    uint8_t* smemA = smem;                                // [NS][128 rows][128 B]
+    uint8_t* smemB = smem + TC_NS * TC_A_BYTES;           // [NS][N1 rows][128 B]
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int64_t i0 = (int64_t)blockIdx.x * TC_BM;
+    const int split = blockIdx.y;
+    const int64_t jb = j0 + (int64_t)split * jspan;
+    const int64_t je = min64(j1, jb + jspan);
+    const int ksteps = jb < je ? (int)((je - jb + TC_BK - 1) / TC_BK) : 0;
+
+    if (tid == 0) {
+        for (int s = 0; s < TC_NS; ++s) {
+            mbar_init(&bar_full[s], 1);
+            mbar_init(&bar_empty[s], 1);
+        }
+        for (int t = 0; t < TC_NT; ++t) {
+            mbar_init(&bar_tfull[t], 4);   // one arrival per split warp
+            mbar_init(&bar_tempty[t], 1);
+        }
+        mbar_init(&bar_acc, 1);
+        abort_sh = 0;
+        fence_mbar_init();
+        prefetch_tmap(&mapS);
+        prefetch_tmap(&mapX);
+    }
+    if (warp == 2) {
+        tmem_alloc(&tmem_base_sh, TC_TMEM_COLS);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tbase = tmem_base_sh;
+
+    if (warp == 0 && lane == 0 && ksteps > 0) {
+        // ---------------- TMA producer
+        int issued = 0;
+        for (int s = 0; s < ksteps; ++s) {
+            if (abort_sh) break;
+            const int slot = s % TC_NS;
+            const uint32_t ph = (uint32_t)(s / TC_NS) & 1u;
+            if (s >= TC_NS && !mbar_wait(&bar_empty[slot], ph ^ 1u)) {
+                tc_fail(err, &abort_sh, 1);
+                break;
+            }
+            mbar_arrive_expect_tx(&bar_full[slot], Cfg::STAGE);
+            const int32_t x = (int32_t)(jb + (int64_t)s * TC_BK);
+            tma_load_2d(smemA + slot * TC_A_BYTES, &mapS, x, (int32_t)i0, &bar_full[slot]);
+            tma_load_2d(smemB + slot * Cfg::B_BYTES, &mapX, x, 0, &bar_full[slot]);
+            ++issued;
+        }
+        if (abort_sh) {  // let the copies already issued land before the CTA exits
+            for (int s = max(0, issued - TC_NS); s < issued; ++s)
+                mbar_wait(&bar_full[s % TC_NS], (uint32_t)(s / TC_NS) & 1u);
+        }
+    } else if (warp == 1 && lane == 0 && ksteps > 0) {
+        // ---------------- MMA issuer
+        constexpr uint32_t id1 = idesc_tf32(TC_BM, Cfg::N1);
+        constexpr uint32_t id2 = idesc_tf32(TC_BM, Cfg::N2);
+        for (int s = 0; s < ksteps; ++s) {
+            if (abort_sh) break;
+            const int slot = s % TC_NS;
+            const uint32_t ph = (uint32_t)(s / TC_NS) & 1u;
+            const int ts = s % TC_NT;
+            const uint32_t tph = (uint32_t)(s / TC_NT) & 1u;
+            if (!mbar_wait(&bar_tfull[ts], tph) || !mbar_wait(&bar_full[slot], ph)) {
+                tc_fail(err, &abort_sh, 2);
+                break;
+            }
+            tc_fence_after();
+            const uint32_t b_base = smem_u32(smemB + slot * Cfg::B_BYTES);
+            const uint32_t a_hi = tbase + TC_COL_A + (uint32_t)ts * 64u;
+#pragma unroll
+            for (int kk = 0; kk < TC_BK / 8; ++kk) {
+                const uint64_t bd = umma_desc_sw128(b_base + (uint32_t)kk * 32u);
+                umma_tf32_ts(tbase, a_hi + (uint32_t)kk * 8u, bd, id1, (s | kk) ? 1u : 0u);
+                umma_tf32_ts(tbase, a_hi + 32u + (uint32_t)kk * 8u, bd, id2, 1u);
+            }
+            umma_commit(&bar_empty[slot]);
+            umma_commit(&bar_tempty[ts]);
+        }
+        umma_commit(&bar_acc);
+        if (abort_sh) mbar_wait(&bar_acc, 0);  // MMAs in flight finish before TMEM is freed
+    } else if (warp >= 4) {
+        // ---------------- split warps (TMEM lane quarter = warp % 4)
+        const int wl = warp & 3;
+        const int r = wl * 32 + lane;
+        const uint32_t lane_off = (uint32_t)(wl * 32) << 16;
+        // control flow stays warp-uniform: tcgen05.st/ld are .sync.aligned
+        for (int s = 0; s < ksteps; ++s) {
+            if (__any_sync(0xffffffffu, abort_sh != 0)) break;
+            const int slot = s % TC_NS;
+            const uint32_t ph = (uint32_t)(s / TC_NS) & 1u;
+            const int ts = s % TC_NT;
+            const uint32_t tph = (uint32_t)(s / TC_NT) & 1u;
+            const bool ok = mbar_wait(&bar_full[slot], ph) &&
+                            (s < TC_NT || mbar_wait(&bar_tempty[ts], tph ^ 1u));
+            if (!__all_sync(0xffffffffu, ok)) {
+                if (lane == 0) tc_fail(err, &abort_sh, 3);
+                break;
+            }
+            const uint8_t* rowp = smemA + slot * TC_A_BYTES + r * 128;
+            uint32_t hi[32], lo[32];
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+                const float4 v = *reinterpret_cast<const float4*>(rowp + ((c ^ (r & 7)) << 4));
+                const float e[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const uint32_t hb = __float_as_uint(e[q]) & 0xFFFFE000u;
+                    hi[c * 4 + q] = hb;
+                    lo[c * 4 + q] = __float_as_uint(e[q] - __uint_as_float(hb));
+                }
+            }
+            const uint32_t tcol = tbase + lane_off + TC_COL_A + (uint32_t)ts * 64u;
+            tmem_st_32x32b_x32(tcol, hi);
+            tmem_st_32x32b_x32(tcol + 32u, lo);
+            tmem_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bar_tfull[ts]);
+        }
+        // epilogue: D row r -> partial row i0 + r
+        const int64_t i = i0 + r;
+        float* out = part + (int64_t)split * n * k + i * (int64_t)k;
+        if (ksteps == 0) {
+            if (i < n)
+                for (int c = 0; c < k; ++c) out[c] = 0.f;
+        } else if (!__any_sync(0xffffffffu, abort_sh != 0) &&
+                   __all_sync(0xffffffffu, mbar_wait(&bar_acc, 0))) {
+            tc_fence_after();
+            // D[:, c] + D[:, K16 + c], read back 8 columns of each half at a time
+#pragma unroll
+            for (int q = 0; q < K16 / 8; ++q) {
+                uint32_t va[8], vb[8];
+                tmem_ld_32x32b_x8(tbase + lane_off + (uint32_t)q * 8u, va);
+                tmem_ld_32x32b_x8(tbase + lane_off + (uint32_t)(K16 + q * 8), vb);
+                tmem_wait_ld();
+                if (i < n) {
+#pragma unroll
+                    for (int e = 0; e < 8; ++e)
+                        if (q * 8 + e < k) out[q * 8 + e] = __uint_as_float(va[e]) + __uint_as_float(vb[e]);
+                }
+            }
+        } else if (lane == 0) {
+            tc_fail(err, &abort_sh, 4);
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 2) {
+        tc_fence_after();
+        tmem_dealloc(tbase, TC_TMEM_COLS);
+    }
+}
+
+// ----------------------------------------------------------------------------
+// [X_hi ; X_lo] in the K-major layout the MMA reads: XT[c][j] (c < K16) and
+// XT[K16 + c][j] for j in [jlo, jhi); X = Xa - Xb on rows [r0, r1) and zero
+// on the other rows of the range; rows c in [k, K16) of each half are zero.
+// ----------------------------------------------------------------------------
+__global__ void split_kernel(const float* __restrict__ Xa, const float* __restrict__ Xb,
+                             int64_t ldx, int k, int K16, int64_t r0, int64_t r1, int64_t jlo,
+                             int64_t jhi, float* __restrict__ XT, int64_t ldxt) {
+    const int64_t j = jlo + (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (j >= jhi) return;
+    const bool in = j >= r0 && j < r1;
+    for (int c = 0; c < K16; ++c) {
+        float x = 0.f;
+        if (in && c < k) {
+            x = Xa[j * ldx + c];
+            if (Xb != nullptr) x -= Xb[j * ldx + c];
+        }
+        const float h = __uint_as_float(__float_as_uint(x) & 0xFFFFE000u);
+        XT[(int64_t)c * ldxt + j] = h;
+        XT[(int64_t)(K16 + c) * ldxt + j] = x - h;
+    }
+}
+
+int launch_split(const float* Xa, const float* Xb, int64_t ldx, int k, int64_t r0, int64_t r1,
+                 int64_t jlo, int64_t jhi, float* XT, int64_t ldxt, cudaStream_t s) {
+    if (jhi <= jlo) return SYMNMF_OK;
+    const int K16 = (k + 15) / 16 * 16;
+    const int64_t len = jhi - jlo;
+    split_kernel<<<(unsigned)((len + 255) / 256), 256, 0, s>>>(Xa, Xb, ldx, k, K16, r0, r1, jlo,
+                                                              jhi, XT, ldxt);
+    SYMNMF_LAUNCH_CHECK();
+    return SYMNMF_OK;
+}
+
+// ----------------------------------------------------------------------------
+// host side
+// ----------------------------------------------------------------------------
+static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (fn == nullptr) {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+    }
+    return fn;
+}
+
+// Row-major fp32 matrix (rows x cols, row pitch `ld` elements) as a 2-D TMA
+// map with boxes of 32 columns x box_rows rows and 128-byte swizzle.
+static int make_map(CUtensorMap* m, const float* base, int64_t cols, int64_t rows, int64_t ld,
+                    uint32_t box_rows) {
+    auto fn = encode_fn();
+    if (fn == nullptr) {
+        set_error("cuTensorMapEncodeTiled is not available from the driver");
+        return SYMNMF_ERR_NOT_SUPPORTED;
+    }
+    cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)ld * sizeof(float)};
+    cuuint32_t box[2] = {(cuuint32_t)TC_BK, box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(base), dims, strides,
+                    box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) {
+        set_error("cuTensorMapEncodeTiled failed (%d)", (int)r);
+        return SYMNMF_ERR_CUDA;
+    }
+    return SYMNMF_OK;
+}
+
+TcPlan plan_stream_tc(const Dev& d, int64_t n, int k, int64_t j0, int64_t j1) {
+    TcPlan p;
+    p.n = n;
+    p.k = k;
+    p.K16 = (k + 15) / 16 * 16;
+    p.j0 = j0 / TC_BK * TC_BK;                                 // 128-byte aligned TMA x
+    p.j1 = std::min<int64_t>(n, (j1 + TC_BK - 1) / TC_BK * TC_BK);
+    p.tiles = (n + TC_BM - 1) / TC_BM;
+    const int64_t steps = std::max<int64_t>(1, (p.j1 - p.j0 + TC_BK - 1) / TC_BK);
+    const int64_t slots = (int64_t)d.sms * 2;                  // two CTAs per SM
+    // contraction splits: fill whole waves of resident CTAs, >= 8 stages each
+    int best = 1;
+    double best_waste = 1e30;
+    for (int s = 1; s <= 32; ++s) {
+        if (s > 1 && steps / s < 8) break;
+        const int64_t ctas = p.tiles * s;
+        const int64_t waves = (ctas + slots - 1) / slots;
+        const double waste = (double)(waves * slots) / (double)ctas - 1.0 + 0.002 * s;
+        if (waste < best_waste - 1e-12) {
+            best_waste = waste;
+            best = s;
+        }
+    }
+    p.splits = best;
+    const int64_t per = (steps + best - 1) / best;
+    p.jspan = per * TC_BK;
+    return p;
+}
+
+size_t tc_partial_floats(const TcPlan& p) { return (size_t)p.splits * p.n * p.k; }
+
+int launch_stream_tc(const TcPlan& p, const float* S, int64_t lds, const float* XT, int64_t ldxt,
+                     float* part, int* err, const FitState* st, cudaStream_t s) {
+    CUtensorMap mapS, mapX;
+    SYMNMF_TRY(make_map(&mapS, S, p.n, p.n, lds, TC_BM));
+    SYMNMF_TRY(make_map(&mapX, XT, p.n, 2 * p.K16, ldxt, (uint32_t)(2 * p.K16)));
+    dim3 grid((unsigned)p.tiles, (unsigned)p.splits);
+#define SYMNMF_TC(K16)                                                                         \
+    do {                                                                                      \
+        auto kern = stream_tc_kernel<K16>;                                                     \
+        SYMNMF_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, \
+                                             (int)TcCfg<K16>::SMEM));                          \
+        kern<<<grid, TC_THREADS, TcCfg<K16>::SMEM, s>>>(mapS, mapX, p.n, p.k, p.j0, p.j1,      \
+                                                       p.jspan, part, err, st);               \
+    } while (0)
+    switch (p.K16) {
+        case 16: SYMNMF_TC(16); break;
+        case 32: SYMNMF_TC(32); break;
+        case 48: SYMNMF_TC(48); break;
+        default: SYMNMF_TC(64); break;
+    }
+#undef SYMNMF_TC
+    SYMNMF_LAUNCH_CHECK();
+    return SYMNMF_OK;
+}
+
+}  // namespace symnmf
