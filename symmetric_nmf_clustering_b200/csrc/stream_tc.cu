@@ -37,18 +37,24 @@ constexpr int TC_BM = 128;                  // S rows per tile = TMEM lanes
 constexpr int TC_BK = 32;                   // columns per stage (128 bytes of fp32)
 constexpr int TC_NS = 4;                    // shared-memory stages
 constexpr int TC_NT = 2;                    // TMEM stages of the split S tile
+constexpr int TC_CHUNK = 4;                 // stages accumulated in TMEM before a drain
 constexpr int TC_THREADS = 256;
-constexpr uint32_t TC_TMEM_COLS = 256;
 constexpr uint32_t TC_A_BYTES = TC_BM * TC_BK * 4;
-constexpr uint32_t TC_COL_A = 128;          // TMEM column of the first S stage (D below)
 
+// TMEM columns: two accumulators D0, D1 of 2*K16 columns each, then the
+// TC_NT stages of the split S tile (32 hi + 32 lo columns each).
 template <int K16>
 struct TcCfg {
-    static constexpr int N1 = 2 * K16;                       // [X_hi ; X_lo]
-    static constexpr int N2 = K16;                           // X_hi
+    static constexpr int N1 = 2 * K16;                      // [X_hi ; X_lo]
+    static constexpr int N2 = K16;                          // X_hi
     static constexpr uint32_t B_BYTES = N1 * TC_BK * 4;     // multiple of 1024
     static constexpr uint32_t STAGE = TC_A_BYTES + B_BYTES;
-    static constexpr uint32_t SMEM = TC_NS * STAGE + 1024;  // + alignment slack
+    static constexpr uint32_t COL_A = 4 * K16 <= 128 ? 128u : 256u;
+    static constexpr uint32_t TMEM_COLS = COL_A + TC_NT * 64 <= 256 ? 256u : 512u;
+    // with 512 TMEM columns only one CTA may be resident: ask for enough smem
+    static constexpr uint32_t SMEM_MIN = TMEM_COLS == 512u ? 120u * 1024u : 0u;
+    static constexpr uint32_t SMEM_RAW = TC_NS * STAGE + 1024;
+    static constexpr uint32_t SMEM = SMEM_RAW > SMEM_MIN ? SMEM_RAW : SMEM_MIN;
 };
 
 __device__ __forceinline__ void tc_fail(int* err, volatile int* abort_flag, int code) {
@@ -67,7 +73,8 @@ stream_tc_kernel(const __grid_constant__ CUtensorMap mapS, const __grid_constant
 
     extern __shared__ uint8_t tc_smem_raw[];
     __shared__ __align__(8) uint64_t bar_full[TC_NS], bar_empty[TC_NS];
-    __shared__ __align__(8) uint64_t bar_tfull[TC_NT], bar_tempty[TC_NT], bar_acc;
+    __shared__ __align__(8) uint64_t bar_tfull[TC_NT], bar_tempty[TC_NT];
+    __shared__ __align__(8) uint64_t bar_dfull[2], bar_dempty[2], bar_fin;
     __shared__ uint32_t tmem_base_sh;
     __shared__ volatile int abort_sh;
 
@@ -82,6 +89,7 @@ stream_tc_kernel(const __grid_constant__ CUtensorMap mapS, const __grid_constant
     const int64_t jb = j0 + (int64_t)split * jspan;
     const int64_t je = min64(j1, jb + jspan);
     const int ksteps = jb < je ? (int)((je - jb + TC_BK - 1) / TC_BK) : 0;
+    const int nchunks = (ksteps + TC_CHUNK - 1) / TC_CHUNK;
 
     if (tid == 0) {
         for (int s = 0; s < TC_NS; ++s) {
@@ -92,14 +100,18 @@ stream_tc_kernel(const __grid_constant__ CUtensorMap mapS, const __grid_constant
             mbar_init(&bar_tfull[t], 4);   // one arrival per split warp
             mbar_init(&bar_tempty[t], 1);
         }
-        mbar_init(&bar_acc, 1);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&bar_dfull[b], 1);
+            mbar_init(&bar_dempty[b], 4);  // one arrival per split warp
+        }
+        mbar_init(&bar_fin, 1);
         abort_sh = 0;
         fence_mbar_init();
         prefetch_tmap(&mapS);
         prefetch_tmap(&mapX);
     }
     if (warp == 2) {
-        tmem_alloc(&tmem_base_sh, TC_TMEM_COLS);
+        tmem_alloc(&tmem_base_sh, Cfg::TMEM_COLS);
         tmem_relinquish();
     }
     tc_fence_before();
@@ -129,7 +141,7 @@ stream_tc_kernel(const __grid_constant__ CUtensorMap mapS, const __grid_constant
                 mbar_wait(&bar_full[s % TC_NS], (uint32_t)(s / TC_NS) & 1u);
         }
     } else if (warp == 1 && lane == 0 && ksteps > 0) {
-        // ---------------- MMA issuer
+        // ---------------- MMA issuer: chunk q accumulates into D[q % 2]
         constexpr uint32_t id1 = idesc_tf32(TC_BM, Cfg::N1);
         constexpr uint32_t id2 = idesc_tf32(TC_BM, Cfg::N2);
         for (int s = 0; s < ksteps; ++s) {
@@ -138,32 +150,72 @@ stream_tc_kernel(const __grid_constant__ CUtensorMap mapS, const __grid_constant
             const uint32_t ph = (uint32_t)(s / TC_NS) & 1u;
             const int ts = s % TC_NT;
             const uint32_t tph = (uint32_t)(s / TC_NT) & 1u;
-            if (!mbar_wait(&bar_tfull[ts], tph) || !mbar_wait(&bar_full[slot], ph)) {
+            const int q = s / TC_CHUNK, b = q & 1;
+            const bool first = (s % TC_CHUNK) == 0;
+            const bool last = (s % TC_CHUNK) == TC_CHUNK - 1 || s == ksteps - 1;
+            bool ok = mbar_wait(&bar_tfull[ts], tph) && mbar_wait(&bar_full[slot], ph);
+            if (ok && first && q >= 2) ok = mbar_wait(&bar_dempty[b], (uint32_t)((q >> 1) - 1) & 1u);
+            if (!ok) {
                 tc_fail(err, &abort_sh, 2);
                 break;
             }
             tc_fence_after();
             const uint32_t b_base = smem_u32(smemB + slot * Cfg::B_BYTES);
-            const uint32_t a_hi = tbase + TC_COL_A + (uint32_t)ts * 64u;
+            const uint32_t a_hi = tbase + Cfg::COL_A + (uint32_t)ts * 64u;
+            const uint32_t d = tbase + (uint32_t)b * (uint32_t)Cfg::N1;
 #pragma unroll
             for (int kk = 0; kk < TC_BK / 8; ++kk) {
                 const uint64_t bd = umma_desc_sw128(b_base + (uint32_t)kk * 32u);
-                umma_tf32_ts(tbase, a_hi + (uint32_t)kk * 8u, bd, id1, (s | kk) ? 1u : 0u);
-                umma_tf32_ts(tbase, a_hi + 32u + (uint32_t)kk * 8u, bd, id2, 1u);
+                umma_tf32_ts(d, a_hi + (uint32_t)kk * 8u, bd, id1, (first && kk == 0) ? 0u : 1u);
+                umma_tf32_ts(d, a_hi + 32u + (uint32_t)kk * 8u, bd, id2, 1u);
             }
             umma_commit(&bar_empty[slot]);
             umma_commit(&bar_tempty[ts]);
+            if (last) umma_commit(&bar_dfull[b]);
         }
-        umma_commit(&bar_acc);
-        if (abort_sh) mbar_wait(&bar_acc, 0);  // MMAs in flight finish before TMEM is freed
+        if (abort_sh) {  // MMAs in flight finish before TMEM is freed
+            umma_commit(&bar_fin);
+            mbar_wait(&bar_fin, 0);
+        }
     } else if (warp >= 4) {
         // ---------------- split warps (TMEM lane quarter = warp % 4)
         const int wl = warp & 3;
         const int r = wl * 32 + lane;
         const uint32_t lane_off = (uint32_t)(wl * 32) << 16;
+        float acc[K16];
+#pragma unroll
+        for (int c = 0; c < K16; ++c) acc[c] = 0.f;
+        bool alive = true;
+
+        // fold accumulator D[q % 2] into acc (round-to-nearest fp32 adds)
+        auto drain = [&](int q) -> bool {
+            const int b = q & 1;
+            if (!__all_sync(0xffffffffu, mbar_wait(&bar_dfull[b], (uint32_t)(q >> 1) & 1u)))
+                return false;
+            tc_fence_after();
+            const uint32_t dcol = tbase + lane_off + (uint32_t)b * (uint32_t)Cfg::N1;
+#pragma unroll
+            for (int g = 0; g < K16 / 8; ++g) {
+                uint32_t va[8], vb[8];
+                tmem_ld_32x32b_x8(dcol + (uint32_t)g * 8u, va);
+                tmem_ld_32x32b_x8(dcol + (uint32_t)(K16 + g * 8), vb);
+                tmem_wait_ld();
+#pragma unroll
+                for (int e = 0; e < 8; ++e)
+                    acc[g * 8 + e] += __uint_as_float(va[e]) + __uint_as_float(vb[e]);
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bar_dempty[b]);
+            return true;
+        };
+
         // control flow stays warp-uniform: tcgen05.st/ld are .sync.aligned
         for (int s = 0; s < ksteps; ++s) {
-            if (__any_sync(0xffffffffu, abort_sh != 0)) break;
+            if (__any_sync(0xffffffffu, abort_sh != 0)) {
+                alive = false;
+                break;
+            }
             const int slot = s % TC_NS;
             const uint32_t ph = (uint32_t)(s / TC_NS) & 1u;
             const int ts = s % TC_NT;
@@ -172,6 +224,7 @@ stream_tc_kernel(const __grid_constant__ CUtensorMap mapS, const __grid_constant
                             (s < TC_NT || mbar_wait(&bar_tempty[ts], tph ^ 1u));
             if (!__all_sync(0xffffffffu, ok)) {
                 if (lane == 0) tc_fail(err, &abort_sh, 3);
+                alive = false;
                 break;
             }
             const uint8_t* rowp = smemA + slot * TC_A_BYTES + r * 128;
@@ -181,44 +234,39 @@ stream_tc_kernel(const __grid_constant__ CUtensorMap mapS, const __grid_constant
                 const float4 v = *reinterpret_cast<const float4*>(rowp + ((c ^ (r & 7)) << 4));
                 const float e[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const uint32_t hb = __float_as_uint(e[q]) & 0xFFFFE000u;
-                    hi[c * 4 + q] = hb;
-                    lo[c * 4 + q] = __float_as_uint(e[q] - __uint_as_float(hb));
+                for (int u = 0; u < 4; ++u) {
+                    const uint32_t hb = __float_as_uint(e[u]) & 0xFFFFE000u;
+                    hi[c * 4 + u] = hb;
+                    lo[c * 4 + u] = __float_as_uint(e[u] - __uint_as_float(hb));
                 }
             }
-            const uint32_t tcol = tbase + lane_off + TC_COL_A + (uint32_t)ts * 64u;
+            const uint32_t tcol = tbase + lane_off + Cfg::COL_A + (uint32_t)ts * 64u;
             tmem_st_32x32b_x32(tcol, hi);
             tmem_st_32x32b_x32(tcol + 32u, lo);
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&bar_tfull[ts]);
-        }
-        // epilogue: D row r -> partial row i0 + r
-        const int64_t i = i0 + r;
-        float* out = part + (int64_t)split * n * k + i * (int64_t)k;
-        if (ksteps == 0) {
-            if (i < n)
-                for (int c = 0; c < k; ++c) out[c] = 0.f;
-        } else if (!__any_sync(0xffffffffu, abort_sh != 0) &&
-                   __all_sync(0xffffffffu, mbar_wait(&bar_acc, 0))) {
-            tc_fence_after();
-            // D[:, c] + D[:, K16 + c], read back 8 columns of each half at a time
-#pragma unroll
-            for (int q = 0; q < K16 / 8; ++q) {
-                uint32_t va[8], vb[8];
-                tmem_ld_32x32b_x8(tbase + lane_off + (uint32_t)q * 8u, va);
-                tmem_ld_32x32b_x8(tbase + lane_off + (uint32_t)(K16 + q * 8), vb);
-                tmem_wait_ld();
-                if (i < n) {
-#pragma unroll
-                    for (int e = 0; e < 8; ++e)
-                        if (q * 8 + e < k) out[q * 8 + e] = __uint_as_float(va[e]) + __uint_as_float(vb[e]);
+            // end of chunk q: fold the previous chunk, whose MMAs are done by now
+            const int q = s / TC_CHUNK;
+            if (((s % TC_CHUNK) == TC_CHUNK - 1 || s == ksteps - 1) && q >= 1) {
+                if (!drain(q - 1)) {
+                    if (lane == 0) tc_fail(err, &abort_sh, 4);
+                    alive = false;
+                    break;
                 }
             }
-        } else if (lane == 0) {
-            tc_fail(err, &abort_sh, 4);
+        }
+        if (alive && nchunks > 0 && !drain(nchunks - 1)) {
+            if (lane == 0) tc_fail(err, &abort_sh, 5);
+            alive = false;
+        }
+        const int64_t i = i0 + r;
+        if (alive && i < n) {
+            float* out = part + (int64_t)split * n * k + i * (int64_t)k;
+#pragma unroll
+            for (int c = 0; c < K16; ++c)
+                if (c < k) out[c] = acc[c];
         }
     }
 
@@ -226,7 +274,7 @@ stream_tc_kernel(const __grid_constant__ CUtensorMap mapS, const __grid_constant
     __syncthreads();
     if (warp == 2) {
         tc_fence_after();
-        tmem_dealloc(tbase, TC_TMEM_COLS);
+        tmem_dealloc(tbase, Cfg::TMEM_COLS);
     }
 }
 
