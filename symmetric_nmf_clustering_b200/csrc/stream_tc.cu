@@ -37,7 +37,7 @@ constexpr int TC_BM = 128;                  // S rows per tile = TMEM lanes
 constexpr int TC_BK = 32;                   // columns per stage (128 bytes of fp32)
 constexpr int TC_NS = 4;                    // shared-memory stages
 constexpr int TC_NT = 2;                    // TMEM stages of the split S tile
-constexpr int TC_CHUNK = 4;                 // stages accumulated in TMEM before a drain
+constexpr int TC_CHUNK = 2;                 // stages accumulated in TMEM before a drain
 constexpr int TC_THREADS = 256;
 constexpr uint32_t TC_A_BYTES = TC_BM * TC_BK * 4;
 
@@ -187,23 +187,22 @@ stream_tc_kernel(const __grid_constant__ CUtensorMap mapS, const __grid_constant
         for (int c = 0; c < K16; ++c) acc[c] = 0.f;
         bool alive = true;
 
-        // fold accumulator D[q % 2] into acc (round-to-nearest fp32 adds)
+        // fold accumulator D[q % 2] into acc (round-to-nearest fp32 adds); the
+        // tensor-core accumulation itself carries a one-signed rounding error
+        // per accumulate, so TMEM chains are kept to TC_CHUNK stages
         auto drain = [&](int q) -> bool {
             const int b = q & 1;
             if (!__all_sync(0xffffffffu, mbar_wait(&bar_dfull[b], (uint32_t)(q >> 1) & 1u)))
                 return false;
             tc_fence_after();
             const uint32_t dcol = tbase + lane_off + (uint32_t)b * (uint32_t)Cfg::N1;
+            uint32_t v[2 * K16 / 8][8];
 #pragma unroll
-            for (int g = 0; g < K16 / 8; ++g) {
-                uint32_t va[8], vb[8];
-                tmem_ld_32x32b_x8(dcol + (uint32_t)g * 8u, va);
-                tmem_ld_32x32b_x8(dcol + (uint32_t)(K16 + g * 8), vb);
-                tmem_wait_ld();
+            for (int g = 0; g < 2 * K16 / 8; ++g) tmem_ld_32x32b_x8(dcol + (uint32_t)g * 8u, v[g]);
+            tmem_wait_ld();
 #pragma unroll
-                for (int e = 0; e < 8; ++e)
-                    acc[g * 8 + e] += __uint_as_float(va[e]) + __uint_as_float(vb[e]);
-            }
+            for (int c = 0; c < K16; ++c)
+                acc[c] += __uint_as_float(v[c / 8][c % 8]) + __uint_as_float(v[(K16 + c) / 8][c % 8]);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&bar_dempty[b]);
