@@ -61,6 +61,20 @@ def corr_abs(R: np.ndarray) -> np.ndarray:
     return S
 
 
+def corr_abs_rows(R: np.ndarray, rows) -> np.ndarray:
+    """Rows ``rows`` of ``corr_abs(R)`` without forming the n x n matrix."""
+    X = np.asarray(R, dtype=np.float64)
+    T, n = X.shape
+    rows = np.asarray(rows)
+    Z = X - X.sum(axis=0) / T
+    ss = (Z * Z).sum(axis=0)
+    ok = ss > 0.0
+    Zn = np.where(ok, Z / np.sqrt(np.where(ok, ss, 1.0)), 0.0)
+    out = np.abs(Zn[:, rows].T @ Zn)
+    out[np.arange(len(rows)), rows] = 1.0
+    return out
+
+
 def tail_count(T: int, tail_frac: float) -> int:
     """N = max(1, floor(tail_frac * T)), evaluated in IEEE double."""
     return max(1, int(math.floor(tail_frac * float(T))))
@@ -106,6 +120,19 @@ def tpdm(R: np.ndarray, tail_frac: float = 0.05, tail_sign: int = 1,
     if return_parts:
         return S, dict(ranks=r, x=x, rho=rho, days=days)
     return S
+
+
+def tpdm_rows(R: np.ndarray, rows, tail_frac: float = 0.05, tail_sign: int = 1) -> np.ndarray:
+    """Rows ``rows`` of ``tpdm(R, tail_frac, tail_sign)`` without the n x n matrix."""
+    X = tail_sign * np.asarray(R, dtype=np.float64)
+    T, n = X.shape
+    r = column_ranks(X)
+    x = (-np.log(r / float(T + 1))) ** -0.5
+    rho = np.sqrt((x * x).sum(axis=1))
+    N = tail_count(T, tail_frac)
+    days = np.lexsort((np.arange(T), -rho))[:N]
+    W = x[days] / rho[days, None]
+    return (float(n) / N) * (W[:, np.asarray(rows)].T @ W)
 
 
 # ---------------------------------------------------------------------------
@@ -491,6 +518,7 @@ def ari(a, b) -> float:
 PINS = {
     "corr_abs": "numpy.corrcoef; T=2 closed form; symmetry, range, unit diagonal, affine invariance",
     "tpdm": "trace(S)=n; PSD of rank <= N; monotone invariance; day-permutation invariance; loop brute force",
+    "corr_abs_rows / tpdm_rows": "equal the rows of corr_abs / tpdm",
     "stats": "math.fsum; planted block closed form",
     "counter_uniform": "published splitmix64 outputs (tests/golden); uniformity",
     "trace_loss": "brute-force ||S - H H^T||_F^2",

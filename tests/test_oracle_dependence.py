@@ -159,3 +159,13 @@ def test_stats_planted_blocks_closed_form():
     S, _ = synth.planted_block_matrix([5, 3, 2])
     s, sq, bad = oracle.stats(S)
     assert (s, sq, bad) == (25 + 9 + 4, 25 + 9 + 4, 0)
+
+
+def test_row_sampled_builders_equal_full_rows():
+    R = _returns(90, 150, 13, dist="t3").astype(np.float64)
+    R[:, 4] = 2.0                                  # a zero-variance column
+    rows = np.array([0, 4, 77, 149])
+    np.testing.assert_allclose(oracle.corr_abs_rows(R, rows), oracle.corr_abs(R)[rows], atol=1e-13)
+    for sign in (1, -1):
+        np.testing.assert_allclose(oracle.tpdm_rows(R, rows, 0.05, sign),
+                                   oracle.tpdm(R, 0.05, sign)[rows], rtol=1e-12, atol=1e-14)
