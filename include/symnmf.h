@@ -238,6 +238,30 @@ SYMNMF_API int symnmf_fit(const float* S, int64_t n, int64_t lds, int k,
 SYMNMF_API int symnmf_labels(const float* H, int64_t n, int k, int32_t* labels,
                   symnmf_stream_t stream);
 
+/*
+ * Y = S X like symnmf_sh, for callers that cannot allocate device memory
+ * when they call in: a runtime whose device memory is owned entirely by its
+ * own pool or by another framework's caching allocator, where an outside
+ * cudaMalloc would fragment the pool or break its budget, or a latency-
+ * critical loop that cannot take cudaMalloc's implicit synchronisation.
+ * The pages have no counterpart of this entry point; it is a packaging
+ * variant of the S-stream.
+ *
+ * It takes no workspace and calls no allocating routine: its scratch (the
+ * TF32 split of X and an error word) lives in a 4 MiB file-scope device array
+ * that every GPU loading the library holds until exit.  Limit:
+ * 2 * roundup(k, 16) * roundup(n, 32) + 64 <= 1,048,576 floats (for k = 24,
+ * n <= 16,352); larger sizes return SYMNMF_ERR_INVALID_ARG.  The first call on
+ * a device looks up the array's device address (cudaGetSymbolAddress) with
+ * that device current; make that first call before any stream capture.
+ * Every call shares the one array and it keeps the last call's contents:
+ * calls that overlap on the GPU (on different streams, or from several host
+ * threads without ordering) race on it.  S, X, Y as for symnmf_sh.
+ * Asynchronous on `stream`.
+ */
+SYMNMF_API int symnmf_sh_noalloc(const float* S, int64_t n, int64_t lds, const float* X, int k,
+                                 float* Y, symnmf_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

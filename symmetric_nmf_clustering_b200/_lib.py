@@ -92,6 +92,7 @@ SIGNATURES = {
     "symnmf_fit": (_int, [_vp, _i64, _i64, _int, C.POINTER(FitParams), _vp, C.POINTER(FitStats),
                           _vp, _sz, _vp]),
     "symnmf_labels": (_int, [_vp, _i64, _int, _vp, _vp]),
+    "symnmf_sh_noalloc": (_int, [_vp, _i64, _i64, _vp, _int, _vp, _vp]),
 }
 
 _lib = None

@@ -1,0 +1,103 @@
+// symnmf_sh_noalloc: the S-stream product Y = S X without a caller workspace.
+//
+// Every other entry point that needs device scratch takes it from the caller
+// as a workspace.  Some callers cannot allocate device memory when they call
+// in: a host runtime whose device memory is owned entirely by its own pool
+// or by another framework's caching allocator (a cudaMalloc from outside
+// would fragment it or break its budget), or a latency-critical loop that
+// cannot take cudaMalloc's implicit device-wide synchronisation.  For them
+// this variant keeps its scratch in a fixed file-scope device array instead.
+#include <mutex>
+
+#include "common.cuh"
+
+namespace symnmf {
+
+// 4 MiB of device scratch.  Every GPU that loads the library holds it until
+// the process exits.  It holds the TF32 split of X and the error word.
+constexpr size_t kNoAllocScratchFloats = size_t(1) << 20;
+constexpr size_t kNoAllocErrFloats = 64;  // error word slot, kept 256-byte aligned
+static __device__ __align__(256) float g_noalloc_scratch[kNoAllocScratchFloats];
+
+// Host code cannot use g_noalloc_scratch's name as a device address: it is a
+// host-side stand-in.  The device address is looked up once per device, with
+// that device current, and cached.
+constexpr int kMaxDevices = 128;
+static std::mutex g_noalloc_mu;
+static float* g_noalloc_ptr[kMaxDevices] = {};
+
+static int noalloc_scratch(float** out) {
+    int dev = 0;
+    SYMNMF_CUDA_TRY(cudaGetDevice(&dev));
+    if (dev < 0 || dev >= kMaxDevices) {
+        set_error("device ordinal %d out of range for the static scratch table", dev);
+        return SYMNMF_ERR_NOT_SUPPORTED;
+    }
+    std::lock_guard<std::mutex> lock(g_noalloc_mu);
+    if (g_noalloc_ptr[dev] == nullptr) {
+        void* p = nullptr;
+        const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+        if (e != cudaSuccess) {
+            set_error("cudaGetSymbolAddress of the static scratch failed: %s",
+                      cudaGetErrorString(e));
+            return SYMNMF_ERR_CUDA;
+        }
+        g_noalloc_ptr[dev] = static_cast<float*>(p);
+    }
+    *out = g_noalloc_ptr[dev];
+    return SYMNMF_OK;
+}
+
+size_t noalloc_floats_needed(int64_t n, int k) {
+    return (size_t)xt_rows(k) * (size_t)xt_ld(n) + kNoAllocErrFloats;
+}
+
+}  // namespace symnmf
+
+using namespace symnmf;
+
+extern "C" int symnmf_sh_noalloc(const float* S, int64_t n, int64_t lds, const float* X, int k,
+                                 float* Y, symnmf_stream_t stream) {
+    clear_error();
+    if (n < 1 || lds < n || lds % 4 != 0) {
+        set_error("n = %lld, lds = %lld: need n >= 1, lds >= n, lds a multiple of 4", (long long)n,
+                  (long long)lds);
+        return SYMNMF_ERR_INVALID_ARG;
+    }
+    if (S == nullptr || (reinterpret_cast<uintptr_t>(S) & 15u) != 0) {
+        set_error("S must be a non-null 16-byte aligned device pointer");
+        return SYMNMF_ERR_INVALID_ARG;
+    }
+    if (k < 1 || k > KMAX) {
+        set_error("k = %d must be in [1, %d]", k, KMAX);
+        return SYMNMF_ERR_INVALID_ARG;
+    }
+    if (X == nullptr || Y == nullptr) {
+        set_error("X and Y must be device pointers");
+        return SYMNMF_ERR_INVALID_ARG;
+    }
+    const size_t need = noalloc_floats_needed(n, k);
+    if (need > kNoAllocScratchFloats) {
+        set_error("symnmf_sh_noalloc: n = %lld with k = %d needs %zu floats of static scratch; "
+                  "the limit is %zu (2 * roundup(k, 16) * roundup(n, 32) + 64 <= 1048576); "
+                  "use symnmf_sh with a workspace",
+                  (long long)n, k, need, kNoAllocScratchFloats);
+        return SYMNMF_ERR_INVALID_ARG;
+    }
+    Dev d;
+    SYMNMF_TRY(device_info(&d));
+    float* scratch = nullptr;
+    SYMNMF_TRY(noalloc_scratch(&scratch));
+    cudaStream_t s = (cudaStream_t)stream;
+    // one contraction split writes Y directly; no partials
+    TcPlan p = plan_stream_tc(d, n, k, 0, n);
+    p.splits = 1;
+    p.jspan = (p.j1 - p.j0 + 31) / 32 * 32;
+    float* XT = scratch + kNoAllocErrFloats;
+    int* err = reinterpret_cast<int*>(scratch);
+    const int64_t ldxt = xt_ld(n);
+    // the array keeps the previous call's contents: the error word starts at zero
+    SYMNMF_CUDA_TRY(cudaMemsetAsync(err, 0, sizeof(int), s));
+    SYMNMF_TRY(launch_split(X, nullptr, k, k, 0, n, p.j0, p.j1, XT, ldxt, s));
+    return launch_stream_tc(p, S, lds, XT, ldxt, Y, err, nullptr, s);
+}
