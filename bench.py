@@ -53,6 +53,7 @@ def parse():
     ap.add_argument("--workload", default="corr_n100000_k24")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-rows", action="store_true", help="skip the per-row timings")
     return ap.parse_args()
 
 
@@ -165,6 +166,65 @@ def oracle_sample(name: str, seed: int, steps: int, warmup: int):
                    f"by (n/r)^2 = {(n / r) ** 2:.1f}"),
         "sample_seconds": dt,
     }
+
+
+def _timed(torch, fn):
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    a.record()
+    out = fn()
+    b.record()
+    torch.cuda.synchronize()
+    return a.elapsed_time(b), out
+
+
+def measure_rows(m, torch, dev, S, H0, n, k, T, rank, workload):
+    """One timing per remaining row of the path on the resident |corr| matrix
+    (probe, labels, statistics) and on a TPDM of the heavy-tailed window of the
+    same size (builder, one Block-SVRG epoch)."""
+    out = {}
+    # statistics pre-pass: one read of S
+    ws = m.workspace(m._lib.OP_STATS, n, device=dev)
+    ms, _ = _timed(torch, lambda: m.stats(S, ws=ws))
+    out["stats_ms"] = ms
+    out["stats_GBs"] = 4.0 * n * n / (ms / 1e3) / 1e9
+    # labels
+    ms, _ = _timed(torch, lambda: m.labels(H0))
+    out["labels_ms"] = ms
+    # spectral probe of the k+2 leading eigenvalues (block Lanczos on the S-stream)
+    p = m.fit_params(probe_block=16, probe_max_iter=12)
+    wsp = m.workspace(m._lib.OP_SPECTRAL_PROBE, n, k + 2, params=p, device=dev)
+    ms, ev = _timed(torch, lambda: m.spectral_probe(S, k + 2, block=16, max_iter=12, tol=1e-7, ws=wsp))
+    out["probe_ms"] = ms
+    out["probe_top"] = [float(x) for x in ev[:3]]
+    out["probe_gamma_k1"] = float(ev[k] / abs(ev[k + 1]))
+    del wsp
+    # TPDM of the heavy-tailed window (same n, T) into a second n x n buffer
+    tname = workload.replace("corr", "tpdm")
+    if tname in synth.WORKLOADS:
+        Rt, _, _ = synth.workload(tname, seed=rank)
+        Rt = torch.from_numpy(Rt).to(dev)
+        S2 = m.alloc_S(n, dev)
+        wst = m.workspace(m._lib.OP_BUILD_TPDM, n, 0, T, device=dev)
+        m.build_tpdm(Rt, 0.05, 1, out=S2, ws=wst)   # warm-up (cudaFuncSetAttribute etc.)
+        ms, _ = _timed(torch, lambda: m.build_tpdm(Rt, 0.05, 1, out=S2, ws=wst))
+        out["tpdm_build_ms"] = ms
+        out["tpdm_build_write_GBs"] = 4.0 * n * n / (ms / 1e3) / 1e9
+        del wst, Rt
+        # one Block-SVRG epoch at the workload's block (snapshot + m block steps)
+        b = 8192 if n >= 100000 else 2048
+        pf = m.fit_params(solver="block_svrg", block_rows=b, max_iters=1, rel_tol=0.0, grow=0)
+        wsf = m.workspace(m._lib.OP_FIT, n, k, params=pf, device=dev)
+        Hs = H0.clone()
+        ms, (_, st) = _timed(torch, lambda: m.fit(S2, k, H0=Hs, out=Hs, solver="block_svrg",
+                                                  block_rows=b, max_iters=1, rel_tol=0.0,
+                                                  grow=False, ws=wsf))
+        out["svrg_epoch_ms"] = ms
+        out["svrg_block_rows"] = b
+        out["svrg_epochs"] = st["epochs"]
+        del S2, wsf, Hs
+        torch.cuda.empty_cache()
+    return out
 
 
 # ----------------------------------------------------------------------------- reference arm
@@ -308,6 +368,11 @@ def run_ours(args):
                "note": "per fit of K iterations: window upload, |corr| build, fit, labels+loss download"}
         del ws_corr
 
+    # --- the other rows of the path, each timed once on this GPU (CUDA events)
+    rows = None
+    if not args.no_rows:
+        rows = measure_rows(m, torch, dev, S, H0, n, k, T, rank, args.workload)
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         res = oracle_sample(args.workload, 0, 20, 2)
@@ -334,6 +399,7 @@ def run_ours(args):
             "clocks": clk,
             "e2e": e2e,
             "cpu_baseline": cpu,
+            "rows": rows,
             "context": {"corr_build_ms": build_ms, "torch_mm_S_H_ms": mm_ms,
                         "ARI_vs_planted": oracle.ari(lab.cpu().numpy(), planted),
                         "final_loss": st["loss"], "loop_ms": st["loop_ms"]},

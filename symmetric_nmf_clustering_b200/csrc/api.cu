@@ -10,6 +10,7 @@
 #include <vector>
 
 #include "common.cuh"
+#include "epilogue.cuh"
 #include "hostla.h"
 
 namespace symnmf {
@@ -97,14 +98,16 @@ struct StreamArgs {
     float* XT;     // [X_hi; X_lo] operand buffer (tensor-core path)
     int64_t ldxt;
     int* err;
+    int* counters; // one per 128-row tile, zero between passes (tensor-core path)
     const FitState* st;
 };
 
-// part[s] = S[:, r0:r1] X[r0:r1, :] with X = Xa - Xb (Xb may be NULL) on the rows
-// [r0, r1).  xt_ready: XT already holds the split of X (tensor-core path).
-static int stream_product(const Dev& d, const StreamArgs& a, const float* Xa, const float* Xb,
-                          int64_t ldx, int64_t r0, int64_t r1, bool xt_ready, cudaStream_t s,
-                          int* splits, struct Timing* tm);
+// One pass over S: part[s] = S[:, r0:r1] X[r0:r1, :] with X = Xa - Xb (Xb may be
+// NULL) on the rows [r0, r1), then the epilogue `epi` (fused into the stream
+// kernel on the tensor-core path).  xt_ready: XT already holds the split of X.
+static int stream_pass(const Dev& d, const StreamArgs& a, const float* Xa, const float* Xb,
+                       int64_t ldx, int64_t r0, int64_t r1, bool xt_ready, EpiArgs epi,
+                       cudaStream_t s, struct Timing* tm);
 
 // ---------------------------------------------------------------- workspace plans
 struct FitLayout {
@@ -122,8 +125,9 @@ struct FitLayout {
     void* probe_ws = nullptr;
     size_t probe_bytes = 0;
     int hist_cap = 0;
-    float* XT = nullptr;
+    float* XT[2] = {nullptr, nullptr};   // split operand of Hb[0] / Hb[1]
     int64_t ldxt = 0;
+    int* counters = nullptr;
 };
 
 static int64_t default_block_rows(int64_t n) {
@@ -144,6 +148,7 @@ struct ProbeLayout {
     float* XT = nullptr;     // split operand of the tensor-core stream
     int64_t ldxt = 0;
     int* err = nullptr;
+    int* counters = nullptr;
     double* tn_part = nullptr;
     double* C64 = nullptr;
     float* C32 = nullptr;
@@ -166,6 +171,7 @@ static size_t probe_workspace(const Dev& d, int64_t n, int block, int max_iter, 
     L->ldxt = xt_ld(n);
     L->XT = a->take<float>((size_t)xt_rows(block) * L->ldxt);
     L->err = a->take<int>(64);
+    L->counters = a->take<int>((size_t)epilogue_blocks(n));
     L->tn_part = a->take<double>((size_t)gemm_tn_blocks(n) * 4096);
     L->C64 = a->take<double>((size_t)mtot * block);
     L->C32 = a->take<float>((size_t)mtot * block);
@@ -195,7 +201,9 @@ static int plan_fit(const Dev& d, Arena& a, int64_t n, int k, const symnmf_fit_p
     }
     L->part = a.take<float>(pf);
     L->ldxt = xt_ld(n);
-    L->XT = a.take<float>((size_t)xt_rows(k) * L->ldxt);
+    L->XT[0] = a.take<float>((size_t)xt_rows(k) * L->ldxt);
+    L->XT[1] = a.take<float>((size_t)xt_rows(k) * L->ldxt);
+    L->counters = a.take<int>((size_t)epilogue_blocks(n));
     const int nb = epilogue_blocks(n);
     L->tr_part = a.take<double>((size_t)nb);
     L->gram_part = a.take<double>((size_t)nb * k * k);
@@ -302,25 +310,38 @@ static int read_state(const FitState* st, HostState* h, cudaStream_t s) {
     return SYMNMF_OK;
 }
 
-static int stream_product(const Dev& d, const StreamArgs& a, const float* Xa, const float* Xb,
-                          int64_t ldx, int64_t r0, int64_t r1, bool xt_ready, cudaStream_t s,
-                          int* splits, Timing* tm) {
+static int stream_pass(const Dev& d, const StreamArgs& a, const float* Xa, const float* Xb,
+                       int64_t ldx, int64_t r0, int64_t r1, bool xt_ready, EpiArgs epi,
+                       cudaStream_t s, Timing* tm) {
+    epi.part = a.part;
     if (use_tc()) {
         const TcPlan p = plan_stream_tc(d, a.n, a.k, r0, r1);
         if (!xt_ready)
             SYMNMF_TRY(launch_split(Xa, Xb, ldx, a.k, r0, r1, p.j0, p.j1, a.XT, a.ldxt, s));
+        epi.splits = p.splits;
         if (tm) SYMNMF_TRY(tm->begin(s));
-        SYMNMF_TRY(launch_stream_tc(p, a.S, a.lds, a.XT, a.ldxt, a.part, a.err, a.st, s));
+        SYMNMF_TRY(launch_stream_tc(p, a.S, a.lds, a.XT, a.ldxt, a.part, a.err, a.st, s, &epi,
+                                    a.counters));
         if (tm) SYMNMF_TRY(tm->end(s));
-        *splits = p.splits;
-    } else {
-        const StreamPlan p = plan_stream(d, a.n, a.k, r0, r1);
-        if (tm) SYMNMF_TRY(tm->begin(s));
-        SYMNMF_TRY(launch_stream_partial(p, a.S, a.lds, Xa, Xb, ldx, a.part, a.st, s));
-        if (tm) SYMNMF_TRY(tm->end(s));
-        *splits = p.splits;
+        return SYMNMF_OK;
     }
-    return SYMNMF_OK;
+    const StreamPlan p = plan_stream(d, a.n, a.k, r0, r1);
+    if (tm) SYMNMF_TRY(tm->begin(s));
+    SYMNMF_TRY(launch_stream_partial(p, a.S, a.lds, Xa, Xb, ldx, a.part, a.st, s));
+    if (tm) SYMNMF_TRY(tm->end(s));
+    return launch_epilogue(epi.mode, epi.n, epi.k, a.part, p.splits, epi.H, epi.G, epi.Hn, epi.Gn,
+                           epi.Psnap, epi.m_scale, epi.lr, epi.eps, epi.tr_part, epi.gram_part,
+                           epi.Y, epi.st, s, epi.XT, epi.ldxt);
+}
+
+static EpiArgs epi_product(int64_t n, int k, float* Y) {
+    EpiArgs e;
+    std::memset(&e, 0, sizeof(e));
+    e.mode = MODE_PRODUCT;
+    e.n = n;
+    e.k = k;
+    e.Y = Y;
+    return e;
 }
 
 struct FitCtx {
@@ -344,24 +365,42 @@ struct FitCtx {
         a.lds = lds;
         a.k = k;
         a.part = L.part;
-        a.XT = L.XT;
+        a.XT = L.XT[cur];
         a.ldxt = L.ldxt;
         a.err = &L.st->kerr;
+        a.counters = L.counters;
         a.st = L.st;
         return a;
+    }
+    // epilogue arguments of a pass that reads Hb[cur] and writes Hb[cur ^ 1]
+    EpiArgs epi(int mode, float m_scale, bool write_xt) const {
+        EpiArgs e;
+        std::memset(&e, 0, sizeof(e));
+        e.mode = mode;
+        e.n = n;
+        e.k = k;
+        e.H = Hb[cur];
+        e.G = Gb[cur];
+        e.Hn = Hb[cur ^ 1];
+        e.Gn = Gb[cur ^ 1];
+        e.Psnap = L.Psnap;
+        e.m_scale = m_scale;
+        e.lr = P->lr;
+        e.eps = P->eps;
+        e.tr_part = L.tr_part;
+        e.gram_part = L.gram_part;
+        e.st = L.st;
+        e.XT = write_xt ? L.XT[cur ^ 1] : nullptr;
+        e.ldxt = L.ldxt;
+        return e;
     }
 };
 
 // One S pass + epilogue + finalise in `mode`, reading Hb[cur], writing Hb[cur^1].
 // xt_ready: the split operand of Hb[cur] is already in XT (full-batch loop).
 static int full_pass(FitCtx& c, int mode, int max_evals, bool xt_ready) {
-    int splits = 0;
-    SYMNMF_TRY(stream_product(c.d, c.args(), c.Hb[c.cur], nullptr, c.k, 0, c.n, xt_ready, c.s,
-                              &splits, &c.tm));
-    SYMNMF_TRY(launch_epilogue(mode, c.n, c.k, c.L.part, splits, c.Hb[c.cur], c.Gb[c.cur],
-                               c.Hb[c.cur ^ 1], c.Gb[c.cur ^ 1], c.L.Psnap, 0.f, c.P->lr,
-                               c.P->eps, c.L.tr_part, c.L.gram_part, nullptr, c.L.st, c.s,
-                               c.L.XT, c.L.ldxt));
+    SYMNMF_TRY(stream_pass(c.d, c.args(), c.Hb[c.cur], nullptr, c.k, 0, c.n, xt_ready,
+                           c.epi(mode, 0.f, mode == MODE_FULL), c.s, &c.tm));
     return launch_finalize(mode, epilogue_blocks(c.n), c.k, c.L.tr_part, c.L.gram_part, c.L.st,
                            c.P->rel_tol, max_evals, c.L.hist, c.L.hist_cap, c.s);
 }
@@ -426,7 +465,7 @@ static int run_svrg(FitCtx& c, int max_evals, HostState* hs, int64_t* block_fina
             SYMNMF_TRY(launch_epilogue(MODE_STEP_SNAP, n, c.k, nullptr, 0, c.Hb[c.cur], c.Gb[c.cur],
                                        c.Hb[c.cur ^ 1], c.Gb[c.cur ^ 1], c.L.Psnap, 0.f, c.P->lr,
                                        c.P->eps, c.L.tr_part, c.L.gram_part, nullptr, c.L.st, c.s,
-                                       c.L.XT, c.L.ldxt));
+                                       c.L.XT[c.cur ^ 1], c.L.ldxt));
             SYMNMF_TRY(launch_finalize(MODE_STEP_SNAP, epilogue_blocks(n), c.k, c.L.tr_part,
                                        c.L.gram_part, c.L.st, c.P->rel_tol, max_evals, c.L.hist,
                                        c.L.hist_cap, c.s));
@@ -441,13 +480,8 @@ static int run_svrg(FitCtx& c, int max_evals, HostState* hs, int64_t* block_fina
                                         cudaMemcpyDeviceToDevice, c.s));
         for (int64_t q = 0; q < m; ++q) {
             const int64_t r0 = perm[q] * b, r1 = std::min(n, r0 + b);
-            int splits = 0;
-            SYMNMF_TRY(stream_product(c.d, c.args(), c.Hb[c.cur], c.L.Hsnap, c.k, r0, r1, false,
-                                      c.s, &splits, &c.tm));
-            SYMNMF_TRY(launch_epilogue(MODE_SVRG_INNER, n, c.k, c.L.part, splits, c.Hb[c.cur],
-                                       c.Gb[c.cur], c.Hb[c.cur ^ 1], c.Gb[c.cur ^ 1], c.L.Psnap,
-                                       (float)m, c.P->lr, c.P->eps, c.L.tr_part, c.L.gram_part,
-                                       nullptr, c.L.st, c.s));
+            SYMNMF_TRY(stream_pass(c.d, c.args(), c.Hb[c.cur], c.L.Hsnap, c.k, r0, r1, false,
+                                   c.epi(MODE_SVRG_INNER, (float)m, false), c.s, &c.tm));
             SYMNMF_TRY(launch_finalize(MODE_SVRG_INNER, epilogue_blocks(n), c.k, c.L.tr_part,
                                        c.L.gram_part, c.L.st, c.P->rel_tol, max_evals, c.L.hist,
                                        c.L.hist_cap, c.s));
@@ -522,10 +556,12 @@ static int fit_impl(const float* S, int64_t n, int64_t lds, int k, const symnmf_
     else
         SYMNMF_CUDA_TRY(cudaMemsetAsync(c.L.G0, 0, (size_t)n * k * sizeof(float), s));
     // Gram of H0 (also writes the split operand of H0; its padding rows stay zero)
-    SYMNMF_CUDA_TRY(cudaMemsetAsync(c.L.XT, 0, (size_t)xt_rows(k) * c.L.ldxt * sizeof(float), s));
+    for (int b = 0; b < 2; ++b)
+        SYMNMF_CUDA_TRY(cudaMemsetAsync(c.L.XT[b], 0, (size_t)xt_rows(k) * c.L.ldxt * sizeof(float), s));
+    SYMNMF_CUDA_TRY(cudaMemsetAsync(c.L.counters, 0, (size_t)epilogue_blocks(n) * sizeof(int), s));
     SYMNMF_TRY(launch_epilogue(MODE_GRAM, n, k, nullptr, 0, H, nullptr, nullptr, nullptr, nullptr,
                                0.f, 0.f, 0.f, c.L.tr_part, c.L.gram_part, nullptr, c.L.st, s,
-                               c.L.XT, c.L.ldxt));
+                               c.L.XT[0], c.L.ldxt));
     SYMNMF_TRY(launch_finalize(MODE_GRAM, epilogue_blocks(n), k, c.L.tr_part, c.L.gram_part,
                                c.L.st, P.rel_tol, P.max_iters + 1, c.L.hist, c.L.hist_cap, s));
 
@@ -783,8 +819,10 @@ static int probe_impl(const Dev& d, const float* S, int64_t n, int64_t lds, int 
     sa.XT = L.XT;
     sa.ldxt = L.ldxt;
     sa.err = L.err;
+    sa.counters = L.counters;
     sa.st = nullptr;
     SYMNMF_CUDA_TRY(cudaMemsetAsync(L.err, 0, sizeof(int), s));
+    SYMNMF_CUDA_TRY(cudaMemsetAsync(L.counters, 0, (size_t)epilogue_blocks(n) * sizeof(int), s));
     std::vector<double> T((size_t)mtot * mtot, 0.0), B, coef, theta, prev;
     // start block: seeded uniform noise, orthonormalised
     SYMNMF_TRY(launch_uniform_fill(L.W, n * (int64_t)b, seed, -0.5f, s));
@@ -796,12 +834,8 @@ static int probe_impl(const Dev& d, const float* S, int64_t n, int64_t lds, int 
     int have = 0;  // columns of T resolved
     for (int j = 0; j < steps; ++j) {
         // W = S Q_j (one S pass)
-        int splits = 0;
-        SYMNMF_TRY(stream_product(d, sa, L.Q + (size_t)j * b, nullptr, ldq, 0, n, false, s,
-                                  &splits, nullptr));
-        SYMNMF_TRY(launch_epilogue(MODE_PRODUCT, n, b, L.part, splits, nullptr, nullptr, nullptr,
-                                   nullptr, nullptr, 0.f, 0.f, 0.f, nullptr, nullptr, L.W, nullptr,
-                                   s));
+        SYMNMF_TRY(stream_pass(d, sa, L.Q + (size_t)j * b, nullptr, ldq, 0, n, false,
+                               epi_product(n, b, L.W), s, nullptr));
         // full reorthogonalisation against Q_0..Q_j, twice; the Q_j coefficients are A_j
         const int nq = (j + 1) * b;
         coef.assign((size_t)nq * b, 0.0);
@@ -965,6 +999,7 @@ int symnmf_workspace_size(int op, int64_t n, int k, int64_t T, const symnmf_fit_
             a.take<float>(stream_partials(d, n, k, 0, n));
             a.take<float>((size_t)xt_rows(k) * xt_ld(n));
             a.take<int>(64);
+            a.take<int>((size_t)epilogue_blocks(n));
             break;
         }
         case SYMNMF_OP_STATS:
@@ -1081,6 +1116,7 @@ int symnmf_sh(const float* S, int64_t n, int64_t lds, const float* X, int k, flo
     sa.ldxt = xt_ld(n);
     sa.XT = a.take<float>((size_t)xt_rows(k) * sa.ldxt);
     sa.err = a.take<int>(64);
+    sa.counters = a.take<int>((size_t)epilogue_blocks(n));
     sa.st = nullptr;
     if (!a.ok()) {
         set_error("workspace too small: %zu given, %zu needed", ws_bytes, a.used);
@@ -1088,10 +1124,8 @@ int symnmf_sh(const float* S, int64_t n, int64_t lds, const float* X, int k, flo
     }
     cudaStream_t s = (cudaStream_t)stream;
     SYMNMF_CUDA_TRY(cudaMemsetAsync(sa.err, 0, sizeof(int), s));
-    int splits = 0;
-    SYMNMF_TRY(stream_product(d, sa, X, nullptr, k, 0, n, false, s, &splits, nullptr));
-    return launch_epilogue(MODE_PRODUCT, n, k, sa.part, splits, nullptr, nullptr, nullptr, nullptr,
-                           nullptr, 0.f, 0.f, 0.f, nullptr, nullptr, Y, nullptr, s);
+    SYMNMF_CUDA_TRY(cudaMemsetAsync(sa.counters, 0, (size_t)epilogue_blocks(n) * sizeof(int), s));
+    return stream_pass(d, sa, X, nullptr, k, 0, n, false, epi_product(n, k, Y), s, nullptr);
 }
 
 int symnmf_spectral_probe(const float* S, int64_t n, int64_t lds, int n_eig, int block,

@@ -78,6 +78,7 @@ constexpr int KMAX = 64;
 struct FitState {
     double s_sum, s_sqnorm, s_bad;     // statistics pre-pass
     double loss, loss_prev, rel;       // last evaluation
+    double a_sqnorm;                   // ||A||_F^2 of the Gram below
     double A64[KMAX * KMAX];           // Gram H^T H of the current iterate (fp64)
     float A32[KMAX * KMAX];            // same, rounded to fp32 for the epilogue
     int t;                             // evaluations done
@@ -133,8 +134,12 @@ struct TcPlan {
 };
 TcPlan plan_stream_tc(const Dev& d, int64_t n, int k, int64_t j0, int64_t j1);
 size_t tc_partial_floats(const TcPlan& p);
+struct EpiArgs;
+// epi != NULL: the last split CTA of each row tile runs the epilogue in place
+// (`counters`: one int per 128-row tile, zero between passes).
 int launch_stream_tc(const TcPlan& p, const float* S, int64_t lds, const float* XT, int64_t ldxt,
-                     float* part, int* err, const FitState* st, cudaStream_t s);
+                     float* part, int* err, const FitState* st, cudaStream_t s,
+                     const EpiArgs* epi = nullptr, int* counters = nullptr);
 int launch_split(const float* Xa, const float* Xb, int64_t ldx, int k, int64_t r0, int64_t r1,
                  int64_t jlo, int64_t jhi, float* XT, int64_t ldxt, cudaStream_t s);
 inline int64_t xt_ld(int64_t n) { return (n + 31) / 32 * 32; }

@@ -1,0 +1,200 @@
+// The per-tile epilogue of an S-stream pass, shared by the standalone
+// epilogue kernel and the tensor-core stream kernel (where the last split CTA
+// of each 128-row tile runs it in place).
+//
+// For the rows i of one tile, with P_i = sum over splits of the partial rows
+// (fixed split order), by mode:
+//   FULL        tr partial sum_c H_ic P_ic; g = 4 (H_i A - P_i);
+//               G' = G + g*g; H' = max(H - lr g / (sqrt(G') + eps), 0)
+//               ([CaS] "Factorizing with SymNMF"; [SMI] AdaptGrow sketch);
+//               Gram partial of H'; exact TF32 split of H' for the next pass
+//   SNAPSHOT    P~_i = P_i; tr partial (Block-SVRG snapshot)
+//   SVRG_INNER  P_i <- P~_i + m Y_i, then the FULL step without the trace
+//   STEP_SNAP   P_i <- P~_i, then the FULL step without the trace
+//   GRAM        Gram partial of H (and its TF32 split)
+//   PRODUCT     Y_i = P_i
+#pragma once
+
+#include "common.cuh"
+
+namespace symnmf {
+
+constexpr int EP_ROWS = 128;
+
+struct EpiArgs {
+    int mode;
+    int64_t n;
+    int k;
+    const float* part;     // splits x n x k partial products
+    int splits;
+    const float* H;
+    const float* G;
+    float* Hn;
+    float* Gn;
+    float* Psnap;
+    float m_scale, lr, eps;
+    double* tr_part;       // one per tile
+    double* gram_part;     // k*k per tile
+    float* Y;
+    const FitState* st;
+    float* XT;             // split operand of the rows left in h (may be null)
+    int64_t ldxt;
+};
+
+// Barrier over the 128 threads that run one tile's epilogue.
+template <bool FUSED>
+__device__ __forceinline__ void ep_sync() {
+    if (FUSED) asm volatile("bar.sync 1, 128;" ::: "memory");
+    else __syncthreads();
+}
+
+// Fixed-shape sum over the 128 threads (warp shuffles, then warp 0); the
+// result is valid in tid 0.
+template <bool FUSED>
+__device__ __forceinline__ double ep_sum(double v, int tid, double* red) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_down_sync(0xffffffffu, v, o);
+    const int w = tid >> 5, l = tid & 31;
+    if (l == 0) red[w] = v;
+    ep_sync<FUSED>();
+    double r = 0.0;
+    if (w == 0) {
+        r = l < EP_ROWS / 32 ? red[l] : 0.0;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) r += __shfl_down_sync(0xffffffffu, r, o);
+    }
+    ep_sync<FUSED>();
+    return r;
+}
+
+// smem: at least max(KE*KE, EP_ROWS*(KE+1)) floats; red: EP_ROWS/32 doubles.
+template <int KE, bool FUSED>
+__device__ void epilogue_tile(const EpiArgs& a, int tile, int tid, float* smem, double* red) {
+    const int mode = a.mode;
+    const int64_t n = a.n;
+    const int k = a.k;
+    float* As = smem;                                            // k x k Gram (step modes)
+    float(*hs)[KE + 1] = reinterpret_cast<float(*)[KE + 1]>(smem);  // rows for the Gram partial
+
+    const int64_t i = (int64_t)tile * EP_ROWS + tid;
+    const bool valid = i < n;
+    const bool step = mode == MODE_FULL || mode == MODE_SVRG_INNER || mode == MODE_STEP_SNAP;
+
+    if (step) {
+        for (int e = tid; e < k * k; e += EP_ROWS) As[(e / k) * KE + (e % k)] = a.st->A32[e];
+        ep_sync<FUSED>();
+    }
+
+    float p[KE], h[KE];
+#pragma unroll
+    for (int c = 0; c < KE; ++c) {
+        p[c] = 0.f;
+        h[c] = 0.f;
+    }
+    if (valid) {
+        const int64_t row = i * (int64_t)k;
+        if (mode != MODE_GRAM && mode != MODE_STEP_SNAP) {
+            for (int s = 0; s < a.splits; ++s) {
+                const float* src = a.part + (int64_t)s * n * k + row;
+#pragma unroll
+                for (int c = 0; c < KE; ++c)
+                    if (c < k) p[c] += __ldcg(src + c);   // written by other CTAs
+            }
+        }
+        if (mode == MODE_STEP_SNAP) {
+#pragma unroll
+            for (int c = 0; c < KE; ++c)
+                if (c < k) p[c] = a.Psnap[row + c];
+        } else if (mode == MODE_SVRG_INNER) {
+#pragma unroll
+            for (int c = 0; c < KE; ++c)
+                if (c < k) p[c] = fmaf(a.m_scale, p[c], a.Psnap[row + c]);
+        }
+        if (mode == MODE_PRODUCT) {
+#pragma unroll
+            for (int c = 0; c < KE; ++c)
+                if (c < k) a.Y[row + c] = p[c];
+            return;
+        }
+        if (mode == MODE_SNAPSHOT) {
+#pragma unroll
+            for (int c = 0; c < KE; ++c)
+                if (c < k) a.Psnap[row + c] = p[c];
+        }
+#pragma unroll
+        for (int c = 0; c < KE; ++c)
+            if (c < k) h[c] = a.H[row + c];
+    }
+    if (mode == MODE_PRODUCT) return;
+
+    // trace partial: sum_i sum_c H_ic (S H)_ic in fp64 (products of fp32 are exact)
+    if (mode == MODE_FULL || mode == MODE_SNAPSHOT) {
+        double tr = 0.0;
+#pragma unroll
+        for (int c = 0; c < KE; ++c) tr += (double)h[c] * (double)p[c];
+        const double tot = ep_sum<FUSED>(tr, tid, red);
+        if (tid == 0) a.tr_part[tile] = tot;
+    }
+    if (mode == MODE_SNAPSHOT) return;
+
+    if (step && valid) {
+        const int64_t row = i * (int64_t)k;
+        float hnew[KE];
+#pragma unroll
+        for (int c = 0; c < KE; ++c) {
+            hnew[c] = 0.f;
+            if (c < k) {
+                float ha = 0.f;
+#pragma unroll
+                for (int d = 0; d < KE; ++d)
+                    if (d < k) ha = fmaf(h[d], As[d * KE + c], ha);
+                const float g = 4.f * (ha - p[c]);
+                const float gg = fmaf(g, g, a.G[row + c]);
+                const float stepv = __fdiv_rn(a.lr * g, __fadd_rn(__fsqrt_rn(gg), a.eps));
+                hnew[c] = fmaxf(h[c] - stepv, 0.f);
+                a.Gn[row + c] = gg;
+                a.Hn[row + c] = hnew[c];
+            }
+        }
+#pragma unroll
+        for (int c = 0; c < KE; ++c) h[c] = hnew[c];
+    }
+
+    // exact TF32 split [h_hi; h_lo] of the rows in h, the next S-stream's operand
+    if (a.XT != nullptr && valid &&
+        (mode == MODE_FULL || mode == MODE_STEP_SNAP || mode == MODE_GRAM)) {
+        const int K16 = (k + 15) / 16 * 16;
+#pragma unroll
+        for (int c = 0; c < KE; ++c) {
+            if (c < k) {
+                const float hb = __uint_as_float(__float_as_uint(h[c]) & 0xFFFFE000u);
+                a.XT[(int64_t)c * a.ldxt + i] = hb;
+                a.XT[(int64_t)(K16 + c) * a.ldxt + i] = h[c] - hb;
+            }
+        }
+    }
+
+    // Gram partial of the rows now in h (new iterate, or the given H for GRAM)
+    ep_sync<FUSED>();  // every thread is done reading As
+#pragma unroll
+    for (int c = 0; c < KE; ++c) hs[tid][c] = valid ? h[c] : 0.f;
+    ep_sync<FUSED>();
+    const int rows = (int)min64(EP_ROWS, n - (int64_t)tile * EP_ROWS);
+    double* gp = a.gram_part + (int64_t)tile * k * k;
+    for (int e = tid; e < k * k; e += EP_ROWS) {
+        const int c = e / k, d = e % k;
+        // four interleaved chains (fixed order), combined as ((s0 + s1) + (s2 + s3))
+        double s0 = 0.0, s1 = 0.0, s2 = 0.0, s3 = 0.0;
+        int r = 0;
+        for (; r + 4 <= rows; r += 4) {
+            s0 = fma((double)hs[r][c], (double)hs[r][d], s0);
+            s1 = fma((double)hs[r + 1][c], (double)hs[r + 1][d], s1);
+            s2 = fma((double)hs[r + 2][c], (double)hs[r + 2][d], s2);
+            s3 = fma((double)hs[r + 3][c], (double)hs[r + 3][d], s3);
+        }
+        for (; r < rows; ++r) s0 = fma((double)hs[r][c], (double)hs[r][d], s0);
+        gp[e] = (s0 + s1) + (s2 + s3);
+    }
+}
+
+}  // namespace symnmf

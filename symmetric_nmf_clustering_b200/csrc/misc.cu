@@ -37,20 +37,31 @@ stats_partial_kernel(const float* __restrict__ S, int64_t n, int64_t lds,
     const int64_t n4 = n >> 2;
     for (int64_t r = blockIdx.x; r < n; r += gridDim.x) {
         const float4* row = reinterpret_cast<const float4*>(S + r * lds);
-        for (int64_t q = threadIdx.x; q < n4; q += blockDim.x) {
-            float4 v;
-            asm volatile("ld.global.nc.L1::no_allocate.v4.f32 {%0,%1,%2,%3}, [%4];"
-                         : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
-                         : "l"(row + q));
-            const float e[4] = {v.x, v.y, v.z, v.w};
+        constexpr int U = 4;  // loads in flight per thread
+        for (int64_t q0 = threadIdx.x; q0 < n4; q0 += (int64_t)U * blockDim.x) {
+            float4 v[U];
 #pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                if (isfinite(e[u])) {
-                    const double d = e[u];
-                    sum += d;
-                    sq = fma(d, d, sq);
-                } else {
-                    bad += 1.0;
+            for (int u = 0; u < U; ++u) {
+                const int64_t q = q0 + (int64_t)u * blockDim.x;
+                if (q < n4)
+                    asm volatile("ld.global.nc.L1::no_allocate.v4.f32 {%0,%1,%2,%3}, [%4];"
+                                 : "=f"(v[u].x), "=f"(v[u].y), "=f"(v[u].z), "=f"(v[u].w)
+                                 : "l"(row + q));
+                else
+                    v[u] = make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const float e[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+                for (int w = 0; w < 4; ++w) {
+                    if (isfinite(e[w])) {
+                        const double d = e[w];
+                        sum += d;
+                        sq = fma(d, d, sq);
+                    } else {
+                        bad += 1.0;
+                    }
                 }
             }
         }

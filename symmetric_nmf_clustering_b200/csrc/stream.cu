@@ -17,6 +17,7 @@
 // the output index i.  Every reduction has a fixed order, so results are
 // bitwise reproducible run to run on a given device.
 #include "common.cuh"
+#include "epilogue.cuh"
 
 namespace symnmf {
 
@@ -166,154 +167,17 @@ int launch_stream_partial(const StreamPlan& p, const float* S, int64_t lds,
 
 // ----------------------------------------------------------------------------
 // Epilogue: gradient, AdaGrad step and Gram partial per block of rows
+// (standalone kernel around epilogue_tile; see epilogue.cuh)
 // ----------------------------------------------------------------------------
-constexpr int EP_ROWS = 128;
-
 int epilogue_blocks(int64_t n) { return (int)((n + EP_ROWS - 1) / EP_ROWS); }
 
-__device__ __forceinline__ double block_sum_fixed(double v, double* red) {
-    // fixed-shape tree: warp shuffle, then warp 0 over the per-warp sums
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v += __shfl_down_sync(0xffffffffu, v, o);
-    const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
-    if (l == 0) red[w] = v;
-    __syncthreads();
-    double r = 0.0;
-    if (w == 0) {
-        r = (l < (int)(blockDim.x >> 5)) ? red[l] : 0.0;
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) r += __shfl_down_sync(0xffffffffu, r, o);
-    }
-    __syncthreads();
-    return r;  // valid in thread 0
-}
-
 template <int KE>
-__global__ void __launch_bounds__(EP_ROWS)
-epilogue_kernel(int mode, int64_t n, int k, const float* __restrict__ part, int splits,
-                const float* __restrict__ H, const float* __restrict__ G,
-                float* __restrict__ Hn, float* __restrict__ Gn, float* __restrict__ Psnap,
-                float m_scale, float lr, float eps, double* __restrict__ tr_part,
-                double* __restrict__ gram_part, float* __restrict__ Y,
-                const FitState* st, float* __restrict__ XT, int64_t ldxt) {
-    if (st != nullptr && st->done) return;
-    // As (k x k Gram, used by the step) and hs (new rows, used by the Gram
-    // partial) are live at different times and share one buffer.
+__global__ void __launch_bounds__(EP_ROWS) epilogue_kernel(const EpiArgs a) {
+    if (a.st != nullptr && a.st->done) return;
     constexpr int SM_FLOATS = KE * KE > EP_ROWS * (KE + 1) ? KE * KE : EP_ROWS * (KE + 1);
     __shared__ float smem[SM_FLOATS];
     __shared__ double red[EP_ROWS / 32];
-    float* As = smem;
-    float (*hs)[KE + 1] = reinterpret_cast<float (*)[KE + 1]>(smem);
-
-    const int tid = threadIdx.x;
-    const int64_t i = (int64_t)blockIdx.x * EP_ROWS + tid;
-    const bool valid = i < n;
-    const bool step = mode == MODE_FULL || mode == MODE_SVRG_INNER || mode == MODE_STEP_SNAP;
-
-    if (step) {
-        for (int e = tid; e < k * k; e += EP_ROWS) As[(e / k) * KE + (e % k)] = st->A32[e];
-        __syncthreads();
-    }
-
-    float p[KE], h[KE];
-#pragma unroll
-    for (int c = 0; c < KE; ++c) { p[c] = 0.f; h[c] = 0.f; }
-
-    if (valid) {
-        const int64_t row = i * (int64_t)k;
-        if (mode != MODE_GRAM && mode != MODE_STEP_SNAP) {
-            for (int s = 0; s < splits; ++s) {
-                const float* src = part + (int64_t)s * n * k + row;
-#pragma unroll
-                for (int c = 0; c < KE; ++c)
-                    if (c < k) p[c] += src[c];
-            }
-        }
-        if (mode == MODE_STEP_SNAP) {
-#pragma unroll
-            for (int c = 0; c < KE; ++c)
-                if (c < k) p[c] = Psnap[row + c];
-        } else if (mode == MODE_SVRG_INNER) {
-#pragma unroll
-            for (int c = 0; c < KE; ++c)
-                if (c < k) p[c] = fmaf(m_scale, p[c], Psnap[row + c]);
-        }
-        if (mode == MODE_PRODUCT) {
-#pragma unroll
-            for (int c = 0; c < KE; ++c)
-                if (c < k) Y[row + c] = p[c];
-            return;
-        }
-        if (mode == MODE_SNAPSHOT) {
-#pragma unroll
-            for (int c = 0; c < KE; ++c)
-                if (c < k) Psnap[row + c] = p[c];
-        }
-#pragma unroll
-        for (int c = 0; c < KE; ++c)
-            if (c < k) h[c] = H[row + c];
-    }
-    if (mode == MODE_PRODUCT) return;
-
-    // trace partial: sum_i sum_c H_ic (S H)_ic, fp64 (products of fp32 are exact)
-    if (mode == MODE_FULL || mode == MODE_SNAPSHOT) {
-        double tr = 0.0;
-#pragma unroll
-        for (int c = 0; c < KE; ++c) tr += (double)h[c] * (double)p[c];
-        const double tot = block_sum_fixed(tr, red);
-        if (tid == 0) tr_part[blockIdx.x] = tot;
-    }
-    if (mode == MODE_SNAPSHOT) return;
-
-    if (step && valid) {
-        const int64_t row = i * (int64_t)k;
-        float hnew[KE];
-#pragma unroll
-        for (int c = 0; c < KE; ++c) {
-            hnew[c] = 0.f;
-            if (c < k) {
-                float ha = 0.f;
-#pragma unroll
-                for (int d = 0; d < KE; ++d)
-                    if (d < k) ha = fmaf(h[d], As[d * KE + c], ha);
-                const float g = 4.f * (ha - p[c]);
-                const float gg = fmaf(g, g, G[row + c]);
-                const float stepv = __fdiv_rn(lr * g, __fadd_rn(__fsqrt_rn(gg), eps));
-                hnew[c] = fmaxf(h[c] - stepv, 0.f);
-                Gn[row + c] = gg;
-                Hn[row + c] = hnew[c];
-            }
-        }
-#pragma unroll
-        for (int c = 0; c < KE; ++c) h[c] = hnew[c];
-    }
-
-    // exact TF32 split [h_hi; h_lo] of the rows in h, the next S-stream's operand
-    if (XT != nullptr && valid && (mode == MODE_FULL || mode == MODE_STEP_SNAP || mode == MODE_GRAM)) {
-        const int K16 = (k + 15) / 16 * 16;
-#pragma unroll
-        for (int c = 0; c < KE; ++c) {
-            if (c < k) {
-                const float hb = __uint_as_float(__float_as_uint(h[c]) & 0xFFFFE000u);
-                XT[(int64_t)c * ldxt + i] = hb;
-                XT[(int64_t)(K16 + c) * ldxt + i] = h[c] - hb;
-            }
-        }
-    }
-
-    // Gram partial of the rows now in h (new iterate, or the given H for MODE_GRAM)
-    __syncthreads();  // every thread is done reading As
-#pragma unroll
-    for (int c = 0; c < KE; ++c) hs[tid][c] = valid ? h[c] : 0.f;
-    __syncthreads();
-    const int rows = (int)min64(EP_ROWS, n - (int64_t)blockIdx.x * EP_ROWS);
-    double* gp = gram_part + (int64_t)blockIdx.x * k * k;
-    for (int e = tid; e < k * k; e += EP_ROWS) {
-        const int c = e / k, d = e % k;
-        double a = 0.0;
-        for (int r = 0; r < rows; ++r) a += (double)hs[r][c] * (double)hs[r][d];
-        gp[e] = a;
-    }
+    epilogue_tile<KE, false>(a, blockIdx.x, threadIdx.x, smem, red);
 }
 
 int launch_epilogue(int mode, int64_t n, int k, const float* part, int splits,
@@ -322,10 +186,27 @@ int launch_epilogue(int mode, int64_t n, int k, const float* part, int splits,
                     double* tr_part, double* gram_part, float* Y,
                     const FitState* st, cudaStream_t s, float* XT, int64_t ldxt) {
     const int nb = epilogue_blocks(n);
-#define SYMNMF_EP(KE)                                                                 \
-    epilogue_kernel<KE><<<nb, EP_ROWS, 0, s>>>(mode, n, k, part, splits, H, G, Hn, Gn, \
-                                               Psnap, m_scale, lr, eps, tr_part,       \
-                                               gram_part, Y, st, XT, ldxt)
+    EpiArgs a;
+    a.mode = mode;
+    a.n = n;
+    a.k = k;
+    a.part = part;
+    a.splits = splits;
+    a.H = H;
+    a.G = G;
+    a.Hn = Hn;
+    a.Gn = Gn;
+    a.Psnap = Psnap;
+    a.m_scale = m_scale;
+    a.lr = lr;
+    a.eps = eps;
+    a.tr_part = tr_part;
+    a.gram_part = gram_part;
+    a.Y = Y;
+    a.st = st;
+    a.XT = XT;
+    a.ldxt = ldxt;
+#define SYMNMF_EP(KE) epilogue_kernel<KE><<<nb, EP_ROWS, 0, s>>>(a)
     if (k <= 8) SYMNMF_EP(8);
     else if (k <= 16) SYMNMF_EP(16);
     else if (k <= 24) SYMNMF_EP(24);
@@ -364,10 +245,16 @@ reduce_finalize_kernel(int mode, int nblk, int k, const double* __restrict__ tr_
 
     if ((int)blockIdx.x < gram_blocks) {
         const int e = blockIdx.x * 32 + l;
-        double a = 0.0;
-        if (e < kk)
-            for (int b = w; b < nblk; b += 8) a += gram_part[(int64_t)b * kk + e];
-        sh[w][l] = a;
+        double a0 = 0.0, a1 = 0.0;
+        if (e < kk) {
+            int b = w;
+            for (; b + 8 < nblk; b += 16) {
+                a0 += gram_part[(int64_t)b * kk + e];
+                a1 += gram_part[(int64_t)(b + 8) * kk + e];
+            }
+            if (b < nblk) a0 += gram_part[(int64_t)b * kk + e];
+        }
+        sh[w][l] = a0 + a1;
         __syncthreads();
         if (w == 0 && e < kk) {
             double t = 0.0;
@@ -403,9 +290,7 @@ reduce_finalize_kernel(int mode, int nblk, int k, const double* __restrict__ tr_
         const int t = st->t;
         bool stop = false;
         if (eval) {
-            double asq = 0.0;
-            for (int e = 0; e < kk; ++e) asq += st->A64[e] * st->A64[e];
-            const double L = st->s_sqnorm - 2.0 * fs->tr + asq;
+            const double L = st->s_sqnorm - 2.0 * __ldcg(&fs->tr) + st->a_sqnorm;
             if (t < history_cap && history != nullptr) history[t] = L;
             if (!isfinite(L)) {
                 st->nonfinite = 1;
@@ -433,11 +318,22 @@ reduce_finalize_kernel(int mode, int nblk, int k, const double* __restrict__ tr_
     }
     __syncthreads();
     if (gram && !st->done) {
+        double q = 0.0;
         for (int e = threadIdx.x; e < kk; e += RF_THREADS) {
-            const double v = fs->A_next[e];
+            const double v = __ldcg(&fs->A_next[e]);
             st->A64[e] = v;
             st->A32[e] = (float)v;
+            q = fma(v, v, q);
         }
+        // ||A||^2 for the next evaluation, fixed-order block sum
+        __shared__ double qs[RF_THREADS];
+        qs[threadIdx.x] = q;
+        __syncthreads();
+        for (int o = RF_THREADS / 2; o > 0; o >>= 1) {
+            if ((int)threadIdx.x < o) qs[threadIdx.x] += qs[threadIdx.x + o];
+            __syncthreads();
+        }
+        if (threadIdx.x == 0) st->a_sqnorm = qs[0];
     }
 }
 

@@ -28,16 +28,33 @@
 //               the end reads D back and writes the partial row
 #include <cudaTypedefs.h>
 
+#include <cstring>
+
 #include "common.cuh"
+#include "epilogue.cuh"
 #include "sm100.cuh"
 
 namespace symnmf {
 
+// Pipeline shape (compile-time).  SYMNMF_TC_A_SMEM = 1: the first MMA reads S
+// straight from shared memory and relies on the tensor core truncating fp32
+// operands to TF32 (S_hi = trunc(S)); only S_lo goes through TMEM.
+#ifndef SYMNMF_TC_NS
+#define SYMNMF_TC_NS 4
+#endif
+#ifndef SYMNMF_TC_CHUNK
+#define SYMNMF_TC_CHUNK 2
+#endif
+#ifndef SYMNMF_TC_A_SMEM
+#define SYMNMF_TC_A_SMEM 0
+#endif
 constexpr int TC_BM = 128;                  // S rows per tile = TMEM lanes
 constexpr int TC_BK = 32;                   // columns per stage (128 bytes of fp32)
-constexpr int TC_NS = 4;                    // shared-memory stages
-constexpr int TC_NT = 2;                    // TMEM stages of the split S tile
-constexpr int TC_CHUNK = 2;                 // stages accumulated in TMEM before a drain
+constexpr int TC_NS = SYMNMF_TC_NS;         // shared-memory stages
+constexpr bool TC_A_SMEM = SYMNMF_TC_A_SMEM != 0;
+constexpr int TC_TSTAGE = TC_A_SMEM ? 32 : 64;   // TMEM columns per stage of the split S tile
+constexpr int TC_NT = TC_A_SMEM ? 4 : 2;         // TMEM stages of the split S tile
+constexpr int TC_CHUNK = SYMNMF_TC_CHUNK;   // stages accumulated in TMEM before a drain
 constexpr int TC_THREADS = 256;
 constexpr uint32_t TC_A_BYTES = TC_BM * TC_BK * 4;
 
@@ -50,7 +67,7 @@ struct TcCfg {
     static constexpr uint32_t B_BYTES = N1 * TC_BK * 4;     // multiple of 1024
     static constexpr uint32_t STAGE = TC_A_BYTES + B_BYTES;
     static constexpr uint32_t COL_A = 4 * K16 <= 128 ? 128u : 256u;
-    static constexpr uint32_t TMEM_COLS = COL_A + TC_NT * 64 <= 256 ? 256u : 512u;
+    static constexpr uint32_t TMEM_COLS = COL_A + TC_NT * TC_TSTAGE <= 256 ? 256u : 512u;
     // with 512 TMEM columns only one CTA may be resident: ask for enough smem
     static constexpr uint32_t SMEM_MIN = TMEM_COLS == 512u ? 120u * 1024u : 0u;
     static constexpr uint32_t SMEM_RAW = TC_NS * STAGE + 1024;
@@ -62,11 +79,14 @@ __device__ __forceinline__ void tc_fail(int* err, volatile int* abort_flag, int 
     if (err != nullptr) atomicExch(err, code);
 }
 
+// Two CTAs per SM for k <= 32 (TMEM and shared memory allow it): registers
+// are capped at 128 per thread; one CTA per SM above that.
 template <int K16>
-__global__ void __launch_bounds__(TC_THREADS, 1)
+__global__ void __launch_bounds__(TC_THREADS, K16 <= 32 ? 2 : 1)
 stream_tc_kernel(const __grid_constant__ CUtensorMap mapS, const __grid_constant__ CUtensorMap mapX,
                  int64_t n, int k, int64_t j0, int64_t j1, int64_t jspan,
-                 float* __restrict__ part, int* __restrict__ err, const FitState* st) {
+                 float* __restrict__ part, int* __restrict__ err, const FitState* st,
+                 const EpiArgs epi, int* __restrict__ counters) {
     using Cfg = TcCfg<K16>;
     using namespace sm100;
     if (st != nullptr && st->done) return;
@@ -77,6 +97,8 @@ stream_tc_kernel(const __grid_constant__ CUtensorMap mapS, const __grid_constant
     __shared__ __align__(8) uint64_t bar_dfull[2], bar_dempty[2], bar_fin;
     __shared__ uint32_t tmem_base_sh;
     __shared__ volatile int abort_sh;
+    __shared__ int go_sh, last_sh;
+    __shared__ double red_sh[EP_ROWS / 32];
 
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(tc_smem_raw) + 1023) & ~uintptr_t(1023));
@@ -161,13 +183,20 @@ stream_tc_kernel(const __grid_constant__ CUtensorMap mapS, const __grid_constant
             }
             tc_fence_after();
             const uint32_t b_base = smem_u32(smemB + slot * Cfg::B_BYTES);
-            const uint32_t a_hi = tbase + Cfg::COL_A + (uint32_t)ts * 64u;
+            const uint32_t a_base = smem_u32(smemA + slot * TC_A_BYTES);
+            const uint32_t a_t = tbase + Cfg::COL_A + (uint32_t)ts * (uint32_t)TC_TSTAGE;
             const uint32_t d = tbase + (uint32_t)b * (uint32_t)Cfg::N1;
 #pragma unroll
             for (int kk = 0; kk < TC_BK / 8; ++kk) {
                 const uint64_t bd = umma_desc_sw128(b_base + (uint32_t)kk * 32u);
-                umma_tf32_ts(d, a_hi + (uint32_t)kk * 8u, bd, id1, (first && kk == 0) ? 0u : 1u);
-                umma_tf32_ts(d, a_hi + 32u + (uint32_t)kk * 8u, bd, id2, 1u);
+                const uint32_t acc0 = (first && kk == 0) ? 0u : 1u;
+                if (TC_A_SMEM) {
+                    umma_tf32_ss(d, umma_desc_sw128(a_base + (uint32_t)kk * 32u), bd, id1, acc0);
+                    umma_tf32_ts(d, a_t + (uint32_t)kk * 8u, bd, id2, 1u);
+                } else {
+                    umma_tf32_ts(d, a_t + (uint32_t)kk * 8u, bd, id1, acc0);
+                    umma_tf32_ts(d, a_t + 32u + (uint32_t)kk * 8u, bd, id2, 1u);
+                }
             }
             umma_commit(&bar_empty[slot]);
             umma_commit(&bar_tempty[ts]);
@@ -239,9 +268,13 @@ stream_tc_kernel(const __grid_constant__ CUtensorMap mapS, const __grid_constant
                     lo[c * 4 + u] = __float_as_uint(e[u] - __uint_as_float(hb));
                 }
             }
-            const uint32_t tcol = tbase + lane_off + Cfg::COL_A + (uint32_t)ts * 64u;
-            tmem_st_32x32b_x32(tcol, hi);
-            tmem_st_32x32b_x32(tcol + 32u, lo);
+            const uint32_t tcol = tbase + lane_off + Cfg::COL_A + (uint32_t)ts * (uint32_t)TC_TSTAGE;
+            if (TC_A_SMEM) {
+                tmem_st_32x32b_x32(tcol, lo);
+            } else {
+                tmem_st_32x32b_x32(tcol, hi);
+                tmem_st_32x32b_x32(tcol + 32u, lo);
+            }
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();
@@ -260,12 +293,31 @@ stream_tc_kernel(const __grid_constant__ CUtensorMap mapS, const __grid_constant
             if (lane == 0) tc_fail(err, &abort_sh, 5);
             alive = false;
         }
+        // ---- tail of the split warps: one decision for all four of them
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+        if (r == 0) go_sh = abort_sh == 0 ? 1 : 0;
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+        const bool go = go_sh != 0;
         const int64_t i = i0 + r;
-        if (alive && i < n) {
+        if (go && i < n) {
             float* out = part + (int64_t)split * n * k + i * (int64_t)k;
 #pragma unroll
             for (int c = 0; c < K16; ++c)
                 if (c < k) out[c] = acc[c];
+        }
+        if (go && counters != nullptr) {
+            // the last split CTA of this row tile runs the epilogue for it (no waiting:
+            // whoever arrives last finds every partial in place)
+            __threadfence();
+            asm volatile("bar.sync 1, 128;" ::: "memory");
+            if (r == 0) last_sh = atomicAdd(&counters[blockIdx.x], 1) == (int)gridDim.y - 1 ? 1 : 0;
+            asm volatile("bar.sync 1, 128;" ::: "memory");
+            if (last_sh) {
+                __threadfence();
+                epilogue_tile<K16, true>(epi, (int)blockIdx.x, r, reinterpret_cast<float*>(smem),
+                                         red_sh);
+                if (r == 0) counters[blockIdx.x] = 0;   // ready for the next pass
+            }
         }
     }
 
@@ -382,7 +434,13 @@ TcPlan plan_stream_tc(const Dev& d, int64_t n, int k, int64_t j0, int64_t j1) {
 size_t tc_partial_floats(const TcPlan& p) { return (size_t)p.splits * p.n * p.k; }
 
 int launch_stream_tc(const TcPlan& p, const float* S, int64_t lds, const float* XT, int64_t ldxt,
-                     float* part, int* err, const FitState* st, cudaStream_t s) {
+                     float* part, int* err, const FitState* st, cudaStream_t s,
+                     const EpiArgs* epi, int* counters) {
+    EpiArgs none;
+    std::memset(&none, 0, sizeof(none));
+    none.mode = -1;
+    const EpiArgs ea = epi != nullptr ? *epi : none;
+    int* cnt = epi != nullptr ? counters : nullptr;
     CUtensorMap mapS, mapX;
     SYMNMF_TRY(make_map(&mapS, S, p.n, p.n, lds, TC_BM));
     SYMNMF_TRY(make_map(&mapX, XT, p.n, 2 * p.K16, ldxt, (uint32_t)(2 * p.K16)));
@@ -393,7 +451,7 @@ int launch_stream_tc(const TcPlan& p, const float* S, int64_t lds, const float* 
         SYMNMF_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, \
                                              (int)TcCfg<K16>::SMEM));                          \
         kern<<<grid, TC_THREADS, TcCfg<K16>::SMEM, s>>>(mapS, mapX, p.n, p.k, p.j0, p.j1,      \
-                                                       p.jspan, part, err, st);               \
+                                                       p.jspan, part, err, st, ea, cnt);      \
     } while (0)
     switch (p.K16) {
         case 16: SYMNMF_TC(16); break;
