@@ -250,8 +250,8 @@ SYMNMF_API int symnmf_labels(const float* H, int64_t n, int k, int32_t* labels,
  * It takes no workspace and calls no allocating routine: its scratch (the
  * TF32 split of X and an error word) lives in a 4 MiB file-scope device array
  * that every GPU loading the library holds until exit.  Limit:
- * 2 * roundup(k, 16) * roundup(n, 32) + 64 <= 1,048,576 floats (for k = 24,
- * n <= 16,352); larger sizes return SYMNMF_ERR_INVALID_ARG.  The first call on
+ * 2 * roundup(k, 8) * roundup(n, 32) + 64 <= 1,048,576 floats (for k = 24,
+ * n <= 21,824); larger sizes return SYMNMF_ERR_INVALID_ARG.  The first call on
  * a device looks up the array's device address (cudaGetSymbolAddress) with
  * that device current; make that first call before any stream capture.
  * Every call shares the one array and it keeps the last call's contents:

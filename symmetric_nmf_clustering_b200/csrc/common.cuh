@@ -123,10 +123,10 @@ int launch_stream_partial(const StreamPlan& p, const float* S, int64_t lds,
 size_t fit_state_bytes();
 
 // Tensor-core S-stream (stream_tc.cu): X enters as its exact TF32 split
-// XT = [X_hi; X_lo] stored K-major (2*K16 rows of length ldxt, K16 = k rounded up to 16).
+// XT = [X_hi; X_lo] stored K-major (2*KP rows of length ldxt, KP = k rounded up to 8).
 struct TcPlan {
     int64_t n;
-    int k, K16;
+    int k, KP;
     int64_t j0, j1;   // contraction range, j0 a multiple of 32
     int64_t tiles;    // 128-row tiles of the output
     int splits;       // contraction splits
@@ -143,7 +143,8 @@ int launch_stream_tc(const TcPlan& p, const float* S, int64_t lds, const float* 
 int launch_split(const float* Xa, const float* Xb, int64_t ldx, int k, int64_t r0, int64_t r1,
                  int64_t jlo, int64_t jhi, float* XT, int64_t ldxt, cudaStream_t s);
 inline int64_t xt_ld(int64_t n) { return (n + 31) / 32 * 32; }
-inline int xt_rows(int k) { return 2 * ((k + 15) / 16 * 16); }
+inline int xt_kp(int k) { return (k + 7) / 8 * 8; }
+inline int xt_rows(int k) { return 2 * xt_kp(k); }
 
 int epilogue_blocks(int64_t n);
 int launch_epilogue(int mode, int64_t n, int k, const float* part, int splits,

@@ -163,13 +163,13 @@ __device__ void epilogue_tile(const EpiArgs& a, int tile, int tid, float* smem, 
     // exact TF32 split [h_hi; h_lo] of the rows in h, the next S-stream's operand
     if (a.XT != nullptr && valid &&
         (mode == MODE_FULL || mode == MODE_STEP_SNAP || mode == MODE_GRAM)) {
-        const int K16 = (k + 15) / 16 * 16;
+        const int KP = (k + 7) / 8 * 8;
 #pragma unroll
         for (int c = 0; c < KE; ++c) {
             if (c < k) {
                 const float hb = __uint_as_float(__float_as_uint(h[c]) & 0xFFFFE000u);
                 a.XT[(int64_t)c * a.ldxt + i] = hb;
-                a.XT[(int64_t)(K16 + c) * a.ldxt + i] = h[c] - hb;
+                a.XT[(int64_t)(KP + c) * a.ldxt + i] = h[c] - hb;
             }
         }
     }

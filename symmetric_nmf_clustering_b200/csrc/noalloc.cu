@@ -79,7 +79,7 @@ extern "C" int symnmf_sh_noalloc(const float* S, int64_t n, int64_t lds, const f
     const size_t need = noalloc_floats_needed(n, k);
     if (need > kNoAllocScratchFloats) {
         set_error("symnmf_sh_noalloc: n = %lld with k = %d needs %zu floats of static scratch; "
-                  "the limit is %zu (2 * roundup(k, 16) * roundup(n, 32) + 64 <= 1048576); "
+                  "the limit is %zu (2 * roundup(k, 8) * roundup(n, 32) + 64 <= 1048576); "
                   "use symnmf_sh with a workspace",
                   (long long)n, k, need, kNoAllocScratchFloats);
         return SYMNMF_ERR_INVALID_ARG;

@@ -17,15 +17,17 @@
 // Per CTA (256 threads, two CTAs per SM): a 128-row tile of S times the
 // contraction range of its split, in stages of 32 columns (128 bytes):
 //   warp 0      TMA producer: S tile (128 x 32, 128-byte swizzle) and the
-//               matching [X_hi; X_lo] tile (2*K16 x 32, K-major) per stage,
-//               K16 = k rounded up to 16 (an MMA with M = 128 and A in TMEM
-//               needs N to be a multiple of 16)
-//   warp 1      MMA issuer: per 8-column step, D[:, 0:2K16] += S_hi [X_hi;X_lo]
-//               and D[:, 0:K16] += S_lo X_hi, A operands read from TMEM
+//               matching [X_hi; X_lo] tile (2*KP x 32, K-major) per stage,
+//               KP = k rounded up to 8
+//   warp 1      MMA issuer: per 8-column step, D[:, 0:2KP] += S_hi [X_hi;X_lo]
+//               (A = the S tile in shared memory, truncated to TF32 by the
+//               tensor core) and D[:, 0:KP] += S_lo X_hi (A = S_lo in TMEM)
 //   warp 2      TMEM allocator
 //   warps 4-7   split warps: thread r reads row r of the S tile from shared
-//               memory, stores its hi and lo planes into TMEM lane r, and at
-//               the end reads D back and writes the partial row
+//               memory, stores its lo plane into TMEM lane r, folds the
+//               finished accumulator into fp32 registers every TC_CHUNK
+//               stages, writes the partial row, and -- in the last split CTA
+//               of the tile -- runs the epilogue (epilogue.cuh)
 #include <cudaTypedefs.h>
 
 #include <cstring>
@@ -37,8 +39,9 @@
 namespace symnmf {
 
 // Pipeline shape (compile-time).  SYMNMF_TC_A_SMEM = 1: the first MMA reads S
-// straight from shared memory and relies on the tensor core truncating fp32
-// operands to TF32 (S_hi = trunc(S)); only S_lo goes through TMEM.
+// straight from shared memory; the tensor core truncates fp32 operands to
+// TF32, which is exactly S_hi (measured on B200: bit-identical results to
+// storing S_hi in TMEM), so only S_lo goes through TMEM.
 #ifndef SYMNMF_TC_NS
 #define SYMNMF_TC_NS 4
 #endif
@@ -46,7 +49,10 @@ namespace symnmf {
 #define SYMNMF_TC_CHUNK 2
 #endif
 #ifndef SYMNMF_TC_A_SMEM
-#define SYMNMF_TC_A_SMEM 0
+#define SYMNMF_TC_A_SMEM 1
+#endif
+#ifndef SYMNMF_TC_L2HINT   // 1: S loads evict-first, the reused X operand evict-last
+#define SYMNMF_TC_L2HINT 1
 #endif
 constexpr int TC_BM = 128;                  // S rows per tile = TMEM lanes
 constexpr int TC_BK = 32;                   // columns per stage (128 bytes of fp32)
@@ -58,15 +64,21 @@ constexpr int TC_CHUNK = SYMNMF_TC_CHUNK;   // stages accumulated in TMEM before
 constexpr int TC_THREADS = 256;
 constexpr uint32_t TC_A_BYTES = TC_BM * TC_BK * 4;
 
-// TMEM columns: two accumulators D0, D1 of 2*K16 columns each, then the
+// TMEM columns: two accumulators D0, D1 of 2*KP columns each (32-column
+// aligned), then the
 // TC_NT stages of the split S tile (32 hi + 32 lo columns each).
-template <int K16>
+template <int KP>
 struct TcCfg {
-    static constexpr int N1 = 2 * K16;                      // [X_hi ; X_lo]
-    static constexpr int N2 = K16;                          // X_hi
+    // An MMA with M = 128 and A in TMEM needs N to be a multiple of 16.  N1 = 2 KP
+    // always is; N2 rounds KP up, and when it does the extra 8 rows of B are the
+    // first 8 rows of X_lo, so D[:, KP:KP+8] also collects S_lo X_lo for those
+    // columns -- a correct (smaller-order) term that the drain keeps.
+    static constexpr int N1 = 2 * KP;                       // [X_hi ; X_lo]
+    static constexpr int N2 = (KP + 15) / 16 * 16;          // X_hi (+ 8 rows of X_lo)
     static constexpr uint32_t B_BYTES = N1 * TC_BK * 4;     // multiple of 1024
     static constexpr uint32_t STAGE = TC_A_BYTES + B_BYTES;
-    static constexpr uint32_t COL_A = 4 * K16 <= 128 ? 128u : 256u;
+    static constexpr uint32_t DSTRIDE = (N1 + 31) / 32 * 32;   // accumulator buffers 32-column aligned
+    static constexpr uint32_t COL_A = 2 * DSTRIDE <= 128 ? 128u : 256u;
     static constexpr uint32_t TMEM_COLS = COL_A + TC_NT * TC_TSTAGE <= 256 ? 256u : 512u;
     // with 512 TMEM columns only one CTA may be resident: ask for enough smem
     static constexpr uint32_t SMEM_MIN = TMEM_COLS == 512u ? 120u * 1024u : 0u;
@@ -81,13 +93,13 @@ __device__ __forceinline__ void tc_fail(int* err, volatile int* abort_flag, int 
 
 // Two CTAs per SM for k <= 32 (TMEM and shared memory allow it): registers
 // are capped at 128 per thread; one CTA per SM above that.
-template <int K16>
-__global__ void __launch_bounds__(TC_THREADS, K16 <= 32 ? 2 : 1)
+template <int KP>
+__global__ void __launch_bounds__(TC_THREADS, TcCfg<KP>::TMEM_COLS == 256u ? 2 : 1)
 stream_tc_kernel(const __grid_constant__ CUtensorMap mapS, const __grid_constant__ CUtensorMap mapX,
                  int64_t n, int k, int64_t j0, int64_t j1, int64_t jspan,
                  float* __restrict__ part, int* __restrict__ err, const FitState* st,
                  const EpiArgs epi, int* __restrict__ counters) {
-    using Cfg = TcCfg<K16>;
+    using Cfg = TcCfg<KP>;
     using namespace sm100;
     if (st != nullptr && st->done) return;
 
@@ -144,6 +156,8 @@ stream_tc_kernel(const __grid_constant__ CUtensorMap mapS, const __grid_constant
     if (warp == 0 && lane == 0 && ksteps > 0) {
         // ---------------- TMA producer
         int issued = 0;
+        const uint64_t pol_s = SYMNMF_TC_L2HINT ? policy_evict_first() : 0;
+        const uint64_t pol_x = SYMNMF_TC_L2HINT ? policy_evict_last() : 0;
         for (int s = 0; s < ksteps; ++s) {
             if (abort_sh) break;
             const int slot = s % TC_NS;
@@ -154,8 +168,13 @@ stream_tc_kernel(const __grid_constant__ CUtensorMap mapS, const __grid_constant
             }
             mbar_arrive_expect_tx(&bar_full[slot], Cfg::STAGE);
             const int32_t x = (int32_t)(jb + (int64_t)s * TC_BK);
-            tma_load_2d(smemA + slot * TC_A_BYTES, &mapS, x, (int32_t)i0, &bar_full[slot]);
-            tma_load_2d(smemB + slot * Cfg::B_BYTES, &mapX, x, 0, &bar_full[slot]);
+            if (SYMNMF_TC_L2HINT) {
+                tma_load_2d_hint(smemA + slot * TC_A_BYTES, &mapS, x, (int32_t)i0, &bar_full[slot], pol_s);
+                tma_load_2d_hint(smemB + slot * Cfg::B_BYTES, &mapX, x, 0, &bar_full[slot], pol_x);
+            } else {
+                tma_load_2d(smemA + slot * TC_A_BYTES, &mapS, x, (int32_t)i0, &bar_full[slot]);
+                tma_load_2d(smemB + slot * Cfg::B_BYTES, &mapX, x, 0, &bar_full[slot]);
+            }
             ++issued;
         }
         if (abort_sh) {  // let the copies already issued land before the CTA exits
@@ -185,7 +204,7 @@ stream_tc_kernel(const __grid_constant__ CUtensorMap mapS, const __grid_constant
             const uint32_t b_base = smem_u32(smemB + slot * Cfg::B_BYTES);
             const uint32_t a_base = smem_u32(smemA + slot * TC_A_BYTES);
             const uint32_t a_t = tbase + Cfg::COL_A + (uint32_t)ts * (uint32_t)TC_TSTAGE;
-            const uint32_t d = tbase + (uint32_t)b * (uint32_t)Cfg::N1;
+            const uint32_t d = tbase + (uint32_t)b * Cfg::DSTRIDE;
 #pragma unroll
             for (int kk = 0; kk < TC_BK / 8; ++kk) {
                 const uint64_t bd = umma_desc_sw128(b_base + (uint32_t)kk * 32u);
@@ -211,9 +230,9 @@ stream_tc_kernel(const __grid_constant__ CUtensorMap mapS, const __grid_constant
         const int wl = warp & 3;
         const int r = wl * 32 + lane;
         const uint32_t lane_off = (uint32_t)(wl * 32) << 16;
-        float acc[K16];
+        float acc[KP];
 #pragma unroll
-        for (int c = 0; c < K16; ++c) acc[c] = 0.f;
+        for (int c = 0; c < KP; ++c) acc[c] = 0.f;
         bool alive = true;
 
         // fold accumulator D[q % 2] into acc (round-to-nearest fp32 adds); the
@@ -224,14 +243,14 @@ stream_tc_kernel(const __grid_constant__ CUtensorMap mapS, const __grid_constant
             if (!__all_sync(0xffffffffu, mbar_wait(&bar_dfull[b], (uint32_t)(q >> 1) & 1u)))
                 return false;
             tc_fence_after();
-            const uint32_t dcol = tbase + lane_off + (uint32_t)b * (uint32_t)Cfg::N1;
-            uint32_t v[2 * K16 / 8][8];
+            const uint32_t dcol = tbase + lane_off + (uint32_t)b * Cfg::DSTRIDE;
+            uint32_t v[2 * KP / 8][8];
 #pragma unroll
-            for (int g = 0; g < 2 * K16 / 8; ++g) tmem_ld_32x32b_x8(dcol + (uint32_t)g * 8u, v[g]);
+            for (int g = 0; g < 2 * KP / 8; ++g) tmem_ld_32x32b_x8(dcol + (uint32_t)g * 8u, v[g]);
             tmem_wait_ld();
 #pragma unroll
-            for (int c = 0; c < K16; ++c)
-                acc[c] += __uint_as_float(v[c / 8][c % 8]) + __uint_as_float(v[(K16 + c) / 8][c % 8]);
+            for (int c = 0; c < KP; ++c)
+                acc[c] += __uint_as_float(v[c / 8][c % 8]) + __uint_as_float(v[(KP + c) / 8][c % 8]);
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&bar_dempty[b]);
@@ -302,7 +321,7 @@ stream_tc_kernel(const __grid_constant__ CUtensorMap mapS, const __grid_constant
         if (go && i < n) {
             float* out = part + (int64_t)split * n * k + i * (int64_t)k;
 #pragma unroll
-            for (int c = 0; c < K16; ++c)
+            for (int c = 0; c < KP; ++c)
                 if (c < k) out[c] = acc[c];
         }
         if (go && counters != nullptr) {
@@ -314,7 +333,7 @@ stream_tc_kernel(const __grid_constant__ CUtensorMap mapS, const __grid_constant
             asm volatile("bar.sync 1, 128;" ::: "memory");
             if (last_sh) {
                 __threadfence();
-                epilogue_tile<K16, true>(epi, (int)blockIdx.x, r, reinterpret_cast<float*>(smem),
+                epilogue_tile<KP, true>(epi, (int)blockIdx.x, r, reinterpret_cast<float*>(smem),
                                          red_sh);
                 if (r == 0) counters[blockIdx.x] = 0;   // ready for the next pass
             }
@@ -330,17 +349,17 @@ stream_tc_kernel(const __grid_constant__ CUtensorMap mapS, const __grid_constant
 }
 
 // ----------------------------------------------------------------------------
-// [X_hi ; X_lo] in the K-major layout the MMA reads: XT[c][j] (c < K16) and
-// XT[K16 + c][j] for j in [jlo, jhi); X = Xa - Xb on rows [r0, r1) and zero
-// on the other rows of the range; rows c in [k, K16) of each half are zero.
+// [X_hi ; X_lo] in the K-major layout the MMA reads: XT[c][j] (c < KP) and
+// XT[KP + c][j] for j in [jlo, jhi); X = Xa - Xb on rows [r0, r1) and zero
+// on the other rows of the range; rows c in [k, KP) of each half are zero.
 // ----------------------------------------------------------------------------
 __global__ void split_kernel(const float* __restrict__ Xa, const float* __restrict__ Xb,
-                             int64_t ldx, int k, int K16, int64_t r0, int64_t r1, int64_t jlo,
+                             int64_t ldx, int k, int KP, int64_t r0, int64_t r1, int64_t jlo,
                              int64_t jhi, float* __restrict__ XT, int64_t ldxt) {
     const int64_t j = jlo + (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
     if (j >= jhi) return;
     const bool in = j >= r0 && j < r1;
-    for (int c = 0; c < K16; ++c) {
+    for (int c = 0; c < KP; ++c) {
         float x = 0.f;
         if (in && c < k) {
             x = Xa[j * ldx + c];
@@ -348,16 +367,16 @@ __global__ void split_kernel(const float* __restrict__ Xa, const float* __restri
         }
         const float h = __uint_as_float(__float_as_uint(x) & 0xFFFFE000u);
         XT[(int64_t)c * ldxt + j] = h;
-        XT[(int64_t)(K16 + c) * ldxt + j] = x - h;
+        XT[(int64_t)(KP + c) * ldxt + j] = x - h;
     }
 }
 
 int launch_split(const float* Xa, const float* Xb, int64_t ldx, int k, int64_t r0, int64_t r1,
                  int64_t jlo, int64_t jhi, float* XT, int64_t ldxt, cudaStream_t s) {
     if (jhi <= jlo) return SYMNMF_OK;
-    const int K16 = (k + 15) / 16 * 16;
+    const int KP = (k + 7) / 8 * 8;
     const int64_t len = jhi - jlo;
-    split_kernel<<<(unsigned)((len + 255) / 256), 256, 0, s>>>(Xa, Xb, ldx, k, K16, r0, r1, jlo,
+    split_kernel<<<(unsigned)((len + 255) / 256), 256, 0, s>>>(Xa, Xb, ldx, k, KP, r0, r1, jlo,
                                                               jhi, XT, ldxt);
     SYMNMF_LAUNCH_CHECK();
     return SYMNMF_OK;
@@ -406,7 +425,7 @@ TcPlan plan_stream_tc(const Dev& d, int64_t n, int k, int64_t j0, int64_t j1) {
     TcPlan p;
     p.n = n;
     p.k = k;
-    p.K16 = (k + 15) / 16 * 16;
+    p.KP = (k + 7) / 8 * 8;
     p.j0 = j0 / TC_BK * TC_BK;                                 // 128-byte aligned TMA x
     p.j1 = std::min<int64_t>(n, (j1 + TC_BK - 1) / TC_BK * TC_BK);
     p.tiles = (n + TC_BM - 1) / TC_BM;
@@ -443,20 +462,24 @@ int launch_stream_tc(const TcPlan& p, const float* S, int64_t lds, const float* 
     int* cnt = epi != nullptr ? counters : nullptr;
     CUtensorMap mapS, mapX;
     SYMNMF_TRY(make_map(&mapS, S, p.n, p.n, lds, TC_BM));
-    SYMNMF_TRY(make_map(&mapX, XT, p.n, 2 * p.K16, ldxt, (uint32_t)(2 * p.K16)));
+    SYMNMF_TRY(make_map(&mapX, XT, p.n, 2 * p.KP, ldxt, (uint32_t)(2 * p.KP)));
     dim3 grid((unsigned)p.tiles, (unsigned)p.splits);
-#define SYMNMF_TC(K16)                                                                         \
+#define SYMNMF_TC(KP)                                                                         \
     do {                                                                                      \
-        auto kern = stream_tc_kernel<K16>;                                                     \
+        auto kern = stream_tc_kernel<KP>;                                                     \
         SYMNMF_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, \
-                                             (int)TcCfg<K16>::SMEM));                          \
-        kern<<<grid, TC_THREADS, TcCfg<K16>::SMEM, s>>>(mapS, mapX, p.n, p.k, p.j0, p.j1,      \
+                                             (int)TcCfg<KP>::SMEM));                          \
+        kern<<<grid, TC_THREADS, TcCfg<KP>::SMEM, s>>>(mapS, mapX, p.n, p.k, p.j0, p.j1,      \
                                                        p.jspan, part, err, st, ea, cnt);      \
     } while (0)
-    switch (p.K16) {
+    switch (p.KP) {
+        case 8: SYMNMF_TC(8); break;
         case 16: SYMNMF_TC(16); break;
+        case 24: SYMNMF_TC(24); break;
         case 32: SYMNMF_TC(32); break;
+        case 40: SYMNMF_TC(40); break;
         case 48: SYMNMF_TC(48); break;
+        case 56: SYMNMF_TC(56); break;
         default: SYMNMF_TC(64); break;
     }
 #undef SYMNMF_TC

@@ -61,6 +61,6 @@ def test_noalloc_rejects_sizes_beyond_its_scratch():
     from symmetric_nmf_clustering_b200 import _lib
     lib = _lib.load()
     fake = 1 << 20   # never dereferenced: the size check comes first
-    # k = 24 -> K16 = 32: the limit is n <= 16,352
-    assert lib.symnmf_sh_noalloc(fake, 16353, 16356, fake, 24, fake, None) == _lib.SYMNMF_ERR_INVALID_ARG
+    # k = 24: 2 * 24 * roundup(n, 32) + 64 <= 1,048,576 allows n <= 21,824
+    assert lib.symnmf_sh_noalloc(fake, 21825, 21828, fake, 24, fake, None) == _lib.SYMNMF_ERR_INVALID_ARG
     assert b"static scratch" in lib.symnmf_last_error()
