@@ -168,6 +168,18 @@ def oracle_sample(name: str, seed: int, steps: int, warmup: int):
     }
 
 
+def job_rate(local_ms: float, units_per_rank: int, world: int, dist=None, device=None):
+    """Whole-job throughput of a weak-scaled run: every rank processed
+    `units_per_rank` units in `local_ms`; the job time is the max over ranks.
+    Returns (units per second over all ranks, job time in ms)."""
+    import torch
+    t = torch.tensor([float(local_ms)], dtype=torch.float64, device=device)
+    if world > 1 and dist is not None:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    t_max = float(t.item())
+    return world * units_per_rank / (t_max / 1000.0), t_max
+
+
 def _timed(torch, fn):
     a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     torch.cuda.synchronize()
@@ -309,11 +321,7 @@ def run_ours(args):
     barrier()
     clk = clocks.stop()
     t_ms = e0.elapsed_time(e1)
-    t_all = torch.tensor([t_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t_all, op=dist.ReduceOp.MAX)
-    t_max = float(t_all.item())
-    value = world * K / (t_max / 1000.0)
+    value, t_max = job_rate(t_ms, K, world, dist, dev)
 
     # dominant kernel: the S-stream, timed by events on its own stream inside the call
     launches = st["stream_launches"]
@@ -358,11 +366,8 @@ def run_ours(args):
         lab_host.copy_(m.labels(He), non_blocking=True)
         b.record()
         barrier()
-        te = torch.tensor([a.elapsed_time(b)], dtype=torch.float64, device=dev)
-        if world > 1:
-            dist.all_reduce(te, op=dist.ReduceOp.MAX)
-        te_ms = float(te.item())
-        e2e = {"value": world * K / (te_ms / 1000.0), "unit": UNIT,
+        e2e_value, te_ms = job_rate(a.elapsed_time(b), K, world, dist, dev)
+        e2e = {"value": e2e_value, "unit": UNIT,
                "h2d_bytes_per_step": int(R_pin.numel() * 4),
                "d2h_bytes_per_step": int(n * 4 + 8),
                "note": "per fit of K iterations: window upload, |corr| build, fit, labels+loss download"}

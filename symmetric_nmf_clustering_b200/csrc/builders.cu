@@ -5,9 +5,27 @@
 // Both end in a symmetric Gram S = c * op(Z^T Z) over the day index, computed
 // by one tiled kernel with the builder's epilogue (abs + unit diagonal for
 // correlation, the n/N scale for TPDM).
+#include <cstdlib>
+#include <cstring>
+
 #include "common.cuh"
 
 namespace symnmf {
+
+int launch_gram_tc(const float* ZF, const float* ZL, int64_t n, int64_t n_pad, int64_t Kp,
+                   bool corr, float scale, float* S, int64_t lds, int* err, cudaStream_t s);
+
+// Tensor-core Gram by default; SYMNMF_STREAM=cuda_core selects the CUDA-core one.
+static bool builders_tc() {
+    static int v = -1;
+    if (v < 0) {
+        const char* e = getenv("SYMNMF_STREAM");
+        v = (e != nullptr && std::strcmp(e, "cuda_core") == 0) ? 0 : 1;
+    }
+    return v == 1;
+}
+constexpr int TCB_ROWS = 128;   // row padding of the transposed operands
+constexpr int TCB_K = 32;       // contraction padding of the transposed operands
 
 constexpr int GB = 128;   // Gram output tile (GB x GB)
 constexpr int GK = 16;    // day-slab per stage
@@ -135,7 +153,10 @@ int corr_plan(Arena& a, int64_t T, int64_t n, double** mu, double** inv, float**
     const int64_t Kp = round_up(T, GK);
     *mu = a.take<double>(n);
     *inv = a.take<double>(n);
-    *Z = a.take<float>((size_t)Kp * *ldz);
+    // CUDA-core layout: Z (Kp x ldz); tensor-core layout: Z^T planes (n_pad x Kt) x 2 + err
+    const size_t cc = (size_t)Kp * *ldz;
+    const size_t tc = 2 * (size_t)round_up(n, TCB_ROWS) * round_up(T, TCB_K) + 64;
+    *Z = a.take<float>(std::max(cc, tc));
     return SYMNMF_OK;
 }
 
@@ -172,12 +193,49 @@ __global__ void normalize_kernel(const float* __restrict__ R, int64_t T, int64_t
     }
 }
 
+// Z^T planes for the tensor-core Gram: ZF[i][t] = z_ti (fp32) and
+// ZL[i][t] = z_ti - trunc_tf32(z_ti), zero in the padding (i >= n, t >= T).
+// 32 x 32 tiles through shared memory: coalesced reads of R rows, writes of ZT rows.
+__global__ void normalize_t_kernel(const float* __restrict__ R, int64_t T, int64_t n,
+                                   int64_t ldr, const double* __restrict__ mu,
+                                   const double* __restrict__ inv, float* __restrict__ ZF,
+                                   float* __restrict__ ZL, int64_t Kt) {
+    __shared__ float tile[32][33];
+    const int64_t t0 = (int64_t)blockIdx.y * 32, i0 = (int64_t)blockIdx.x * 32;
+    const int tx = threadIdx.x, ty = threadIdx.y;     // 32 x 8
+    for (int r = ty; r < 32; r += 8) {
+        const int64_t t = t0 + r, i = i0 + tx;
+        float z = 0.f;
+        if (t < T && i < n) z = (float)(((double)R[t * ldr + i] - mu[i]) * inv[i]);
+        tile[r][tx] = z;
+    }
+    __syncthreads();
+    for (int r = ty; r < 32; r += 8) {
+        const int64_t i = i0 + r, t = t0 + tx;
+        const float z = tile[tx][r];
+        const float hi = __uint_as_float(__float_as_uint(z) & 0xFFFFE000u);
+        ZF[i * Kt + t] = z;
+        ZL[i * Kt + t] = z - hi;
+    }
+}
+
 int launch_corr(const float* R, int64_t T, int64_t n, int64_t ldr, float* S,
                 int64_t lds, double* mu, double* inv, float* Z, int64_t ldz,
                 cudaStream_t s) {
-    const int64_t Kp = round_up(T, GK);
     colstats_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(R, T, n, ldr, mu, inv);
     SYMNMF_LAUNCH_CHECK();
+    if (builders_tc()) {
+        const int64_t n_pad = round_up(n, TCB_ROWS), Kt = round_up(T, TCB_K);
+        float* ZF = Z;
+        float* ZL = Z + (size_t)n_pad * Kt;
+        int* err = reinterpret_cast<int*>(ZL + (size_t)n_pad * Kt);
+        SYMNMF_CUDA_TRY(cudaMemsetAsync(err, 0, sizeof(int), s));
+        dim3 grid((unsigned)(n_pad / 32), (unsigned)(Kt / 32));
+        normalize_t_kernel<<<grid, dim3(32, 8), 0, s>>>(R, T, n, ldr, mu, inv, ZF, ZL, Kt);
+        SYMNMF_LAUNCH_CHECK();
+        return launch_gram_tc(ZF, ZL, n, n_pad, Kt, true, 1.f, S, lds, err, s);
+    }
+    const int64_t Kp = round_up(T, GK);
     const int64_t total = Kp * ldz;
     const int64_t blocks = min64((total + 255) / 256, 8192);
     normalize_kernel<<<(unsigned)blocks, 256, 0, s>>>(R, T, n, ldr, mu, inv, Z, ldz, Kp);
@@ -195,7 +253,9 @@ int tpdm_plan(Arena& a, int64_t T, int64_t n, int N, int32_t** ranks, double** p
     *phi = a.take<double>((size_t)T + 1);
     *rho = a.take<double>((size_t)T);
     *days = a.take<int32_t>((size_t)N);
-    *W = a.take<float>((size_t)round_up(N, GK) * *ldw);
+    const size_t cc = (size_t)round_up(N, GK) * *ldw;
+    const size_t tc = 2 * (size_t)round_up(n, TCB_ROWS) * round_up(N, TCB_K) + 64;
+    *W = a.take<float>(std::max(cc, tc));
     return SYMNMF_OK;
 }
 
@@ -302,6 +362,26 @@ __global__ void gather_w_kernel(const int32_t* __restrict__ ranks, const double*
     }
 }
 
+// W^T planes: WF[i][p] = phi[r_{days[p], i}] / rho_{days[p]} (fp32) and
+// WL = WF - trunc_tf32(WF); zero padding to n_pad x Kt.
+__global__ void gather_wt_kernel(const int32_t* __restrict__ ranks, const double* __restrict__ phi,
+                                 const double* __restrict__ rho, const int32_t* __restrict__ days,
+                                 int N, int64_t n, float* __restrict__ WF, float* __restrict__ WL,
+                                 int64_t n_pad, int64_t Kt) {
+    const int64_t total = n_pad * Kt;
+    for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < total;
+         e += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t i = e / Kt, p = e % Kt;
+        float v = 0.f;
+        if (p < N && i < n) {
+            const int64_t t = days[p];
+            v = (float)(phi[ranks[t * n + i]] / rho[t]);
+        }
+        WF[e] = v;
+        WL[e] = v - __uint_as_float(__float_as_uint(v) & 0xFFFFE000u);
+    }
+}
+
 int launch_tpdm(const float* R, int64_t T, int64_t n, int64_t ldr, int N,
                 int tail_sign, float* S, int64_t lds, int32_t* ranks, double* phi,
                 double* rho, int32_t* days, float* W, int64_t ldw, cudaStream_t s) {
@@ -323,12 +403,24 @@ int launch_tpdm(const float* R, int64_t T, int64_t n, int64_t ldr, int N,
     SYMNMF_LAUNCH_CHECK();
     select_kernel<<<(unsigned)((T + 255) / 256), 256, 0, s>>>(rho, T, N, days);
     SYMNMF_LAUNCH_CHECK();
+    const float scale = (float)((double)n / (double)N);
+    if (builders_tc()) {
+        const int64_t n_pad = round_up(n, TCB_ROWS), Kt = round_up(N, TCB_K);
+        float* WF = W;
+        float* WL = W + (size_t)n_pad * Kt;
+        int* err = reinterpret_cast<int*>(WL + (size_t)n_pad * Kt);
+        SYMNMF_CUDA_TRY(cudaMemsetAsync(err, 0, sizeof(int), s));
+        const int64_t total = n_pad * Kt;
+        const int64_t blocks = min64((total + 255) / 256, 8192);
+        gather_wt_kernel<<<(unsigned)blocks, 256, 0, s>>>(ranks, phi, rho, days, N, n, WF, WL, n_pad, Kt);
+        SYMNMF_LAUNCH_CHECK();
+        return launch_gram_tc(WF, WL, n, n_pad, Kt, false, scale, S, lds, err, s);
+    }
     const int64_t Np = round_up(N, GK);
     const int64_t total = Np * ldw;
     const int64_t blocks = min64((total + 255) / 256, 8192);
     gather_w_kernel<<<(unsigned)blocks, 256, 0, s>>>(ranks, phi, rho, days, N, n, W, ldw, Np);
     SYMNMF_LAUNCH_CHECK();
-    const float scale = (float)((double)n / (double)N);
     return launch_gram(W, ldw, (int)Np, n, S, lds, GRAM_TPDM, scale, s);
 }
 

@@ -1,0 +1,56 @@
+"""Multi-rank host logic of bench.py on the CPU (gloo, world size 2): the job
+time is the max over ranks, the value counts every rank's units, and the
+reference arm prints from rank 0 only."""
+import os
+import subprocess
+import sys
+
+import pytest
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _worker(rank, world, port, q):
+    import torch.distributed as dist
+    sys.path.insert(0, ROOT)
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    import bench
+    local_ms = 100.0 * (rank + 1)          # rank 1 is the slow one
+    value, t_max = bench.job_rate(local_ms, 50, world, dist, "cpu")
+    q.put((rank, value, t_max))
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+def test_job_rate_takes_max_over_ranks_gloo():
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = 29500 + (os.getpid() % 1000)
+    procs = [ctx.Process(target=_worker, args=(r, 2, port, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = sorted(q.get(timeout=120) for _ in procs)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    for rank, value, t_max in res:
+        assert t_max == 200.0                       # the slowest rank's time
+        assert value == pytest.approx(2 * 50 / 0.2)  # all ranks' units over the job time
+
+
+def test_job_rate_single_rank():
+    sys.path.insert(0, ROOT)
+    import bench
+    value, t_max = bench.job_rate(250.0, 100, 1)
+    assert (value, t_max) == (400.0, 250.0)
+
+
+def test_reference_arm_non_zero_rank_exits_silently():
+    env = dict(os.environ, RANK="1", WORLD_SIZE="2", LOCAL_RANK="1")
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                        "--steps", "3", "--warmup", "3", "--gpus", "2"],
+                       capture_output=True, text=True, env=env, timeout=300)
+    assert r.returncode == 0
+    assert r.stdout.strip() == ""
