@@ -248,10 +248,26 @@ static int check_params(const symnmf_fit_params& P, int64_t n, int k) {
 // ---------------------------------------------------------------- fit drivers
 struct Timing {
     bool on = false;
+    bool capturing = false;       // inside graph capture: records become graph nodes
     std::vector<cudaEvent_t> ev;  // pairs
     int used = 0;
     double ms = 0.0;
     int launches = 0;
+    int record(cudaEvent_t e, cudaStream_t s) {
+        if (capturing) SYMNMF_CUDA_TRY(cudaEventRecordWithFlags(e, s, cudaEventRecordExternal));
+        else SYMNMF_CUDA_TRY(cudaEventRecord(e, s));
+        return SYMNMF_OK;
+    }
+    // after a graph replay: the first `count` captured pairs did work
+    int harvest_pairs(int count) {
+        for (int i = 0; i < 2 * count && i + 1 < used; i += 2) {
+            float ms1 = 0.f;
+            SYMNMF_CUDA_TRY(cudaEventElapsedTime(&ms1, ev[i], ev[i + 1]));
+            ms += ms1;
+            ++launches;
+        }
+        return SYMNMF_OK;
+    }
     ~Timing() {
         for (auto e : ev) cudaEventDestroy(e);
     }
@@ -264,12 +280,11 @@ struct Timing {
             ev.push_back(a);
             ev.push_back(b);
         }
-        SYMNMF_CUDA_TRY(cudaEventRecord(ev[used], s));
-        return SYMNMF_OK;
+        return record(ev[used], s);
     }
     int end(cudaStream_t s) {
         if (!on) return SYMNMF_OK;
-        SYMNMF_CUDA_TRY(cudaEventRecord(ev[used + 1], s));
+        SYMNMF_TRY(record(ev[used + 1], s));
         used += 2;
         return SYMNMF_OK;
     }
@@ -405,6 +420,98 @@ static int full_pass(FitCtx& c, int mode, int max_evals, bool xt_ready) {
                            c.P->rel_tol, max_evals, c.L.hist, c.L.hist_cap, c.s);
 }
 
+static bool use_graphs() {
+    static int v = -1;
+    if (v < 0) {
+        const char* e = getenv("SYMNMF_GRAPHS");
+        v = (e != nullptr && std::strcmp(e, "0") == 0) ? 0 : 1;
+    }
+    return v == 1;
+}
+
+// Replays a captured graph of G full-batch passes on a private stream (ordered
+// after the caller's stream) until the device raises the stop flag.  Returns
+// SYMNMF_OK with *used = false when the graph could not be built; the caller
+// then continues eagerly.
+static int run_full_graph(FitCtx& c, int G, int max_evals, HostState* hs, bool* used) {
+    *used = false;
+    cudaStream_t user = c.s, cs = nullptr;
+    cudaEvent_t dep = nullptr;
+    cudaGraph_t graph = nullptr;
+    cudaGraphExec_t exec = nullptr;
+    if (cudaStreamCreateWithFlags(&cs, cudaStreamNonBlocking) != cudaSuccess ||
+        cudaEventCreateWithFlags(&dep, cudaEventDisableTiming) != cudaSuccess) {
+        cudaGetLastError();
+        if (cs) cudaStreamDestroy(cs);
+        return SYMNMF_OK;
+    }
+    auto cleanup = [&]() {
+        if (exec) cudaGraphExecDestroy(exec);
+        if (graph) cudaGraphDestroy(graph);
+        if (dep) cudaEventDestroy(dep);
+        if (cs) cudaStreamDestroy(cs);
+        c.s = user;
+        c.tm.capturing = false;
+    };
+    // timing events for the captured passes, allocated before capture
+    if (c.tm.on) {
+        c.tm.used = 0;
+        while ((int)c.tm.ev.size() < 2 * G) {
+            cudaEvent_t a;
+            if (cudaEventCreate(&a) != cudaSuccess) { cleanup(); return SYMNMF_ERR_CUDA; }
+            c.tm.ev.push_back(a);
+        }
+    }
+    const int cur0 = c.cur;
+    const int launches_before = launches();   // captured launches are not real ones
+    c.s = cs;
+    c.tm.capturing = true;
+    bool ok = cudaStreamBeginCapture(cs, cudaStreamCaptureModeThreadLocal) == cudaSuccess;
+    for (int p = 0; ok && p < G; ++p) {
+        ok = full_pass(c, MODE_FULL, max_evals, true) == SYMNMF_OK;
+        c.cur ^= 1;
+    }
+    const bool ended = cudaStreamEndCapture(cs, &graph) == cudaSuccess;
+    c.tm.capturing = false;
+    c.cur = cur0;
+    const int per_replay = launches() - launches_before;
+    reset_launches();
+    for (int i = 0; i < launches_before; ++i) note_launch();
+    if (!ok || !ended || cudaGraphInstantiate(&exec, graph, 0) != cudaSuccess) {
+        cudaGetLastError();
+        clear_error();
+        cleanup();
+        if (c.tm.on) c.tm.used = 0;
+        return SYMNMF_OK;
+    }
+    *used = true;
+    SYMNMF_CUDA_TRY(cudaEventRecord(dep, user));
+    SYMNMF_CUDA_TRY(cudaStreamWaitEvent(cs, dep, 0));
+    int rc = SYMNMF_OK;
+    for (;;) {
+        const int t_before = hs->t;
+        if (cudaGraphLaunch(exec, cs) != cudaSuccess) {
+            set_error("cudaGraphLaunch failed: %s", cudaGetErrorString(cudaGetLastError()));
+            rc = SYMNMF_ERR_CUDA;
+            break;
+        }
+        for (int i = 0; i < per_replay; ++i) note_launch();
+        if ((rc = read_state(c.L.st, hs, cs)) != SYMNMF_OK) break;
+        if (c.tm.on && (rc = c.tm.harvest_pairs(std::min(G, hs->t - t_before))) != SYMNMF_OK) break;
+        if (hs->done) break;
+    }
+    // the caller's stream continues after the replays
+    if (rc == SYMNMF_OK) {
+        if (cudaEventRecord(dep, cs) != cudaSuccess || cudaStreamWaitEvent(user, dep, 0) != cudaSuccess) {
+            set_error("stream ordering after the graph failed");
+            rc = SYMNMF_ERR_CUDA;
+        }
+    }
+    if (c.tm.on) c.tm.used = 0;
+    cleanup();
+    return rc;
+}
+
 // Full-batch projected AdaGrad until the device-side stop flag is raised.
 static int run_full(FitCtx& c, int max_evals, HostState* hs) {
     SYMNMF_TRY(read_state(c.L.st, hs, c.s));
@@ -413,13 +520,26 @@ static int run_full(FitCtx& c, int max_evals, HostState* hs) {
     const int cur_begin = c.cur;
     const int iters_begin = c.iters;
     const int check = c.P->check_every;
+    const int G = std::max(2, (check + 1) / 2 * 2);   // passes per graph: even, so parity returns
+    bool graphed = false;
     for (int launched = 0;; ++launched) {
         SYMNMF_TRY(full_pass(c, MODE_FULL, max_evals, true));
         c.cur ^= 1;
-        if ((launched + 1) % check == 0 || t_begin + launched + 1 >= max_evals) {
+        const bool last = t_begin + launched + 1 >= max_evals;
+        if ((launched + 1) % check == 0 || last || launched == 0) {
             SYMNMF_TRY(read_state(c.L.st, hs, c.s));
             SYMNMF_TRY(c.tm.harvest());
             if (hs->done) break;
+            // after the first (eager) pass, replay graphs while enough passes remain
+            if (!graphed && use_graphs() && max_evals - hs->t > G) {
+                bool used = false;
+                SYMNMF_TRY(run_full_graph(c, G, max_evals, hs, &used));
+                graphed = true;
+                if (used) {
+                    if (hs->done) break;
+                    // the graph ran an even number of passes: parity is back where it was
+                }
+            }
         }
     }
     const int steps = hs->t_stop - t_begin;  // updates between the first and the returned evaluation

@@ -467,8 +467,12 @@ int launch_stream_tc(const TcPlan& p, const float* S, int64_t lds, const float* 
 #define SYMNMF_TC(KP)                                                                         \
     do {                                                                                      \
         auto kern = stream_tc_kernel<KP>;                                                     \
-        SYMNMF_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, \
-                                             (int)TcCfg<KP>::SMEM));                          \
+        static bool attr_set = false; /* once per process: keeps graph capture clean */        \
+        if (!attr_set) {                                                                      \
+            SYMNMF_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, \
+                                                 (int)TcCfg<KP>::SMEM));                      \
+            attr_set = true;                                                                  \
+        }                                                                                     \
         kern<<<grid, TC_THREADS, TcCfg<KP>::SMEM, s>>>(mapS, mapX, p.n, p.k, p.j0, p.j1,      \
                                                        p.jspan, part, err, st, ea, cnt);      \
     } while (0)

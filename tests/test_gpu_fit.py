@@ -189,3 +189,31 @@ def test_errors(m):
     with pytest.raises(_lib.SymNMFError) as e:
         m.fit(Sd, 2, ws=tiny)
     assert e.value.status == _lib.SYMNMF_ERR_WORKSPACE
+
+
+_EAGER_SCRIPT = r"""
+import sys, numpy as np, torch
+sys.path.insert(0, sys.argv[1])
+import symmetric_nmf_clustering_b200 as m
+S = torch.from_numpy(np.load(sys.argv[2])).cuda()
+H, st = m.fit(S, 8, seed=5, max_iters=70, rel_tol=0.0, history=True)
+np.save(sys.argv[3], H.cpu().numpy())
+np.save(sys.argv[4], st["history"])
+"""
+
+
+def test_graph_replay_matches_eager_launches(m, tmp_path):
+    import os
+    import subprocess
+    import sys
+    _, _, S = corr_problem(1200, 100, seed=13)
+    Hg, st, _ = _fit(m, S, 8, seed=5, max_iters=70, rel_tol=0.0)
+    np.save(tmp_path / "S.npy", S)
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = dict(os.environ, SYMNMF_GRAPHS="0")
+    r = subprocess.run([sys.executable, "-c", _EAGER_SCRIPT, root, str(tmp_path / "S.npy"),
+                        str(tmp_path / "H.npy"), str(tmp_path / "hist.npy")],
+                       env=env, capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0, r.stderr
+    assert np.array_equal(np.load(tmp_path / "H.npy"), Hg)
+    assert np.array_equal(np.load(tmp_path / "hist.npy"), st["history"])
