@@ -470,6 +470,84 @@ def adaptgrow(S, k, lr=0.1, eps=1e-10, max_iters=2000, rel_tol=1e-5, seed=0,
 
 
 # ---------------------------------------------------------------------------
+# spherical k-means (hard-label baseline)
+# ---------------------------------------------------------------------------
+
+KMEANS_STREAM = 0x5851F42D4C957F2D   # splitmix64 stream separation for the initial centroids
+
+
+def forgy_indices(n: int, k: int, seed: int) -> list:
+    """k distinct row indices: the first k entries of a Fisher-Yates shuffle of
+    0..n-1 driven upwards (position q swaps with q + r mod (n - q)) by the
+    splitmix64 stream seeded with seed XOR KMEANS_STREAM."""
+    state = (seed ^ KMEANS_STREAM) & MASK64
+    draws = splitmix64_stream(state, k)
+    perm = {}
+    out = []
+    for q in range(k):
+        j = q + draws[q] % (n - q)
+        vq, vj = perm.get(q, q), perm.get(j, j)
+        perm[q], perm[j] = vj, vq
+        out.append(perm[q])
+    return out
+
+
+@dataclass
+class KMeansResult:
+    labels: np.ndarray       # int32 [n], the last assignment
+    centroids: np.ndarray    # [k, n], unit rows
+    steps: int               # assignment steps taken
+    converged: bool          # the labels stopped changing
+    objective: list          # sum_i <x_i, c_{l_i}> at each assignment step
+    min_gap: list            # smallest best-minus-second score over the rows, per step
+
+
+def spherical_kmeans(S, k: int, seed: int = 0, max_iters: int = 100) -> KMeansResult:
+    """Spherical k-means on the L2-normalised rows of S ([CaS] "Spherical
+    k-means for direct hard clustering": cosine similarity on the normalised
+    rows of S).
+
+    x_i = S_i / ||S_i|| (a zero row stays zero); centroids start at the rows
+    ``forgy_indices(n, k, seed)``; each step assigns l_i = argmax_c <x_i, c_c>
+    (lowest index on ties) and stops when no label changed, else sets
+    c_c = sum_{l_i = c} x_i / ||.|| (an empty cluster keeps its centroid).
+    ``min_gap`` records how close each step came to a tie, so that a caller
+    comparing against another precision knows whether the labels are decided.
+    """
+    S = np.asarray(S, dtype=np.float64)
+    n = S.shape[0]
+    norms = np.sqrt((S * S).sum(axis=1))
+    X = np.where(norms[:, None] > 0, S / np.where(norms > 0, norms, 1.0)[:, None], 0.0)
+    C = X[forgy_indices(n, k, seed)].copy()
+    lab = None
+    objective, min_gap = [], []
+    steps = 0
+    converged = False
+    while steps < max_iters:
+        scores = X @ C.T
+        new = np.argmax(scores, axis=1).astype(np.int32)
+        steps += 1
+        objective.append(float(scores[np.arange(n), new].sum()))
+        if k > 1:
+            top2 = np.sort(scores, axis=1)[:, -2:]
+            min_gap.append(float((top2[:, 1] - top2[:, 0]).min()))
+        else:
+            min_gap.append(float("inf"))
+        if lab is not None and np.array_equal(new, lab):
+            converged = True
+            break
+        lab = new
+        for c in range(k):
+            members = lab == c
+            if members.any():
+                v = X[members].sum(axis=0)
+                nv = np.sqrt((v * v).sum())
+                if nv > 0:
+                    C[c] = v / nv
+    return KMeansResult(lab, C, steps, converged, objective, min_gap)
+
+
+# ---------------------------------------------------------------------------
 # labels and agreement
 # ---------------------------------------------------------------------------
 
@@ -530,5 +608,7 @@ PINS = {
     "top_eigenvalues": "block-of-ones closed form; sum = trace",
     "gap_ratio": "hand values",
     "labels": "hand cases with ties",
+    "spherical_kmeans": "objective non-decreasing; unit centroids; brute-force assignment; planted blocks recovered",
+    "forgy_indices": "distinct, in range; uniform first index",
     "ari": "sklearn.metrics.adjusted_rand_score; O(n^2) pair brute force",
 }
