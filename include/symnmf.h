@@ -79,7 +79,8 @@ enum {
     SYMNMF_OP_SPECTRAL_PROBE = 2,
     SYMNMF_OP_FIT = 3,
     SYMNMF_OP_SH = 4,
-    SYMNMF_OP_STATS = 5
+    SYMNMF_OP_STATS = 5,
+    SYMNMF_OP_SPHERICAL_KMEANS = 6
 };
 
 /*
@@ -237,6 +238,31 @@ SYMNMF_API int symnmf_fit(const float* S, int64_t n, int64_t lds, int k,
  */
 SYMNMF_API int symnmf_labels(const float* H, int64_t n, int k, int32_t* labels,
                   symnmf_stream_t stream);
+
+/*
+ * Spherical k-means on the L2-normalised rows x_i = S_i / ||S_i|| of S, the
+ * hard-label baseline of [CaS] "Spherical k-means for direct hard
+ * clustering" (cosine similarity; a zero row stays zero).
+ *   start:   centroid c = x_{r_c}, r_0..r_{k-1} the first k entries of a
+ *            Fisher-Yates shuffle of 0..n-1 taken upwards (position q swaps
+ *            with q + (z_q mod (n - q))), z_q the q-th splitmix64 output
+ *            seeded with seed XOR 0x5851F42D4C957F2D;
+ *   assign:  l_i = argmax_c <x_i, c_c>, lowest c on ties (one S pass:
+ *            S C^T, whose row i is ||S_i|| times the cosine scores);
+ *   stop:    when no label changed, or after max_iters assignment steps;
+ *   update:  c_c = sum_{l_i = c} x_i / ||.||; an empty cluster keeps its
+ *            centroid (one S pass: S M, M_ic = [l_i = c] / ||S_i||, by the
+ *            symmetry of S).
+ * S: n x n symmetric, 1 <= k <= min(64, n).  labels: n int32 (device), the
+ * last assignment.  centroids: n x k row-major fp32 (device; column c is
+ * centroid c) or NULL.  steps_host / converged_host (may be NULL): assignment
+ * steps taken and whether the labels stopped changing.  Synchronises `stream`
+ * once per step (to read the change count).
+ */
+SYMNMF_API int symnmf_spherical_kmeans(const float* S, int64_t n, int64_t lds, int k,
+                                       uint64_t seed, int max_iters, int32_t* labels,
+                                       float* centroids, int* steps_host, int* converged_host,
+                                       void* ws, size_t ws_bytes, symnmf_stream_t stream);
 
 /*
  * Y = S X like symnmf_sh, for callers that cannot allocate device memory

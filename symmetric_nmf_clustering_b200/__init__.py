@@ -3,6 +3,6 @@ AdaGrad / Block-SVRG factorisation and argmax labels behind a C ABI
 (include/symnmf.h, libsymnmf.so) with a thin PyTorch binding."""
 from . import _lib
 from .api import (alloc_S, build_corr, build_tpdm, fit, fit_params, labels, sh,  # noqa: F401
-                  spectral_probe, stats, workspace)
+                  spectral_probe, spherical_kmeans, stats, workspace)
 
 __version__ = "0.1.0"

@@ -21,7 +21,8 @@ SYMNMF_ERR_NOT_SUPPORTED = 6
 
 SOLVER_ADAGRAD, SOLVER_BLOCK_SVRG, SOLVER_AUTO = 0, 1, 2
 INIT_SEEDED, INIT_USER = 0, 1
-OP_BUILD_CORR, OP_BUILD_TPDM, OP_SPECTRAL_PROBE, OP_FIT, OP_SH, OP_STATS = range(6)
+(OP_BUILD_CORR, OP_BUILD_TPDM, OP_SPECTRAL_PROBE, OP_FIT, OP_SH, OP_STATS,
+ OP_SPHERICAL_KMEANS) = range(7)
 
 
 class FitParams(C.Structure):
@@ -93,6 +94,8 @@ SIGNATURES = {
                           _vp, _sz, _vp]),
     "symnmf_labels": (_int, [_vp, _i64, _int, _vp, _vp]),
     "symnmf_sh_noalloc": (_int, [_vp, _i64, _i64, _vp, _int, _vp, _vp]),
+    "symnmf_spherical_kmeans": (_int, [_vp, _i64, _i64, _int, C.c_uint64, _int, _vp, _vp,
+                                       C.POINTER(_int), C.POINTER(_int), _vp, _sz, _vp]),
 }
 
 _lib = None

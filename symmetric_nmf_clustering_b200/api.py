@@ -199,3 +199,23 @@ def labels(H: torch.Tensor) -> torch.Tensor:
     L.check("symnmf_labels", _lib().symnmf_labels(H.data_ptr(), n, k, out.data_ptr(),
                                                   _stream(H.device)))
     return out
+
+
+def spherical_kmeans(S: torch.Tensor, k: int, *, seed: int = 0, max_iters: int = 100,
+                     ws: torch.Tensor | None = None):
+    """Spherical k-means on the L2-normalised rows of S (cosine similarity).
+
+    Returns (labels int32 [n], centroids fp32 [n, k] with centroid c in column
+    c, assignment steps, converged).  Two passes over S per step.
+    """
+    n, _, lds = _matrix(S, "S")
+    labels_out = torch.empty(n, dtype=torch.int32, device=S.device)
+    cent = torch.empty((n, k), dtype=torch.float32, device=S.device)
+    ws = workspace(L.OP_SPHERICAL_KMEANS, n, k, device=S.device) if ws is None else ws
+    steps, conv = C.c_int(0), C.c_int(0)
+    L.check("symnmf_spherical_kmeans",
+            _lib().symnmf_spherical_kmeans(S.data_ptr(), n, lds, k, seed, max_iters,
+                                           labels_out.data_ptr(), cent.data_ptr(), C.byref(steps),
+                                           C.byref(conv), ws.data_ptr(), ws.numel(),
+                                           _stream(S.device)))
+    return labels_out, cent, steps.value, bool(conv.value)

@@ -7,6 +7,7 @@
 #include <cstdlib>
 #include <cstring>
 #include <limits>
+#include <unordered_map>
 #include <vector>
 
 #include "common.cuh"
@@ -1019,6 +1020,125 @@ static int probe_impl(const Dev& d, const float* S, int64_t n, int64_t lds, int 
 // =============================================================================
 using namespace symnmf;
 
+// ---------------------------------------------------------------- spherical k-means
+struct KmeansLayout {
+    double* inv_norm = nullptr;  // 1 / ||S_i||
+    float* CT = nullptr;         // centroids as columns (n x k), when the caller gives none
+    float* Y = nullptr;          // S C^T, then S M
+    float* M = nullptr;          // membership weights
+    int32_t* old = nullptr;      // previous labels
+    int64_t* idx = nullptr;      // starting rows
+    double* colsq = nullptr;     // per-block column sums of squares
+    int* count = nullptr;        // labels changed this step
+    StreamArgs sa{};
+};
+
+static void kmeans_plan(const Dev& d, Arena& a, int64_t n, int k, bool own_centroids,
+                        KmeansLayout* L) {
+    L->inv_norm = a.take<double>((size_t)n);
+    L->CT = own_centroids ? a.take<float>((size_t)n * k) : nullptr;
+    L->Y = a.take<float>((size_t)n * k);
+    L->M = a.take<float>((size_t)n * k);
+    L->old = a.take<int32_t>((size_t)n);
+    L->idx = a.take<int64_t>((size_t)k);
+    L->colsq = a.take<double>((size_t)km_colsq_blocks(n) * k);
+    L->count = a.take<int>(64);
+    L->sa.part = a.take<float>(stream_partials(d, n, k, 0, n));
+    L->sa.ldxt = xt_ld(n);
+    L->sa.XT = a.take<float>((size_t)xt_rows(k) * L->sa.ldxt);
+    L->sa.err = a.take<int>(64);
+    L->sa.counters = a.take<int>((size_t)epilogue_blocks(n));
+}
+
+// The first k entries of a Fisher-Yates shuffle of 0..n-1 taken upwards,
+// driven by splitmix64 seeded with seed ^ 0x5851F42D4C957F2D.
+static void forgy_rows(int64_t n, int k, uint64_t seed, std::vector<int64_t>& out) {
+    std::unordered_map<int64_t, int64_t> perm;  // sparse: only touched positions
+    auto at = [&](int64_t q) {
+        auto it = perm.find(q);
+        return it == perm.end() ? q : it->second;
+    };
+    uint64_t state = seed ^ 0x5851F42D4C957F2Dull;
+    out.resize(k);
+    for (int q = 0; q < k; ++q) {
+        state += 0x9E3779B97F4A7C15ull;
+        uint64_t z = state;
+        z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+        z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+        z ^= z >> 31;
+        const int64_t j = q + (int64_t)(z % (uint64_t)(n - q));
+        const int64_t vq = at(q), vj = at(j);
+        perm[q] = vj;
+        perm[j] = vq;
+        out[q] = vj;
+    }
+}
+
+static int kmeans_impl(const float* S, int64_t n, int64_t lds, int k, uint64_t seed,
+                       int max_iters, int32_t* labels, float* centroids, int* steps_host,
+                       int* converged_host, void* ws, size_t ws_bytes, cudaStream_t s) {
+    Dev d;
+    SYMNMF_TRY(device_info(&d));
+    Arena a;
+    a.base = static_cast<char*>(ws);
+    a.cap = ws_bytes;
+    KmeansLayout L;
+    kmeans_plan(d, a, n, k, centroids == nullptr, &L);
+    if (!a.ok()) {
+        set_error("workspace too small: %zu given, %zu needed", ws_bytes, a.used);
+        return SYMNMF_ERR_WORKSPACE;
+    }
+    float* CT = centroids != nullptr ? centroids : L.CT;
+    StreamArgs sa = L.sa;
+    sa.S = S;
+    sa.n = n;
+    sa.lds = lds;
+    sa.k = k;
+    sa.st = nullptr;
+
+    std::vector<int64_t> rows;
+    forgy_rows(n, k, seed, rows);
+    SYMNMF_CUDA_TRY(cudaMemcpyAsync(L.idx, rows.data(), (size_t)k * sizeof(int64_t),
+                                    cudaMemcpyHostToDevice, s));
+    SYMNMF_CUDA_TRY(cudaMemsetAsync(sa.err, 0, sizeof(int), s));
+    SYMNMF_CUDA_TRY(cudaMemsetAsync(sa.counters, 0, (size_t)epilogue_blocks(n) * sizeof(int), s));
+    SYMNMF_CUDA_TRY(cudaMemsetAsync(L.old, 0xFF, (size_t)n * sizeof(int32_t), s));  // no label
+    SYMNMF_TRY(launch_rownorm(S, n, lds, L.inv_norm, s));
+    SYMNMF_TRY(launch_init_centroids(S, n, lds, k, L.idx, L.inv_norm, CT, s));
+
+    int steps = 0, converged = 0;
+    while (steps < max_iters) {
+        // assignment: argmax_c of (S C^T)_ic = ||S_i|| <x_i, c_c>
+        SYMNMF_TRY(stream_pass(d, sa, CT, nullptr, k, 0, n, false, epi_product(n, k, L.Y), s,
+                               nullptr));
+        SYMNMF_TRY(launch_labels(L.Y, n, k, labels, s));
+        ++steps;
+        SYMNMF_CUDA_TRY(cudaMemsetAsync(L.count, 0, sizeof(int), s));
+        SYMNMF_TRY(launch_label_change(labels, L.old, n, L.count, s));
+        int changed = 0, err = 0;
+        SYMNMF_CUDA_TRY(cudaMemcpyAsync(&changed, L.count, sizeof(int), cudaMemcpyDeviceToHost, s));
+        SYMNMF_CUDA_TRY(cudaMemcpyAsync(&err, sa.err, sizeof(int), cudaMemcpyDeviceToHost, s));
+        SYMNMF_CUDA_TRY(cudaStreamSynchronize(s));
+        if (err != 0) {
+            set_error("a bounded device-side wait of the S-stream gave up (code %d)", err);
+            return SYMNMF_ERR_TIMEOUT;
+        }
+        if (changed == 0) {
+            converged = 1;
+            break;
+        }
+        // update: column c of S M is the sum of the normalised member rows
+        SYMNMF_TRY(launch_member(labels, L.inv_norm, n, k, L.M, s));
+        SYMNMF_TRY(stream_pass(d, sa, L.M, nullptr, k, 0, n, false, epi_product(n, k, L.Y), s,
+                               nullptr));
+        SYMNMF_TRY(launch_normalize_centroids(L.Y, n, k, L.colsq, CT, s));
+    }
+    SYMNMF_CUDA_TRY(cudaStreamSynchronize(s));
+    if (steps_host) *steps_host = steps;
+    if (converged_host) *converged_host = converged;
+    return SYMNMF_OK;
+}
+
 extern "C" {
 
 void symnmf_fit_params_default(symnmf_fit_params* p) {
@@ -1125,6 +1245,12 @@ int symnmf_workspace_size(int op, int64_t n, int k, int64_t T, const symnmf_fit_
         case SYMNMF_OP_STATS:
             a.take<double>((size_t)stats_blocks() * 3);
             break;
+        case SYMNMF_OP_SPHERICAL_KMEANS: {
+            SYMNMF_CHECK_ARG(k >= 1 && k <= KMAX, "k must be in [1, 64]");
+            KmeansLayout L;
+            kmeans_plan(d, a, n, k, true, &L);   // sized for the internal centroid buffer
+            break;
+        }
         default:
             set_error("unknown op %d", op);
             return SYMNMF_ERR_INVALID_ARG;
@@ -1288,6 +1414,22 @@ int symnmf_labels(const float* H, int64_t n, int k, int32_t* labels, symnmf_stre
     Dev d;
     SYMNMF_TRY(device_info(&d));
     return launch_labels(H, n, k, labels, (cudaStream_t)stream);
+}
+
+int symnmf_spherical_kmeans(const float* S, int64_t n, int64_t lds, int k, uint64_t seed,
+                            int max_iters, int32_t* labels, float* centroids, int* steps_host,
+                            int* converged_host, void* ws, size_t ws_bytes,
+                            symnmf_stream_t stream) {
+    clear_error();
+    SYMNMF_TRY(check_S(S, n, lds));
+    SYMNMF_CHECK_ARG(k >= 1 && k <= KMAX && k <= n, "k = %d must be in [1, min(64, n)]", k);
+    SYMNMF_CHECK_ARG(max_iters >= 1, "max_iters must be >= 1");
+    SYMNMF_CHECK_ARG(labels != nullptr, "labels must not be NULL");
+    SYMNMF_CHECK_ARG(centroids == nullptr || aligned4(centroids), "centroids must be a device pointer");
+    SYMNMF_CHECK_ARG(mul_ok(n, k), "n * k overflows");
+    SYMNMF_TRY(check_ws(ws, ws_bytes));
+    return kmeans_impl(S, n, lds, k, seed, max_iters, labels, centroids, steps_host,
+                       converged_host, ws, ws_bytes, (cudaStream_t)stream);
 }
 
 }  // extern "C"

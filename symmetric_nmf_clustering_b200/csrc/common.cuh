@@ -164,6 +164,16 @@ int stats_blocks();
 int launch_init(float* H, int64_t n, int k, uint64_t seed, const FitState* st,
                 cudaStream_t s);
 int launch_labels(const float* H, int64_t n, int k, int32_t* labels, cudaStream_t s);
+// spherical k-means pieces (kmeans.cu)
+int km_colsq_blocks(int64_t n);
+int launch_rownorm(const float* S, int64_t n, int64_t lds, double* inv_norm, cudaStream_t s);
+int launch_init_centroids(const float* S, int64_t n, int64_t lds, int k, const int64_t* idx,
+                          const double* inv_norm, float* CT, cudaStream_t s);
+int launch_member(const int32_t* lab, const double* inv_norm, int64_t n, int k, float* X,
+                  cudaStream_t s);
+int launch_normalize_centroids(const float* Z, int64_t n, int k, double* part, float* CT,
+                               cudaStream_t s);
+int launch_label_change(const int32_t* lab, int32_t* old, int64_t n, int* count, cudaStream_t s);
 
 // builders
 int corr_plan(Arena& a, int64_t T, int64_t n, double** mu, double** inv, float** Z,
