@@ -558,38 +558,137 @@ def labels(H: np.ndarray) -> np.ndarray:
     return np.argmax(np.asarray(H), axis=1).astype(np.int32)
 
 
-def _comb2(x):
-    x = np.asarray(x, dtype=np.int64)
-    return x * (x - 1) // 2
+def contingency(a, b, ka: int, kb: int) -> np.ndarray:
+    """n_ij = #{t : a_t = i, b_t = j} for labels a in [0, ka), b in [0, kb) (int64)."""
+    a = np.asarray(a, dtype=np.int64).ravel()
+    b = np.asarray(b, dtype=np.int64).ravel()
+    if a.size and (a.min() < 0 or a.max() >= ka or b.min() < 0 or b.max() >= kb):
+        raise ValueError("label out of range")
+    table = np.zeros((ka, kb), dtype=np.int64)
+    np.add.at(table, (a, b), 1)
+    return table
+
+
+def ari_from_table(table) -> float:
+    """Adjusted Rand index (Hubert & Arabie 1985) from a contingency table.
+
+    [CaS] "The metric": pair agreement corrected for chance, 1 for identical
+    clusterings and about 0 for unrelated ones.  The pair counts
+    I = sum C(n_ij, 2), A = sum C(a_i, 2), B = sum C(b_j, 2), P = C(n, 2) are
+    exact integers; then, in float64 and in this order,
+    e = (A * B) / P, m = (A + B) / 2, ARI = (I - e) / (m - e).
+    Returns 1.0 when P = 0 or the exact denominator (A + B) P - 2 A B is 0
+    (both labelings trivial).
+    """
+    t = np.asarray(table, dtype=np.int64)
+    n = int(t.sum())
+    comb = lambda x: sum(int(v) * (int(v) - 1) // 2 for v in np.asarray(x).ravel())
+    I, A, B = comb(t), comb(t.sum(axis=1)), comb(t.sum(axis=0))
+    P = n * (n - 1) // 2
+    if P == 0 or (A + B) * P - 2 * A * B == 0:
+        return 1.0
+    e = (float(A) * float(B)) / float(P)
+    m = (float(A) + float(B)) / 2.0
+    return (float(I) - e) / (m - e)
 
 
 def ari(a, b) -> float:
-    """Adjusted Rand index (Hubert & Arabie 1985) of two labelings.
-
-    [CaS] "The metric": pair agreement corrected for chance, 1 for identical
-    clusterings and about 0 for unrelated ones.  Pair counts are int64; one
-    final float64 division.  Returns 1.0 when the chance-corrected
-    denominator vanishes (both labelings trivial).
-    """
+    """Adjusted Rand index of two labelings (any integer label values)."""
     a = np.asarray(a).ravel()
     b = np.asarray(b).ravel()
-    n = a.size
     _, ai = np.unique(a, return_inverse=True)
     _, bi = np.unique(b, return_inverse=True)
-    table = np.zeros((ai.max() + 1, bi.max() + 1), dtype=np.int64)
-    np.add.at(table, (ai, bi), 1)
-    sum_ij = int(_comb2(table).sum())
-    sum_a = int(_comb2(table.sum(axis=1)).sum())
-    sum_b = int(_comb2(table.sum(axis=0)).sum())
-    total = n * (n - 1) // 2
-    if total == 0:
+    if a.size == 0:
         return 1.0
-    expected_num = sum_a * sum_b          # divided by total below
-    num = sum_ij * total - expected_num
-    den = (sum_a + sum_b) * total / 2 - expected_num
-    if den == 0:
-        return 1.0
-    return float(num / den)
+    return ari_from_table(contingency(ai, bi, int(ai.max()) + 1, int(bi.max()) + 1))
+
+
+# ---------------------------------------------------------------------------
+# rolling windows: stability, the control limit, the cross-sector monitor
+# ---------------------------------------------------------------------------
+
+def cross_sector_mean(S, groups, stressed) -> float:
+    """Mean of S_ij over the pairs (i, j) whose instruments sit in two
+    different stressed groups ([CaS] "Stability and break detection": the
+    cross-sector dependence among the stressed sectors, read off the
+    off-diagonal blocks of S)."""
+    S = np.asarray(S, dtype=np.float64)
+    groups = np.asarray(groups)
+    idx = [np.flatnonzero(groups == g) for g in stressed]
+    total, count = 0.0, 0
+    for a in range(len(idx)):
+        for b in range(len(idx)):
+            if a != b:
+                total += float(S[np.ix_(idx[a], idx[b])].sum())
+                count += len(idx[a]) * len(idx[b])
+    return total / count if count else float("nan")
+
+
+def control_limit(series, calib_windows):
+    """Self-calibrating 3-sigma limit ([CaS] "Stability and break detection"):
+    mean and sample standard deviation (ddof = 1) of the series over the calm
+    calibration windows (NaNs skipped); limit = mean - 3 * std."""
+    vals = np.array([series[t] for t in calib_windows if np.isfinite(series[t])], dtype=np.float64)
+    if vals.size < 2:
+        return float("nan"), float("nan"), float("nan")
+    mu = float(vals.mean())
+    sd = float(np.sqrt(((vals - mu) ** 2).sum() / (vals.size - 1)))
+    return mu, sd, mu - 3.0 * sd
+
+
+def rolling_pipeline(R, T: int, k: int, n_windows: int | None = None, stride: int = 1,
+                     kinds=("corr", "tpdm"), tail_frac: float = 0.05, tail_sign: int = 1,
+                     delta: int = 50, calib=None, groups=None, stressed=(), iters: int = 100,
+                     lr: float = 0.1, eps: float = 1e-10, seed: int = 0) -> dict:
+    """The rolling-window study ([CaS] "The temporal setup", "Tracking
+    stability through time", "Stability and break detection").
+
+    Window w holds days [w * stride, w * stride + T).  For each window and
+    each kind of dependence matrix: S = the matrix of that window (float64,
+    rounded to float32 as stored); an independent fit from the same
+    scale-matched seeded start ("Factorizing with SymNMF": fixed-seed
+    initialisation, no warm start), ``iters`` full-batch AdaGrad updates;
+    labels = row-wise argmax; ARI against the previous window and against
+    the window ``delta`` earlier; the cross-sector mean over ``stressed``
+    groups of ``groups``.  Then the 3-sigma limit of ARI(t - delta, t) over
+    the windows ``calib`` (default: every window with ARI(t - delta, t)) and
+    a flag on every window whose ARI(t - delta, t) falls below it.
+    """
+    R = np.asarray(R)
+    days, n = R.shape
+    W = (days - T) // stride + 1 if n_windows is None else n_windows
+    if W < 1 or (W - 1) * stride + T > days:
+        raise ValueError("windows do not fit in the stream")
+    out = {}
+    for kind in kinds:
+        lab = np.zeros((W, n), dtype=np.int32)
+        loss = np.zeros(W)
+        cross = np.full(W, np.nan)
+        for w in range(W):
+            Rw = R[w * stride: w * stride + T]
+            if kind == "corr":
+                S = corr_abs(Rw).astype(np.float32)
+            else:
+                S = tpdm(Rw, tail_frac, tail_sign).astype(np.float32)
+            if groups is not None and len(stressed) > 1:
+                cross[w] = cross_sector_mean(S, groups, stressed)
+            s_sum, sq, _ = stats(S)
+            H0 = scale_matched_init(s_sum, n, k, seed)
+            r = fit_adagrad(S, k, H0, lr=lr, eps=eps, max_iters=iters, rel_tol=0.0, S_sqnorm=sq)
+            lab[w] = labels(_f32(r.H))
+            loss[w] = r.loss
+        ari_prev = np.full(W, np.nan)
+        ari_delta = np.full(W, np.nan)
+        for w in range(1, W):
+            ari_prev[w] = ari_from_table(contingency(lab[w - 1], lab[w], k, k))
+            if w >= delta:
+                ari_delta[w] = ari_from_table(contingency(lab[w - delta], lab[w], k, k))
+        cw = range(delta, W) if calib is None else range(max(calib[0], delta), min(calib[1], W))
+        mu, sd, limit = control_limit(ari_delta, cw)
+        flags = np.array([np.isfinite(x) and x < limit for x in ari_delta], dtype=bool)
+        out[kind] = dict(labels=lab, loss=loss, cross=cross, ari_prev=ari_prev,
+                         ari_delta=ari_delta, mean=mu, std=sd, limit=limit, flags=flags)
+    return out
 
 
 # What pins each function in the CPU test suite (tests/test_oracle_*.py).
@@ -611,4 +710,8 @@ PINS = {
     "spherical_kmeans": "objective non-decreasing; unit centroids; brute-force assignment; planted blocks recovered",
     "forgy_indices": "distinct, in range; uniform first index",
     "ari": "sklearn.metrics.adjusted_rand_score; O(n^2) pair brute force",
+    "contingency": "loop count; row and column sums",
+    "cross_sector_mean": "pair loop brute force; planted constant blocks",
+    "control_limit": "hand values",
+    "rolling_pipeline": "windows equal standalone window runs; planted switch flagged, calm windows not",
 }

@@ -30,6 +30,8 @@ __all__ = [
     "workload",
     "uniform_h0",
     "planted_block_matrix",
+    "rolling_stream",
+    "RollingStream",
     "WORKLOADS",
 ]
 
@@ -138,3 +140,66 @@ def planted_block_matrix(sizes, order_seed: int | None = None):
         labels = labels[np.random.default_rng(order_seed).permutation(n)]
     S = (labels[:, None] == labels[None, :]).astype(np.float32)
     return S, labels
+
+
+class RollingStream:
+    """A synthetic daily return stream with a membership switch and a joint
+    tail shock (fields below), for the rolling-window pipeline."""
+
+    def __init__(self, R, groups_before, groups_after, switchers, stressed, spec):
+        self.R = R                          # days x n float32, row = day
+        self.groups_before = groups_before  # planted hard labels before the switch day
+        self.groups_after = groups_after    # ... from the switch day on
+        self.switchers = switchers          # instruments that change group
+        self.stressed = stressed            # groups hit by the joint tail shock
+        self.spec = spec
+
+
+def rolling_stream(seed: int = 0, n: int = 5000, g: int = 24, days: int = 499,
+                   sigma: float = 1.5, boundary: float = 0.1, switch_day: int = 250,
+                   switch_frac: float = 0.05, shock_days=(180, 200), shock_groups: int = 3,
+                   shock_scale: float = 1.0) -> RollingStream:
+    """The rolling workload's stream ("The temporal setup": planted groups, some
+    instruments changing group, several groups in a joint tail-stress episode
+    without changing membership).
+
+    r_d = B_d f_d + sigma * eps_d with f, eps iid N(0,1); B_d = B before
+    ``switch_day`` and B' from it on, where B' moves a seeded set of
+    round(switch_frac * n) instruments' whole loading onto another group drawn
+    uniformly from the rest.  On the days shock_days[0]..shock_days[1]
+    (inclusive) every member (planted label before the switch) of
+    ``shock_groups`` seeded groups gets -shock_scale * |z_d| added, z_d one
+    Student-t(2) draw per day shared by all of them: a joint crash, which
+    sits in the lower tail of the returns.  With the defaults a
+    250-day window starting at day w holds w post-switch days, so the labels
+    turn over around window 125.
+    """
+    rng = np.random.default_rng(seed)
+    B, before = planted_loadings(n, g, boundary, rng)
+    n_sw = int(round(switch_frac * n))
+    switchers = np.sort(rng.choice(n, size=n_sw, replace=False)) if n_sw else np.zeros(0, np.int64)
+    shift = rng.integers(1, g, size=n_sw) if g > 1 else np.zeros(n_sw, np.int64)
+    new_group = (before[switchers] + shift) % g
+    B_after = B.copy()
+    total = B[switchers].sum(axis=1)
+    B_after[switchers] = 0.0
+    B_after[switchers, new_group] = total
+    after = before.copy()
+    after[switchers] = new_group
+    stressed = np.sort(rng.choice(g, size=min(shock_groups, g), replace=False))
+    F = rng.standard_normal((days, g))
+    E = rng.standard_normal((days, n))
+    z = rng.standard_t(2.0, size=days)
+    R = np.empty((days, n), dtype=np.float64)
+    R[:switch_day] = F[:switch_day] @ B.T
+    R[switch_day:] = F[switch_day:] @ B_after.T
+    R += sigma * E
+    members = np.isin(before, stressed)
+    d0, d1 = shock_days
+    for d in range(max(d0, 0), min(d1 + 1, days)):
+        R[d, members] -= shock_scale * abs(z[d])
+    spec = dict(seed=seed, n=n, g=g, days=days, sigma=sigma, boundary=boundary,
+                switch_day=switch_day, switch_frac=switch_frac, shock_days=tuple(shock_days),
+                shock_groups=shock_groups, shock_scale=shock_scale)
+    return RollingStream(R.astype(np.float32), before, after, switchers, stressed, spec)
+

@@ -1,0 +1,125 @@
+"""Pins of the oracle's rolling-window pieces (CPU only): the contingency
+table, the cross-sector monitor, the 3-sigma control limit and the window
+pipeline itself."""
+import itertools
+
+import numpy as np
+import pytest
+
+import oracle
+import synth
+
+
+def test_contingency_by_loop():
+    rng = np.random.default_rng(0)
+    a = rng.integers(0, 5, 300)
+    b = rng.integers(0, 7, 300)
+    t = oracle.contingency(a, b, 5, 7)
+    for i in range(5):
+        for j in range(7):
+            assert t[i, j] == sum(1 for x, y in zip(a, b) if x == i and y == j)
+    assert t.sum() == 300
+    with pytest.raises(ValueError):
+        oracle.contingency([0, 5], [0, 0], 5, 1)
+
+
+def test_ari_from_table_special_cases():
+    # all in one cluster on both sides, all singletons on both sides, n <= 1
+    assert oracle.ari_from_table([[10]]) == 1.0
+    assert oracle.ari_from_table(np.eye(6, dtype=np.int64)) == 1.0
+    assert oracle.ari_from_table([[1]]) == 1.0
+    assert oracle.ari_from_table(np.zeros((2, 2), dtype=np.int64)) == 1.0
+    # one side trivial, the other not: no agreement beyond chance
+    assert oracle.ari_from_table([[3, 3]]) == 0.0
+
+
+def test_cross_sector_mean_brute_force():
+    rng = np.random.default_rng(1)
+    n = 30
+    A = rng.random((n, n))
+    S = A + A.T
+    groups = rng.integers(0, 5, n)
+    stressed = [1, 3, 4]
+    tot, cnt = 0.0, 0
+    for i, j in itertools.product(range(n), range(n)):
+        gi, gj = groups[i], groups[j]
+        if gi in stressed and gj in stressed and gi != gj:
+            tot += S[i, j]
+            cnt += 1
+    assert oracle.cross_sector_mean(S, groups, stressed) == pytest.approx(tot / cnt, rel=1e-13)
+
+
+def test_cross_sector_mean_planted_blocks():
+    # block constant c_ab between groups a != b, 1 inside a group
+    groups = np.repeat(np.arange(4), [5, 6, 7, 8])
+    c = np.array([[1, .2, .3, .4], [.2, 1, .5, .6], [.3, .5, 1, .7], [.4, .6, .7, 1]])
+    S = c[groups][:, groups]
+    sizes = {0: 5, 1: 6, 2: 7, 3: 8}
+    st = [0, 2, 3]
+    num = sum(c[a, b] * sizes[a] * sizes[b] for a in st for b in st if a != b)
+    den = sum(sizes[a] * sizes[b] for a in st for b in st if a != b)
+    assert oracle.cross_sector_mean(S, groups, st) == pytest.approx(num / den, rel=1e-14)
+
+
+def test_control_limit_hand_values():
+    mu, sd, lim = oracle.control_limit([np.nan, 1.0, 0.9, 0.8, 0.1], range(0, 4))
+    assert mu == pytest.approx(0.9) and sd == pytest.approx(0.1) and lim == pytest.approx(0.6)
+    assert np.isnan(oracle.control_limit([0.5], range(1))[2])
+
+
+def _small_stream(seed=0, sigma=0.3, days=80, switch_day=30, switch_frac=0.1, shock_scale=6.0):
+    return synth.rolling_stream(seed=seed, n=120, g=4, days=days, sigma=sigma, boundary=0.0,
+                                switch_day=switch_day, switch_frac=switch_frac,
+                                shock_days=(10, 14), shock_groups=2, shock_scale=shock_scale)
+
+
+def test_windows_equal_standalone_runs():
+    st = _small_stream()
+    T, k, W = 40, 4, 5
+    out = oracle.rolling_pipeline(st.R, T, k, n_windows=W, stride=3, kinds=("corr",), delta=2,
+                                  iters=30)
+    for w in (0, 4):
+        S = oracle.corr_abs(st.R[3 * w: 3 * w + T]).astype(np.float32)
+        s_sum, sq, _ = oracle.stats(S)
+        r = oracle.fit_adagrad(S, k, oracle.scale_matched_init(s_sum, 120, k, 0), max_iters=30)
+        assert np.array_equal(out["corr"]["labels"][w], oracle.labels(r.H))
+    assert np.isnan(out["corr"]["ari_prev"][0]) and np.isnan(out["corr"]["ari_delta"][1])
+    assert out["corr"]["ari_delta"][2] == pytest.approx(
+        oracle.ari(out["corr"]["labels"][0], out["corr"]["labels"][2]), abs=1e-15)
+
+
+def test_planted_switch_is_flagged_and_calm_windows_are_not():
+    # low noise and no shock: a window's labels are the planted membership of
+    # the days it holds, so ARI(t - delta, t) is 1 unless the two windows
+    # straddle the switch (day 80; windows of 40 days, w = 0..100)
+    st = _small_stream(sigma=0.3, days=140, switch_day=80, shock_scale=0.0)
+    T, delta = 40, 20
+    out = oracle.rolling_pipeline(st.R, T, 4, kinds=("corr",), delta=delta, calib=(20, 40),
+                                  iters=300)["corr"]
+    W = 140 - T + 1
+    assert oracle.ari(out["labels"][0], st.groups_before) == 1.0
+    assert oracle.ari(out["labels"][W - 1], st.groups_after) == 1.0
+    dipped = [w for w in range(delta, W) if out["ari_delta"][w] < 1.0]
+    # a dip needs window t to hold post-switch days (t > 40) and window t - delta
+    # to hold pre-switch days (t - delta < 80)
+    assert dipped and min(dipped) > 40 and max(dipped) < 100
+    assert out["ari_delta"][W - 1] == 1.0
+    # the calm windows show identical clusterings: the limit sits at 1
+    assert out["std"] == 0.0 and out["limit"] == 1.0
+    assert set(np.flatnonzero(out["flags"])) == set(dipped)
+
+
+# A check of the workload rather than of the oracle: the co-crash on days
+# 180-200 lifts the lower-tail TPDM's cross-sector block far more than the
+# correlation's ("Stability and break detection").  Seed 2 is left out: its
+# Student-t(2) draw on one shock day is large enough to dominate the
+# correlation as well.
+@pytest.mark.parametrize("seed", [0, 1, 3])
+def test_joint_crash_lifts_the_tail_matrix_more(seed):
+    st = synth.rolling_stream(seed=seed, n=480, switch_frac=0.0)
+    lift = {}
+    for kind, build in [("corr", oracle.corr_abs), ("tpdm", lambda R: oracle.tpdm(R, 0.05, -1))]:
+        calm = oracle.cross_sector_mean(build(st.R[249:499]), st.groups_before, st.stressed)
+        shock = oracle.cross_sector_mean(build(st.R[0:250]), st.groups_before, st.stressed)
+        lift[kind] = shock / calm
+    assert lift["tpdm"] > 1.5 and lift["tpdm"] > lift["corr"]
