@@ -80,8 +80,11 @@ enum {
     SYMNMF_OP_FIT = 3,
     SYMNMF_OP_SH = 4,
     SYMNMF_OP_STATS = 5,
-    SYMNMF_OP_SPHERICAL_KMEANS = 6
+    SYMNMF_OP_SPHERICAL_KMEANS = 6,
+    SYMNMF_OP_ARI = 7,
+    SYMNMF_OP_ROLLING = 8
 };
+enum { SYMNMF_KIND_CORR = 1, SYMNMF_KIND_TPDM = 2 };
 
 /*
  * Parameters of symnmf_fit ([SMI] AdaptGrow sketch: adaptgrow(S, k, lr, phi,
@@ -263,6 +266,82 @@ SYMNMF_API int symnmf_spherical_kmeans(const float* S, int64_t n, int64_t lds, i
                                        uint64_t seed, int max_iters, int32_t* labels,
                                        float* centroids, int* steps_host, int* converged_host,
                                        void* ws, size_t ws_bytes, symnmf_stream_t stream);
+
+/*
+ * Adjusted Rand index of two labelings ([CaS] "The metric": pair agreement
+ * corrected for chance; Hubert & Arabie).  a, b: n int32 labels in [0, k)
+ * (device), 1 <= k <= 64.  The k x k contingency table is counted on the GPU
+ * in exact integers; from it I = sum C(n_ij,2), A = sum C(a_i,2),
+ * B = sum C(b_j,2), P = C(n,2) (int64), then in float64 and in this order
+ * e = A*B/P, m = (A+B)/2, ARI = (I-e)/(m-e); 1.0 when P = 0 or
+ * (A+B)P - 2AB = 0.  Writes ari_host and, if not NULL, the table (k x k
+ * int64, row = label of a) to table_host.  A label outside [0, k) gives
+ * SYMNMF_ERR_INVALID_ARG.  Workspace: SYMNMF_OP_ARI.  Synchronises `stream`.
+ */
+SYMNMF_API int symnmf_ari(const int32_t* a, const int32_t* b, int64_t n, int k, double* ari_host,
+                          int64_t* table_host, void* ws, size_t ws_bytes, symnmf_stream_t stream);
+
+/*
+ * The rolling-window study ([CaS] "The temporal setup", "Tracking stability
+ * through time", "Stability and break detection").  Window w holds the days
+ * [w*stride, w*stride + window) of the returns stream R (days x n fp32,
+ * row = day, leading dimension ldr, device).  For every window and every
+ * kind of dependence matrix selected in `kinds`, in this order: build S
+ * (symnmf_build_corr / symnmf_build_tpdm) into the caller's n x n buffer;
+ * the cross-sector monitor, when n_stressed >= 2: the mean of S_ij over the
+ * pairs of instruments in two different stressed groups (group ids from
+ * `groups`, n int32 device); an independent fit from the same seeded start
+ * ("Factorizing with SymNMF": fixed-seed initialisation, no warm start) with
+ * the `fit` parameters; argmax labels into labels[kind] + w*n; ARI against
+ * window w-1 and window w-delta.  Then the 3-sigma control limit of
+ * ARI(t-delta, t): mean and sample standard deviation (n-1) over the
+ * calibration windows [calib_begin, calib_end) where it is defined,
+ * limit = mean - 3 std, and a flag on every window below the limit.
+ * Kind index 0 is |corr|, 1 is TPDM.
+ */
+typedef struct {
+    int64_t window;          /* T, days per window (>= 2); default 250 */
+    int64_t stride;          /* days between window starts (>= 1); default 1 */
+    int64_t n_windows;       /* windows to run; 0 = all that fit, (days - window)/stride + 1 */
+    int k;                   /* rank (1..64); default 24 */
+    int kinds;               /* SYMNMF_KIND_* bits; default both */
+    double tail_frac;        /* TPDM tail fraction; default 0.05 */
+    int tail_sign;           /* TPDM tail: -1 lower (joint crashes, default), +1 upper */
+    int delta;               /* ARI(t - delta, t) spacing (>= 1); default 50 */
+    int64_t calib_begin;     /* calibration windows [calib_begin, calib_end); */
+    int64_t calib_end;       /*   default 0, 0 = every window with ARI(t - delta, t) */
+    int n_stressed;          /* groups in the cross-sector monitor: 0 = off, else 2..8 */
+    int stressed[8];         /* their group ids */
+    symnmf_fit_params fit;   /* per-window fit; default ADAGRAD, 100 iterations, rel_tol 0 */
+} symnmf_rolling_params;
+
+typedef struct {             /* caller-owned outputs, [0] = |corr|, [1] = TPDM */
+    int32_t* labels[2];      /* device, n_windows x n: required for each selected kind */
+    double* ari_prev[2];     /* host, n_windows (NaN at window 0) or NULL */
+    double* ari_delta[2];    /* host, n_windows (NaN below delta) or NULL */
+    double* cross[2];        /* host, n_windows (NaN with the monitor off) or NULL */
+    double* loss[2];         /* host, n_windows: f(H) of each window's fit, or NULL */
+    uint8_t* flag[2];        /* host, n_windows: ARI(t - delta, t) < limit, or NULL */
+    double mean[2], std[2], limit[2];  /* written: the calibration (NaN if < 2 windows) */
+    int64_t n_windows;       /* written: windows run */
+    double build_ms[2];      /* written: CUDA-event time of the builders */
+    double fit_ms[2];        /* written: CUDA-event time of the fits and labels */
+    double total_ms;         /* written: CUDA-event time of the whole call */
+    int kernel_launches;     /* written: kernels launched */
+} symnmf_rolling_out;
+
+SYMNMF_API void symnmf_rolling_params_default(symnmf_rolling_params* p);
+
+/*
+ * Runs the study above.  S: the caller's n x n fp32 buffer (lds a multiple of
+ * 4), overwritten window by window.  groups may be NULL when n_stressed = 0.
+ * Workspace: SYMNMF_OP_ROLLING with T = window and params = &p->fit.
+ * Synchronises `stream` once per window and kind (the fit reads its state).
+ */
+SYMNMF_API int symnmf_rolling(const float* R, int64_t days, int64_t n, int64_t ldr,
+                              const int32_t* groups, float* S, int64_t lds,
+                              const symnmf_rolling_params* params, symnmf_rolling_out* out,
+                              void* ws, size_t ws_bytes, symnmf_stream_t stream);
 
 /*
  * Y = S X like symnmf_sh, for callers that cannot allocate device memory

@@ -637,9 +637,10 @@ def control_limit(series, calib_windows):
 
 
 def rolling_pipeline(R, T: int, k: int, n_windows: int | None = None, stride: int = 1,
-                     kinds=("corr", "tpdm"), tail_frac: float = 0.05, tail_sign: int = 1,
+                     kinds=("corr", "tpdm"), tail_frac: float = 0.05, tail_sign: int = -1,
                      delta: int = 50, calib=None, groups=None, stressed=(), iters: int = 100,
-                     lr: float = 0.1, eps: float = 1e-10, seed: int = 0) -> dict:
+                     lr: float = 0.1, eps: float = 1e-10, seed: int = 0, only=None,
+                     keep_H: bool = False) -> dict:
     """The rolling-window study ([CaS] "The temporal setup", "Tracking
     stability through time", "Stability and break detection").
 
@@ -653,23 +654,31 @@ def rolling_pipeline(R, T: int, k: int, n_windows: int | None = None, stride: in
     groups of ``groups``.  Then the 3-sigma limit of ARI(t - delta, t) over
     the windows ``calib`` (default: every window with ARI(t - delta, t)) and
     a flag on every window whose ARI(t - delta, t) falls below it.
+
+    ``only`` (a set of window indices) restricts the work to those windows:
+    the others keep label -1 and NaN entries, and an ARI needs both of its
+    windows.  ``keep_H`` also returns each window's factor (float32).
     """
     R = np.asarray(R)
     days, n = R.shape
     W = (days - T) // stride + 1 if n_windows is None else n_windows
     if W < 1 or (W - 1) * stride + T > days:
         raise ValueError("windows do not fit in the stream")
+    todo = set(range(W)) if only is None else {int(w) for w in only if 0 <= w < W}
     out = {}
     for kind in kinds:
-        lab = np.zeros((W, n), dtype=np.int32)
-        loss = np.zeros(W)
+        lab = np.full((W, n), -1, dtype=np.int32)
+        loss = np.full(W, np.nan)
         cross = np.full(W, np.nan)
-        for w in range(W):
+        smax = np.full(W, np.nan)
+        Hs = {}
+        for w in sorted(todo):
             Rw = R[w * stride: w * stride + T]
             if kind == "corr":
                 S = corr_abs(Rw).astype(np.float32)
             else:
                 S = tpdm(Rw, tail_frac, tail_sign).astype(np.float32)
+            smax[w] = float(np.abs(S).max())
             if groups is not None and len(stressed) > 1:
                 cross[w] = cross_sector_mean(S, groups, stressed)
             s_sum, sq, _ = stats(S)
@@ -677,17 +686,22 @@ def rolling_pipeline(R, T: int, k: int, n_windows: int | None = None, stride: in
             r = fit_adagrad(S, k, H0, lr=lr, eps=eps, max_iters=iters, rel_tol=0.0, S_sqnorm=sq)
             lab[w] = labels(_f32(r.H))
             loss[w] = r.loss
+            if keep_H:
+                Hs[w] = _f32(r.H)
         ari_prev = np.full(W, np.nan)
         ari_delta = np.full(W, np.nan)
         for w in range(1, W):
-            ari_prev[w] = ari_from_table(contingency(lab[w - 1], lab[w], k, k))
-            if w >= delta:
+            if w in todo and w - 1 in todo:
+                ari_prev[w] = ari_from_table(contingency(lab[w - 1], lab[w], k, k))
+            if w >= delta and w in todo and w - delta in todo:
                 ari_delta[w] = ari_from_table(contingency(lab[w - delta], lab[w], k, k))
         cw = range(delta, W) if calib is None else range(max(calib[0], delta), min(calib[1], W))
         mu, sd, limit = control_limit(ari_delta, cw)
         flags = np.array([np.isfinite(x) and x < limit for x in ari_delta], dtype=bool)
-        out[kind] = dict(labels=lab, loss=loss, cross=cross, ari_prev=ari_prev,
+        out[kind] = dict(labels=lab, loss=loss, cross=cross, smax=smax, ari_prev=ari_prev,
                          ari_delta=ari_delta, mean=mu, std=sd, limit=limit, flags=flags)
+        if keep_H:
+            out[kind]["H"] = Hs
     return out
 
 

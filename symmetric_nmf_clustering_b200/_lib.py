@@ -22,7 +22,8 @@ SYMNMF_ERR_NOT_SUPPORTED = 6
 SOLVER_ADAGRAD, SOLVER_BLOCK_SVRG, SOLVER_AUTO = 0, 1, 2
 INIT_SEEDED, INIT_USER = 0, 1
 (OP_BUILD_CORR, OP_BUILD_TPDM, OP_SPECTRAL_PROBE, OP_FIT, OP_SH, OP_STATS,
- OP_SPHERICAL_KMEANS) = range(7)
+ OP_SPHERICAL_KMEANS, OP_ARI, OP_ROLLING) = range(9)
+KIND_CORR, KIND_TPDM = 1, 2
 
 
 class FitParams(C.Structure):
@@ -75,6 +76,46 @@ class FitStats(C.Structure):
         return {name: getattr(self, name) for name, _ in self._fields_}
 
 
+class RollingParams(C.Structure):
+    _fields_ = [
+        ("window", C.c_int64),
+        ("stride", C.c_int64),
+        ("n_windows", C.c_int64),
+        ("k", C.c_int),
+        ("kinds", C.c_int),
+        ("tail_frac", C.c_double),
+        ("tail_sign", C.c_int),
+        ("delta", C.c_int),
+        ("calib_begin", C.c_int64),
+        ("calib_end", C.c_int64),
+        ("n_stressed", C.c_int),
+        ("stressed", C.c_int * 8),
+        ("fit", FitParams),
+    ]
+
+
+_P2 = lambda t: C.POINTER(t) * 2   # noqa: E731
+
+
+class RollingOut(C.Structure):
+    _fields_ = [
+        ("labels", C.c_void_p * 2),
+        ("ari_prev", _P2(C.c_double)),
+        ("ari_delta", _P2(C.c_double)),
+        ("cross", _P2(C.c_double)),
+        ("loss", _P2(C.c_double)),
+        ("flag", _P2(C.c_uint8)),
+        ("mean", C.c_double * 2),
+        ("std", C.c_double * 2),
+        ("limit", C.c_double * 2),
+        ("n_windows", C.c_int64),
+        ("build_ms", C.c_double * 2),
+        ("fit_ms", C.c_double * 2),
+        ("total_ms", C.c_double),
+        ("kernel_launches", C.c_int),
+    ]
+
+
 _vp, _i64, _int, _sz = C.c_void_p, C.c_int64, C.c_int, C.c_size_t
 
 # name -> (restype, argtypes); every symbol include/symnmf.h declares
@@ -96,6 +137,11 @@ SIGNATURES = {
     "symnmf_sh_noalloc": (_int, [_vp, _i64, _i64, _vp, _int, _vp, _vp]),
     "symnmf_spherical_kmeans": (_int, [_vp, _i64, _i64, _int, C.c_uint64, _int, _vp, _vp,
                                        C.POINTER(_int), C.POINTER(_int), _vp, _sz, _vp]),
+    "symnmf_ari": (_int, [_vp, _vp, _i64, _int, C.POINTER(C.c_double), C.POINTER(C.c_int64), _vp,
+                          _sz, _vp]),
+    "symnmf_rolling_params_default": (None, [C.POINTER(RollingParams)]),
+    "symnmf_rolling": (_int, [_vp, _i64, _i64, _i64, _vp, _vp, _i64, C.POINTER(RollingParams),
+                              C.POINTER(RollingOut), _vp, _sz, _vp]),
 }
 
 _lib = None

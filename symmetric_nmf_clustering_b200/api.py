@@ -219,3 +219,102 @@ def spherical_kmeans(S: torch.Tensor, k: int, *, seed: int = 0, max_iters: int =
                                            C.byref(conv), ws.data_ptr(), ws.numel(),
                                            _stream(S.device)))
     return labels_out, cent, steps.value, bool(conv.value)
+
+
+def ari(a: torch.Tensor, b: torch.Tensor, k: int, ws: torch.Tensor | None = None):
+    """Adjusted Rand index of two int32 labelings in [0, k) (device tensors).
+
+    Returns (ari, contingency table as a k x k int64 numpy array)."""
+    _check_cuda(a, "a", torch.int32)
+    _check_cuda(b, "b", torch.int32)
+    if a.numel() != b.numel():
+        raise ValueError("a and b must have the same length")
+    ws = workspace(L.OP_ARI, a.numel(), k, device=a.device) if ws is None else ws
+    out = C.c_double(0.0)
+    table = np.zeros((k, k), dtype=np.int64)
+    L.check("symnmf_ari", _lib().symnmf_ari(a.data_ptr(), b.data_ptr(), a.numel(), k, C.byref(out),
+                                            table.ctypes.data_as(C.POINTER(C.c_int64)),
+                                            ws.data_ptr(), ws.numel(), _stream(a.device)))
+    return out.value, table
+
+
+def rolling_params(**kw) -> "L.RollingParams":
+    """Rolling-study parameters: the library defaults overridden by ``kw``;
+    ``fit`` may be a dict of fit-parameter overrides."""
+    p = L.RollingParams()
+    _lib().symnmf_rolling_params_default(C.byref(p))
+    fit_kw = kw.pop("fit", {})
+    stressed = kw.pop("stressed", None)
+    for key, v in kw.items():
+        if not hasattr(p, key):
+            raise TypeError(f"unknown rolling parameter {key!r}")
+        setattr(p, key, v)
+    if stressed is not None:
+        stressed = [int(g) for g in stressed]
+        if len(stressed) > 8:
+            raise ValueError("at most 8 stressed groups")
+        p.n_stressed = len(stressed)
+        for i, g in enumerate(stressed):
+            p.stressed[i] = g
+    for key, v in fit_kw.items():
+        if not hasattr(p.fit, key):
+            raise TypeError(f"unknown fit parameter {key!r}")
+        setattr(p.fit, key, v)
+    return p
+
+
+def rolling(R: torch.Tensor, *, groups: torch.Tensor | None = None, S: torch.Tensor | None = None,
+            ws: torch.Tensor | None = None, **kw) -> dict:
+    """The rolling-window study over a device-resident returns stream R (days x n).
+
+    Keyword arguments are ``symnmf_rolling_params`` fields (window, stride,
+    n_windows, k, kinds, tail_frac, tail_sign, delta, calib_begin, calib_end,
+    stressed=[group ids], fit={...}).  Returns per kind ("corr", "tpdm") the
+    labels (device, n_windows x n), ari_prev, ari_delta, cross, loss, flags
+    (numpy), mean, std, limit, build_ms, fit_ms, plus total_ms and launches.
+    """
+    days, n, ldr = _matrix(R, "R")
+    p = rolling_params(**kw)
+    # output buffers; the library itself rejects windows that do not fit
+    W = max(1, p.n_windows if p.n_windows > 0 else (days - p.window) // max(p.stride, 1) + 1)
+    S = alloc_S(n, device=R.device) if S is None else S
+    _, _, lds = _matrix(S, "S")
+    if groups is not None:
+        _check_cuda(groups, "groups", torch.int32)
+    size = C.c_size_t(0)
+    L.check("symnmf_workspace_size",
+            _lib().symnmf_workspace_size(L.OP_ROLLING, n, p.k, p.window, C.byref(p.fit), C.byref(size)))
+    if ws is None:
+        ws = torch.empty(max(int(size.value), 256), dtype=torch.uint8, device=R.device)
+    out = L.RollingOut()
+    kinds = [("corr", L.KIND_CORR), ("tpdm", L.KIND_TPDM)]
+    res = {}
+    for c, (name, bit) in enumerate(kinds):
+        if not p.kinds & bit:
+            continue
+        r = dict(labels=torch.empty((W, n), dtype=torch.int32, device=R.device),
+                 ari_prev=np.zeros(W), ari_delta=np.zeros(W), cross=np.zeros(W), loss=np.zeros(W),
+                 flags=np.zeros(W, dtype=np.uint8))
+        out.labels[c] = r["labels"].data_ptr()
+        out.ari_prev[c] = r["ari_prev"].ctypes.data_as(C.POINTER(C.c_double))
+        out.ari_delta[c] = r["ari_delta"].ctypes.data_as(C.POINTER(C.c_double))
+        out.cross[c] = r["cross"].ctypes.data_as(C.POINTER(C.c_double))
+        out.loss[c] = r["loss"].ctypes.data_as(C.POINTER(C.c_double))
+        out.flag[c] = r["flags"].ctypes.data_as(C.POINTER(C.c_uint8))
+        res[name] = r
+    L.check("symnmf_rolling",
+            _lib().symnmf_rolling(R.data_ptr(), days, n, ldr,
+                                  groups.data_ptr() if groups is not None else None,
+                                  S.data_ptr(), lds, C.byref(p), C.byref(out), ws.data_ptr(),
+                                  ws.numel(), _stream(R.device)))
+    for c, (name, bit) in enumerate(kinds):
+        if name in res:
+            r = res[name]
+            r["flags"] = r["flags"].astype(bool)
+            r.update(mean=out.mean[c], std=out.std[c], limit=out.limit[c],
+                     build_ms=out.build_ms[c], fit_ms=out.fit_ms[c])
+    res["total_ms"] = out.total_ms
+    res["launches"] = out.kernel_launches
+    res["n_windows"] = out.n_windows
+    return res
+

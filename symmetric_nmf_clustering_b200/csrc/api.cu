@@ -1245,6 +1245,14 @@ int symnmf_workspace_size(int op, int64_t n, int k, int64_t T, const symnmf_fit_
         case SYMNMF_OP_STATS:
             a.take<double>((size_t)stats_blocks() * 3);
             break;
+        case SYMNMF_OP_ARI:
+            *bytes = ari_workspace_bytes();
+            return SYMNMF_OK;
+        case SYMNMF_OP_ROLLING: {
+            SYMNMF_CHECK_ARG(T >= 2, "T (the window) must be >= 2");
+            SYMNMF_TRY(check_params(P, n, k));
+            return rolling_workspace_bytes(d, n, k, T, P, bytes);
+        }
         case SYMNMF_OP_SPHERICAL_KMEANS: {
             SYMNMF_CHECK_ARG(k >= 1 && k <= KMAX, "k must be in [1, 64]");
             KmeansLayout L;

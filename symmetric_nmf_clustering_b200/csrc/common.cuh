@@ -164,6 +164,10 @@ int stats_blocks();
 int launch_init(float* H, int64_t n, int k, uint64_t seed, const FitState* st,
                 cudaStream_t s);
 int launch_labels(const float* H, int64_t n, int k, int32_t* labels, cudaStream_t s);
+// rolling windows (rolling.cu)
+size_t ari_workspace_bytes();
+int rolling_workspace_bytes(const Dev& d, int64_t n, int k, int64_t T, const symnmf_fit_params& P,
+                            size_t* bytes);
 // spherical k-means pieces (kmeans.cu)
 int km_colsq_blocks(int64_t n);
 int launch_rownorm(const float* S, int64_t n, int64_t lds, double* inv_norm, cudaStream_t s);

@@ -1,0 +1,170 @@
+"""GPU parity of symnmf_ari and symnmf_rolling against the CPU oracle.
+
+ARI: the contingency table is integer work (bit-exact) and the index is the
+same float64 expression on both sides, so the values must be bit-equal.
+
+Rolling study: both sides get the same returns stream; the GPU builds its own
+S, so the builders' rounding (per entry e_S = 5e-6 for |corr|, 1e-5 max|S|
+for TPDM) enters the fit.  Per window: labels equal wherever the oracle's
+top-two margin of H exceeds 1e-3 max|H| (the fit's H tolerance); loss within
+1e-4 (the fit's loss tolerance) plus 2 sqrt(f) n e_S, the most an entrywise
+perturbation of e_S moves f = ||S - H H^T||^2 to first order; cross-sector
+mean within e_S plus 1e-6 relative; an ARI bit-equal whenever both of its
+windows' label vectors are equal; the 3-sigma limit and flags equal when
+every calibration ARI is.
+"""
+import numpy as np
+import pytest
+
+import oracle
+import synth
+from gpu_util import to_dev
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda:0"
+
+
+@pytest.fixture(scope="module")
+def m():
+    import torch
+    from symmetric_nmf_clustering_b200 import build
+    build.build()
+    import symmetric_nmf_clustering_b200 as m
+    torch.cuda.init()
+    return m
+
+
+@pytest.mark.parametrize("n,k,seed", [(1, 1, 0), (5, 3, 1), (1000, 7, 2), (100003, 24, 3),
+                                      (4096, 64, 4)])
+def test_ari_bit_exact(m, n, k, seed):
+    rng = np.random.default_rng(seed)
+    a = rng.integers(0, k, n).astype(np.int32)
+    # b: a relabelled copy of a with a fraction of the rows redrawn
+    b = np.random.default_rng(seed + 100).permutation(k).astype(np.int32)[a]
+    flip = rng.random(n) < 0.2
+    b[flip] = rng.integers(0, k, int(flip.sum()))
+    v, table = m.ari(to_dev(a, DEV), to_dev(b, DEV), k)
+    ref_table = oracle.contingency(a, b, k, k)
+    assert np.array_equal(table, ref_table)
+    assert v == oracle.ari_from_table(ref_table)
+
+
+def test_ari_identical_and_trivial(m):
+    a = np.arange(50, dtype=np.int32) % 5
+    assert m.ari(to_dev(a, DEV), to_dev(a, DEV), 5)[0] == 1.0
+    z = np.zeros(50, dtype=np.int32)
+    assert m.ari(to_dev(z, DEV), to_dev(z, DEV), 5)[0] == 1.0
+    assert m.ari(to_dev(z, DEV), to_dev(a, DEV), 5)[0] == oracle.ari_from_table(
+        oracle.contingency(z, a, 5, 5))
+
+
+def test_ari_rejects_out_of_range_labels(m):
+    from symmetric_nmf_clustering_b200 import _lib as L
+    a = np.array([0, 1, 2, 5], dtype=np.int32)
+    with pytest.raises(L.SymNMFError) as e:
+        m.ari(to_dev(a, DEV), to_dev(a, DEV), 4)
+    assert "outside" in str(e.value)
+
+
+def _compare_windows(got, ref, k, windows, H, kind):
+    """Labels on the oracle's clear rows, loss, cross; returns windows whose
+    label vectors are fully equal."""
+    equal = set()
+    lab = got["labels"].cpu().numpy()
+    n = lab.shape[1]
+    for w in windows:
+        e_S = 5e-6 if kind == "corr" else 1e-5 * ref["smax"][w]
+        Hw = H[w]
+        srt = np.sort(Hw, axis=1)
+        clear = (srt[:, -1] - srt[:, -2]) > 1e-3 * np.abs(Hw).max()
+        assert np.array_equal(lab[w][clear], ref["labels"][w][clear]), w
+        assert (~clear).sum() <= max(3, 0.05 * len(clear)), w
+        if np.array_equal(lab[w], ref["labels"][w]):
+            equal.add(w)
+        f = ref["loss"][w]
+        assert abs(got["loss"][w] - f) <= 1e-4 * f + 2.0 * np.sqrt(f) * n * e_S, w
+        if np.isfinite(ref["cross"][w]):
+            c = ref["cross"][w]
+            assert abs(got["cross"][w] - c) <= e_S + 1e-6 * abs(c), w
+    return equal
+
+
+def _stream_small():
+    return synth.rolling_stream(seed=5, n=360, g=6, days=90, sigma=1.0, boundary=0.1,
+                                switch_day=45, switch_frac=0.1, shock_days=(5, 9),
+                                shock_groups=2, shock_scale=1.0)
+
+
+def test_rolling_parity_small(m):
+    st = _stream_small()
+    T, k, delta, iters = 60, 6, 10, 60
+    kw = dict(tail_frac=0.05, tail_sign=-1, delta=delta, calib=(10, 20), groups=st.groups_before,
+              stressed=list(st.stressed), iters=iters, seed=3)
+    ref = oracle.rolling_pipeline(st.R, T, k, keep_H=True, **kw)
+    R = to_dev(st.R, DEV, pad4=True)
+    groups = to_dev(st.groups_before.astype(np.int32), DEV)
+    got = m.rolling(R, groups=groups, window=T, k=k, delta=delta, calib_begin=10, calib_end=20,
+                    tail_frac=0.05, tail_sign=-1, stressed=list(st.stressed),
+                    fit=dict(max_iters=iters, seed=3))
+    W = 90 - T + 1
+    assert got["n_windows"] == W
+    for kind in ("corr", "tpdm"):
+        g, r = got[kind], ref[kind]
+        equal = _compare_windows(g, r, k, range(W), r["H"], kind)
+        for w in range(1, W):
+            if w in equal and w - 1 in equal:
+                assert g["ari_prev"][w] == r["ari_prev"][w], (kind, w)
+            if w >= delta and w in equal and w - delta in equal:
+                assert g["ari_delta"][w] == r["ari_delta"][w], (kind, w)
+        assert np.isnan(g["ari_prev"][0]) and np.all(np.isnan(g["ari_delta"][:delta]))
+        if all(w in equal and w - delta in equal for w in range(10, 20)):
+            assert g["mean"] == r["mean"] and g["std"] == r["std"] and g["limit"] == r["limit"]
+            assert np.array_equal(g["flags"], r["flags"])
+        assert g["build_ms"] > 0 and g["fit_ms"] > 0
+    assert got["launches"] > 0
+
+
+def test_rolling_kinds_and_stride(m):
+    st = _stream_small()
+    R = to_dev(st.R, DEV, pad4=True)
+    got = m.rolling(R, window=40, stride=7, k=6, kinds=1, delta=2, fit=dict(max_iters=20))
+    assert "tpdm" not in got and got["n_windows"] == (90 - 40) // 7 + 1
+    ref = oracle.rolling_pipeline(st.R, 40, 6, stride=7, kinds=("corr",), delta=2, iters=20,
+                                  keep_H=True)
+    _compare_windows(got["corr"], ref["corr"], 6, range(got["n_windows"]), ref["corr"]["H"], "corr")
+    assert np.all(np.isnan(got["corr"]["cross"]))
+
+
+def test_rolling_rejects_bad_arguments(m):
+    from symmetric_nmf_clustering_b200 import _lib as L
+    st = _stream_small()
+    R = to_dev(st.R, DEV, pad4=True)
+    for kw in [dict(window=100), dict(window=40, n_windows=60), dict(window=40, kinds=0),
+               dict(window=40, stressed=[1]), dict(window=40, delta=0)]:
+        with pytest.raises(L.SymNMFError):
+            m.rolling(R, k=6, **kw)
+
+
+def test_rolling_full_size_sampled_windows(m):
+    # the rolling workload at its full size: n = 5,000, k = 24, 250 windows of
+    # 250 days over 499 days, delta = 50; the oracle computes windows 0, 1,
+    # 124, 125 and 174 (both kinds) and the GPU run is compared there
+    st = synth.rolling_stream(seed=0)
+    R = to_dev(st.R, DEV, pad4=True)
+    groups = to_dev(st.groups_before.astype(np.int32), DEV)
+    got = m.rolling(R, groups=groups, window=250, k=24, delta=50, calib_begin=50, calib_end=125,
+                    tail_frac=0.05, tail_sign=-1, stressed=list(st.stressed))
+    assert got["n_windows"] == 250
+    sample = [0, 1, 124, 125, 174]
+    ref = oracle.rolling_pipeline(st.R, 250, 24, tail_frac=0.05, tail_sign=-1, delta=50,
+                                  groups=st.groups_before, stressed=list(st.stressed),
+                                  only=sample, keep_H=True)
+    for kind in ("corr", "tpdm"):
+        equal = _compare_windows(got[kind], ref[kind], 24, sample, ref[kind]["H"], kind)
+        for w in (1, 125):
+            if w in equal and w - 1 in equal:
+                assert got[kind]["ari_prev"][w] == ref[kind]["ari_prev"][w]
+        if 174 in equal and 124 in equal:
+            assert got[kind]["ari_delta"][174] == ref[kind]["ari_delta"][174]
+        a = got[kind]["ari_delta"]
+        assert np.all(np.isnan(a[:50])) and np.all((a[50:] >= -1.0) & (a[50:] <= 1.0))
