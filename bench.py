@@ -190,10 +190,11 @@ def _timed(torch, fn):
     return a.elapsed_time(b), out
 
 
-def measure_rows(m, torch, dev, S, H0, n, k, T, rank, workload):
+def measure_rows(m, torch, dev, S, H0, lab, n, k, T, rank, workload):
     """One timing per remaining row of the path on the resident |corr| matrix
-    (probe, labels, statistics) and on a TPDM of the heavy-tailed window of the
-    same size (builder, one Block-SVRG epoch)."""
+    (probe, labels, statistics, spherical k-means), on a TPDM of the
+    heavy-tailed window of the same size (builder, one Block-SVRG epoch), and
+    the rolling-window study at its own size (n = 5,000, 250 windows)."""
     out = {}
     # statistics pre-pass: one read of S
     ws = m.workspace(m._lib.OP_STATS, n, device=dev)
@@ -236,6 +237,46 @@ def measure_rows(m, torch, dev, S, H0, n, k, T, rank, workload):
         out["svrg_epochs"] = st["epochs"]
         del S2, wsf, Hs
         torch.cuda.empty_cache()
+    # spherical k-means on the resident |corr| matrix (two S passes per step),
+    # and its agreement with the SymNMF labels (the pages quote about 0.83 on
+    # their own data)
+    wsk = m.workspace(m._lib.OP_SPHERICAL_KMEANS, n, k, device=dev)
+    km_iters = 10
+    ms, (klab, _, ksteps, kconv) = _timed(
+        torch, lambda: m.spherical_kmeans(S, k, seed=rank, max_iters=km_iters, ws=wsk))
+    out["kmeans_ms"] = ms
+    out["kmeans_steps"] = ksteps
+    out["kmeans_ms_per_step"] = ms / max(ksteps, 1)
+    out["kmeans_S_GBs"] = (2 * ksteps - (1 if kconv else 0)) * 4.0 * n * n / (ms / 1e3) / 1e9
+    out["kmeans_vs_symnmf_ARI"] = m.ari(klab, lab, k)[0]
+    del wsk
+    # the rolling study: 250 windows of 250 days, |corr| and TPDM, 100-iteration
+    # fits, ARI series, 3-sigma limit, cross-sector monitor
+    st = synth.rolling_stream(seed=rank)
+    Rr = torch.from_numpy(st.R).to(dev)
+    groups = torch.from_numpy(st.groups_before.astype("int32")).to(dev)
+    kw = dict(groups=groups, window=250, k=24, delta=50, calib_begin=50, calib_end=125,
+              tail_frac=0.05, tail_sign=-1, stressed=list(st.stressed))
+    m.rolling(Rr, n_windows=2, **kw)                  # warm-up
+    ms, res = _timed(torch, lambda: m.rolling(Rr, **kw))
+    W = res["n_windows"]
+    out["rolling_windows"] = W
+    out["rolling_s"] = ms / 1e3
+    out["rolling_ms_per_window"] = ms / W
+    for kind in ("corr", "tpdm"):
+        r = res[kind]
+        ad = r["ari_delta"]
+        out[f"rolling_{kind}_build_ms_per_window"] = r["build_ms"] / W
+        out[f"rolling_{kind}_fit_ms_per_window"] = r["fit_ms"] / W
+        out[f"rolling_{kind}_calm_ari_delta"] = r["mean"]
+        out[f"rolling_{kind}_limit"] = r["limit"]
+        out[f"rolling_{kind}_flagged_windows"] = [int(w) for w in np.flatnonzero(r["flags"])][:12]
+        out[f"rolling_{kind}_min_ari_delta"] = float(np.nanmin(ad))
+        out[f"rolling_{kind}_cross_max"] = float(np.nanmax(r["cross"]))
+        out[f"rolling_{kind}_cross_last"] = float(r["cross"][-1])
+    out["rolling_kernel_launches"] = res["launches"]
+    del Rr, groups
+    torch.cuda.empty_cache()
     return out
 
 
@@ -368,15 +409,18 @@ def run_ours(args):
         barrier()
         e2e_value, te_ms = job_rate(a.elapsed_time(b), K, world, dist, dev)
         e2e = {"value": e2e_value, "unit": UNIT,
-               "h2d_bytes_per_step": int(R_pin.numel() * 4),
-               "d2h_bytes_per_step": int(n * 4 + 8),
-               "note": "per fit of K iterations: window upload, |corr| build, fit, labels+loss download"}
+               "h2d_bytes_per_step": int(R_pin.numel() * 4) / K,
+               "d2h_bytes_per_step": int(n * 4 + 8) / K,
+               "h2d_bytes_per_call": int(R_pin.numel() * 4),
+               "d2h_bytes_per_call": int(n * 4 + 8),
+               "note": "one call = window upload, |corr| build, K-iteration fit, labels + loss "
+                       "download; per-step bytes = per-call bytes / K"}
         del ws_corr
 
     # --- the other rows of the path, each timed once on this GPU (CUDA events)
     rows = None
     if not args.no_rows:
-        rows = measure_rows(m, torch, dev, S, H0, n, k, T, rank, args.workload)
+        rows = measure_rows(m, torch, dev, S, H0, lab, n, k, T, rank, args.workload)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -396,7 +440,7 @@ def run_ours(args):
                        "parallelism": f"independent windows x{world}" if world > 1 else "single"},
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak, "traffic": None,
-                         "kernel": "stream_partial_kernel", "peak_source": peak_src,
+                         "kernel": "stream_tc_kernel", "peak_source": peak_src,
                          "alg_bytes_per_launch": alg_bytes, "launch_ms": stream_ms,
                          "frac_of_8000": achieved / 8000.0},
             "s_stream_gbs": achieved,

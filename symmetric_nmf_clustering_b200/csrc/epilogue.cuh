@@ -198,3 +198,235 @@ __device__ void epilogue_tile(const EpiArgs& a, int tile, int tid, float* smem, 
 }
 
 }  // namespace symnmf
+
+namespace symnmf {
+
+// Shared-memory floats epilogue_tile_cta<KE> needs (tiles, Gram, reduction).
+template <int KE>
+constexpr size_t epilogue_cta_floats() {
+    return 3 * (size_t)EP_ROWS * KE + (size_t)KE * KE + 32;
+}
+
+// The same per-tile epilogue, run by all 256 threads of one CTA (the last
+// split CTA of the tile in the tensor-core stream kernel).  Global loads and
+// stores are coalesced through shared-memory tiles; each element sees the
+// same arithmetic as epilogue_tile (partials summed in split order, H A
+// accumulated in d order, the same AdaGrad expression), and each Gram entry
+// the same four-chain fp64 sum (products of fp32 values are exact in fp64, so
+// entry (c, d) equals entry (d, c) and is computed once).  The trace partial
+// is summed in a different, fixed order.
+// smem: epilogue_cta_floats<KE>() floats.  Callers: every thread of the CTA.
+template <int KE>
+__device__ void epilogue_tile_cta(const EpiArgs& a, int tile, int tid, float* smem) {
+    constexpr int NT = 256;
+    static_assert(EP_ROWS * KE % NT == 0, "whole elements per thread");
+    const int mode = a.mode;
+    const int64_t n = a.n;
+    const int k = a.k;
+    const int64_t i0 = (int64_t)tile * EP_ROWS;
+    const int rows = (int)min64(EP_ROWS, n - i0);
+    const int tot = rows * k;                       // elements of the tile, row-major, stride k
+    const int64_t base = i0 * (int64_t)k;
+    float* P = smem;                                // [EP_ROWS * KE] partial sums
+    float* T2 = P + EP_ROWS * KE;                   // G, then G'
+    float* T1 = T2 + EP_ROWS * KE;                  // H, then H'
+    float* As = T1 + EP_ROWS * KE;                  // k x k Gram of the iterate
+    double* red = reinterpret_cast<double*>(As + KE * KE);   // 16 doubles
+    double* Hd = reinterpret_cast<double*>(P);      // H' in fp64, aliases P and T2
+    const bool step = mode == MODE_FULL || mode == MODE_SVRG_INNER || mode == MODE_STEP_SNAP;
+
+    // ---- stage the tile: P = sum of partials (or the snapshot product), H, G, A.
+    // Thread tid owns elements tid + q*NT (q < EPT).  Every global load is
+    // issued before the first shared-memory store (the compiler cannot tell the
+    // two address spaces apart through these pointers), and each split's loads
+    // for all of a thread's elements go out together, so the tile costs about
+    // one L2 round trip per split (per two splits when registers allow).
+    constexpr int EPT = EP_ROWS * KE / NT;
+    constexpr int AEL = (KE * KE + NT - 1) / NT;
+    const bool snap_in = mode == MODE_STEP_SNAP || mode == MODE_SVRG_INNER;
+    float ps[EPT], hv[EPT], gv[EPT], av[AEL];
+    if (mode != MODE_PRODUCT) {
+#pragma unroll
+        for (int q = 0; q < EPT; ++q) {
+            const int e = tid + q * NT;
+            const bool in = e < tot;
+            ps[q] = (in && snap_in) ? __ldcg(a.Psnap + base + e) : 0.f;
+            hv[q] = in ? __ldcg(a.H + base + e) : 0.f;
+            gv[q] = (in && step) ? __ldcg(a.G + base + e) : 0.f;
+        }
+#pragma unroll
+        for (int q = 0; q < AEL; ++q) {
+            const int e = tid + q * NT;
+            av[q] = (step && e < k * k) ? a.st->A32[e] : 0.f;
+        }
+    }
+    float acc[EPT];
+#pragma unroll
+    for (int q = 0; q < EPT; ++q) acc[q] = 0.f;
+    if (mode != MODE_GRAM && mode != MODE_STEP_SNAP) {
+        int s = 0;
+        if constexpr (EPT <= 16) {
+            for (; s + 1 < a.splits; s += 2) {
+                const float* s0 = a.part + (int64_t)s * n * k + base;
+                const float* s1 = s0 + n * k;
+                float v0[EPT], v1[EPT];
+#pragma unroll
+                for (int q = 0; q < EPT; ++q) {
+                    const int e = tid + q * NT;
+                    v0[q] = e < tot ? __ldcg(s0 + e) : 0.f;
+                    v1[q] = e < tot ? __ldcg(s1 + e) : 0.f;
+                }
+#pragma unroll
+                for (int q = 0; q < EPT; ++q) {
+                    acc[q] += v0[q];
+                    acc[q] += v1[q];
+                }
+            }
+        }
+        for (; s < a.splits; ++s) {
+            const float* src = a.part + (int64_t)s * n * k + base;
+            float v[EPT];
+#pragma unroll
+            for (int q = 0; q < EPT; ++q) {
+                const int e = tid + q * NT;
+                v[q] = e < tot ? __ldcg(src + e) : 0.f;
+            }
+#pragma unroll
+            for (int q = 0; q < EPT; ++q) acc[q] += v[q];
+        }
+    }
+    if (mode == MODE_PRODUCT) {
+#pragma unroll
+        for (int q = 0; q < EPT; ++q) {
+            const int e = tid + q * NT;
+            if (e < tot) a.Y[base + e] = acc[q];
+        }
+        return;
+    }
+#pragma unroll
+    for (int q = 0; q < EPT; ++q) {
+        const int e = tid + q * NT;
+        if (e >= tot) continue;
+        float p = acc[q];
+        if (mode == MODE_STEP_SNAP) p = ps[q];
+        else if (mode == MODE_SVRG_INNER) p = fmaf(a.m_scale, p, ps[q]);
+        if (mode == MODE_SNAPSHOT) a.Psnap[base + e] = p;
+        P[e] = p;
+        T1[e] = hv[q];
+        if (step) T2[e] = gv[q];
+    }
+    if (step) {
+#pragma unroll
+        for (int q = 0; q < AEL; ++q) {
+            const int e = tid + q * NT;
+            if (e < k * k) As[(e / k) * KE + (e % k)] = av[q];
+        }
+    }
+    __syncthreads();
+
+    // ---- trace partial sum_i sum_c H_ic P_ic (fp64; fp32 products are exact)
+    if (mode == MODE_FULL || mode == MODE_SNAPSHOT) {
+        double tr = 0.0;
+        for (int e = tid; e < tot; e += NT) tr += (double)T1[e] * (double)P[e];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) tr += __shfl_down_sync(0xffffffffu, tr, o);
+        if ((tid & 31) == 0) red[tid >> 5] = tr;
+        __syncthreads();
+        if (tid == 0) {
+            double t = 0.0;
+            for (int w = 0; w < NT / 32; ++w) t += red[w];
+            a.tr_part[tile] = t;
+        }
+    }
+    if (mode == MODE_SNAPSHOT) return;
+
+    // ---- projected AdaGrad step: two threads per row, KE/2 columns each
+    if (step) {
+        constexpr int HALF = KE / 2;
+        const int r = tid >> 1, c0 = (tid & 1) * HALF;
+        float h[KE], hn[HALF], gn[HALF];
+        const bool valid = r < rows;
+#pragma unroll
+        for (int d = 0; d < KE; ++d) h[d] = (valid && d < k) ? T1[r * k + d] : 0.f;
+#pragma unroll
+        for (int j = 0; j < HALF; ++j) {
+            const int c = c0 + j;
+            hn[j] = 0.f;
+            gn[j] = 0.f;
+            if (valid && c < k) {
+                float ha = 0.f;
+#pragma unroll
+                for (int d = 0; d < KE; ++d)
+                    if (d < k) ha = fmaf(h[d], As[d * KE + c], ha);
+                const float g = 4.f * (ha - P[r * k + c]);
+                const float gg = fmaf(g, g, T2[r * k + c]);
+                const float stepv = __fdiv_rn(a.lr * g, __fadd_rn(__fsqrt_rn(gg), a.eps));
+                hn[j] = fmaxf(T1[r * k + c] - stepv, 0.f);   // = h[c]
+                gn[j] = gg;
+            }
+        }
+        __syncthreads();   // every thread holds its row of H: T1, T2 may be overwritten
+        if (valid) {
+#pragma unroll
+            for (int j = 0; j < HALF; ++j) {
+                const int c = c0 + j;
+                if (c < k) {
+                    T1[r * k + c] = hn[j];
+                    T2[r * k + c] = gn[j];
+                }
+            }
+        }
+        __syncthreads();
+        for (int e = tid; e < tot; e += NT) {
+            a.Hn[base + e] = T1[e];
+            a.Gn[base + e] = T2[e];
+        }
+    }
+
+    // ---- exact TF32 split [h_hi; h_lo] of the rows now in T1 (the next pass's operand)
+    if (a.XT != nullptr && (mode == MODE_FULL || mode == MODE_STEP_SNAP || mode == MODE_GRAM)) {
+        const int KP = (k + 7) / 8 * 8;
+        for (int e = tid; e < k * EP_ROWS; e += NT) {
+            const int c = e / EP_ROWS, r = e % EP_ROWS;
+            if (r < rows) {
+                const float v = T1[r * k + c];
+                const float hb = __uint_as_float(__float_as_uint(v) & 0xFFFFE000u);
+                a.XT[(int64_t)c * a.ldxt + i0 + r] = hb;
+                a.XT[(int64_t)(KP + c) * a.ldxt + i0 + r] = v - hb;
+            }
+        }
+    }
+
+    // ---- Gram partial of the rows in T1, in fp64 (Hd aliases P and T2, both dead)
+    __syncthreads();
+    for (int e = tid; e < EP_ROWS * KE; e += NT) {
+        const int r = e / KE, c = e % KE;
+        Hd[e] = (r < rows && c < k) ? (double)T1[r * k + c] : 0.0;
+    }
+    __syncthreads();
+    double* gp = a.gram_part + (int64_t)tile * k * k;
+    const int pairs = k * (k + 1) / 2;
+    for (int q = tid; q < pairs; q += NT) {
+        // q -> (c, d), c <= d, row-major over the upper triangle
+        int c = 0, rem = q;
+        while (rem >= k - c) {
+            rem -= k - c;
+            ++c;
+        }
+        const int d = c + rem;
+        double s0 = 0.0, s1 = 0.0, s2 = 0.0, s3 = 0.0;
+        int r = 0;
+        for (; r + 4 <= rows; r += 4) {
+            s0 = fma(Hd[r * KE + c], Hd[r * KE + d], s0);
+            s1 = fma(Hd[(r + 1) * KE + c], Hd[(r + 1) * KE + d], s1);
+            s2 = fma(Hd[(r + 2) * KE + c], Hd[(r + 2) * KE + d], s2);
+            s3 = fma(Hd[(r + 3) * KE + c], Hd[(r + 3) * KE + d], s3);
+        }
+        for (; r < rows; ++r) s0 = fma(Hd[r * KE + c], Hd[r * KE + d], s0);
+        const double v = (s0 + s1) + (s2 + s3);
+        gp[c * k + d] = v;
+        gp[d * k + c] = v;
+    }
+}
+
+}  // namespace symnmf

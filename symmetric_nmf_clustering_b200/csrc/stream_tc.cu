@@ -19,15 +19,18 @@
 //   warp 0      TMA producer: S tile (128 x 32, 128-byte swizzle) and the
 //               matching [X_hi; X_lo] tile (2*KP x 32, K-major) per stage,
 //               KP = k rounded up to 8
-//   warp 1      MMA issuer: per 8-column step, D[:, 0:2KP] += S_hi [X_hi;X_lo]
+//   warps 1, 3  MMA issuers (one thread each, alternate chunks of TC_CHUNK
+//               stages): per 8-column step, D[:, 0:2KP] += S_hi [X_hi;X_lo]
 //               (A = the S tile in shared memory, truncated to TF32 by the
-//               tensor core) and D[:, 0:KP] += S_lo X_hi (A = S_lo in TMEM)
+//               tensor core) and D[:, 0:KP] += S_lo X_hi (A = S_lo in TMEM).
+//               Issuing a tcgen05 MMA or commit costs the issuing thread tens
+//               of cycles, and one thread alone could not keep up with HBM.
 //   warp 2      TMEM allocator
 //   warps 4-7   split warps: thread r reads row r of the S tile from shared
 //               memory, stores its lo plane into TMEM lane r, folds the
 //               finished accumulator into fp32 registers every TC_CHUNK
-//               stages, writes the partial row, and -- in the last split CTA
-//               of the tile -- runs the epilogue (epilogue.cuh)
+//               stages and writes the partial row
+//   all warps   in the last split CTA of the tile, the epilogue (epilogue.cuh)
 #include <cudaTypedefs.h>
 
 #include <cstring>
@@ -43,7 +46,7 @@ namespace symnmf {
 // TF32, which is exactly S_hi (measured on B200: bit-identical results to
 // storing S_hi in TMEM), so only S_lo goes through TMEM.
 #ifndef SYMNMF_TC_NS
-#define SYMNMF_TC_NS 4
+#define SYMNMF_TC_NS 5
 #endif
 #ifndef SYMNMF_TC_CHUNK
 #define SYMNMF_TC_CHUNK 2
@@ -106,11 +109,12 @@ stream_tc_kernel(const __grid_constant__ CUtensorMap mapS, const __grid_constant
     extern __shared__ uint8_t tc_smem_raw[];
     __shared__ __align__(8) uint64_t bar_full[TC_NS], bar_empty[TC_NS];
     __shared__ __align__(8) uint64_t bar_tfull[TC_NT], bar_tempty[TC_NT];
-    __shared__ __align__(8) uint64_t bar_dfull[2], bar_dempty[2], bar_fin;
+    __shared__ __align__(8) uint64_t bar_dfull[2], bar_dempty[2], bar_fin[2];
     __shared__ uint32_t tmem_base_sh;
     __shared__ volatile int abort_sh;
     __shared__ int go_sh, last_sh;
-    __shared__ double red_sh[EP_ROWS / 32];
+    static_assert(epilogue_cta_floats<KP>() * sizeof(float) <= Cfg::SMEM - 1024,
+                  "the epilogue tiles must fit in the pipeline's shared memory");
 
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(tc_smem_raw) + 1023) & ~uintptr_t(1023));
@@ -138,8 +142,10 @@ stream_tc_kernel(const __grid_constant__ CUtensorMap mapS, const __grid_constant
             mbar_init(&bar_dfull[b], 1);
             mbar_init(&bar_dempty[b], 4);  // one arrival per split warp
         }
-        mbar_init(&bar_fin, 1);
+        mbar_init(&bar_fin[0], 1);
+        mbar_init(&bar_fin[1], 1);
         abort_sh = 0;
+        last_sh = 0;
         fence_mbar_init();
         prefetch_tmap(&mapS);
         prefetch_tmap(&mapX);
@@ -181,11 +187,16 @@ stream_tc_kernel(const __grid_constant__ CUtensorMap mapS, const __grid_constant
             for (int s = max(0, issued - TC_NS); s < issued; ++s)
                 mbar_wait(&bar_full[s % TC_NS], (uint32_t)(s / TC_NS) & 1u);
         }
-    } else if (warp == 1 && lane == 0 && ksteps > 0) {
-        // ---------------- MMA issuer: chunk q accumulates into D[q % 2]
+    } else if ((warp == 1 || warp == 3) && lane == 0 && ksteps > 0) {
+        // ---------------- MMA issuers: chunk q accumulates into D[q % 2] and is
+        // issued by warp 1 (q even) or warp 3 (q odd).  A tcgen05.commit tracks
+        // the MMAs of its own thread, and each accumulator has one issuer, so
+        // the two run independently; together they issue twice as fast as one.
+        const int par = warp == 1 ? 0 : 1;
         constexpr uint32_t id1 = idesc_tf32(TC_BM, Cfg::N1);
         constexpr uint32_t id2 = idesc_tf32(TC_BM, Cfg::N2);
         for (int s = 0; s < ksteps; ++s) {
+            if (((s / TC_CHUNK) & 1) != par) continue;
             if (abort_sh) break;
             const int slot = s % TC_NS;
             const uint32_t ph = (uint32_t)(s / TC_NS) & 1u;
@@ -222,8 +233,8 @@ stream_tc_kernel(const __grid_constant__ CUtensorMap mapS, const __grid_constant
             if (last) umma_commit(&bar_dfull[b]);
         }
         if (abort_sh) {  // MMAs in flight finish before TMEM is freed
-            umma_commit(&bar_fin);
-            mbar_wait(&bar_fin, 0);
+            umma_commit(&bar_fin[par]);
+            mbar_wait(&bar_fin[par], 0);
         }
     } else if (warp >= 4) {
         // ---------------- split warps (TMEM lane quarter = warp % 4)
@@ -330,13 +341,6 @@ stream_tc_kernel(const __grid_constant__ CUtensorMap mapS, const __grid_constant
             __threadfence();
             asm volatile("bar.sync 1, 128;" ::: "memory");
             if (r == 0) last_sh = atomicAdd(&counters[blockIdx.x], 1) == (int)gridDim.y - 1 ? 1 : 0;
-            asm volatile("bar.sync 1, 128;" ::: "memory");
-            if (last_sh) {
-                __threadfence();
-                epilogue_tile<KP, true>(epi, (int)blockIdx.x, r, reinterpret_cast<float*>(smem),
-                                         red_sh);
-                if (r == 0) counters[blockIdx.x] = 0;   // ready for the next pass
-            }
         }
     }
 
@@ -345,6 +349,13 @@ stream_tc_kernel(const __grid_constant__ CUtensorMap mapS, const __grid_constant
     if (warp == 2) {
         tc_fence_after();
         tmem_dealloc(tbase, Cfg::TMEM_COLS);
+    }
+    // every stage has landed and been consumed: the pipeline's shared memory is
+    // free, and all eight warps run the tile's epilogue
+    if (last_sh) {
+        __threadfence();
+        epilogue_tile_cta<KP>(epi, (int)blockIdx.x, tid, reinterpret_cast<float*>(smem));
+        if (tid == 0) counters[blockIdx.x] = 0;   // ready for the next pass
     }
 }
 
