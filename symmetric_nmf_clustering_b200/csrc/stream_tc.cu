@@ -64,6 +64,14 @@ constexpr bool TC_A_SMEM = SYMNMF_TC_A_SMEM != 0;
 constexpr int TC_TSTAGE = TC_A_SMEM ? 32 : 64;   // TMEM columns per stage of the split S tile
 constexpr int TC_NT = TC_A_SMEM ? 4 : 2;         // TMEM stages of the split S tile
 constexpr int TC_CHUNK = SYMNMF_TC_CHUNK;   // stages accumulated in TMEM before a drain
+// The two MMA issuers take alternate chunks.  An mbarrier wait checks phase
+// parity, so a thread may only wait on a barrier whose phases between its own
+// consecutive waits are all its own.  With TC_NT == 2 * TC_CHUNK each issuer
+// owns half of the TMEM stage slots (and their tfull barriers); its wait on
+// the shared full barrier of a stage comes after its tfull wait, by which
+// point the split warps have consumed that phase and no later phase of the
+// slot can complete before this issuer's own commit.
+static_assert(TC_NT == 2 * TC_CHUNK, "each MMA issuer must own its TMEM stage slots");
 constexpr int TC_THREADS = 256;
 constexpr uint32_t TC_A_BYTES = TC_BM * TC_BK * 4;
 
