@@ -72,6 +72,17 @@ constexpr int TC_CHUNK = SYMNMF_TC_CHUNK;   // stages accumulated in TMEM before
 // point the split warps have consumed that phase and no later phase of the
 // slot can complete before this issuer's own commit.
 static_assert(TC_NT == 2 * TC_CHUNK, "each MMA issuer must own its TMEM stage slots");
+// Completion of stage s's MMAs is signalled once, by one tcgen05.commit to
+// bar_done[s % TC_NDONE]; the producer (shared-memory slot of stage s - TC_NS),
+// the split warps (TMEM slot of stage s - TC_NT) and the drain (last stage of
+// a chunk) all wait on it.  Each waiter visits stages in order, and TC_NDONE
+// exceeds both ring depths, so no barrier completes a second phase before its
+// waiters have seen the first; the split warps reach stage x + TC_NT only after
+// stage x completed, so a barrier's phases complete in stage order even though
+// two threads issue.
+constexpr int TC_NDONE = TC_NS * TC_NT;   // a common multiple of both ring depths
+static_assert(TC_NDONE > TC_NS && TC_NDONE > TC_NT && TC_NDONE % TC_NS == 0 && TC_NDONE % TC_NT == 0,
+              "stage-completion barriers must outnumber both rings");
 constexpr int TC_THREADS = 256;
 constexpr uint32_t TC_A_BYTES = TC_BM * TC_BK * 4;
 
@@ -115,9 +126,8 @@ stream_tc_kernel(const __grid_constant__ CUtensorMap mapS, const __grid_constant
     if (st != nullptr && st->done) return;
 
     extern __shared__ uint8_t tc_smem_raw[];
-    __shared__ __align__(8) uint64_t bar_full[TC_NS], bar_empty[TC_NS];
-    __shared__ __align__(8) uint64_t bar_tfull[TC_NT], bar_tempty[TC_NT];
-    __shared__ __align__(8) uint64_t bar_dfull[2], bar_dempty[2], bar_fin[2];
+    __shared__ __align__(8) uint64_t bar_full[TC_NS], bar_tfull[TC_NT], bar_done[TC_NDONE];
+    __shared__ __align__(8) uint64_t bar_dempty[2], bar_fin[2];
     __shared__ uint32_t tmem_base_sh;
     __shared__ volatile int abort_sh;
     __shared__ int go_sh, last_sh;
@@ -140,16 +150,16 @@ stream_tc_kernel(const __grid_constant__ CUtensorMap mapS, const __grid_constant
     if (tid == 0) {
         for (int s = 0; s < TC_NS; ++s) {
             mbar_init(&bar_full[s], 1);
-            mbar_init(&bar_empty[s], 1);
         }
         for (int t = 0; t < TC_NT; ++t) {
             mbar_init(&bar_tfull[t], 4);   // one arrival per split warp
-            mbar_init(&bar_tempty[t], 1);
+
         }
         for (int b = 0; b < 2; ++b) {
-            mbar_init(&bar_dfull[b], 1);
+
             mbar_init(&bar_dempty[b], 4);  // one arrival per split warp
         }
+        for (int d = 0; d < TC_NDONE; ++d) mbar_init(&bar_done[d], 1);
         mbar_init(&bar_fin[0], 1);
         mbar_init(&bar_fin[1], 1);
         abort_sh = 0;
@@ -175,8 +185,8 @@ stream_tc_kernel(const __grid_constant__ CUtensorMap mapS, const __grid_constant
         for (int s = 0; s < ksteps; ++s) {
             if (abort_sh) break;
             const int slot = s % TC_NS;
-            const uint32_t ph = (uint32_t)(s / TC_NS) & 1u;
-            if (s >= TC_NS && !mbar_wait(&bar_empty[slot], ph ^ 1u)) {
+            if (s >= TC_NS && !mbar_wait(&bar_done[(s - TC_NS) % TC_NDONE],
+                                         (uint32_t)((s - TC_NS) / TC_NDONE) & 1u)) {
                 tc_fail(err, &abort_sh, 1);
                 break;
             }
@@ -212,7 +222,6 @@ stream_tc_kernel(const __grid_constant__ CUtensorMap mapS, const __grid_constant
             const uint32_t tph = (uint32_t)(s / TC_NT) & 1u;
             const int q = s / TC_CHUNK, b = q & 1;
             const bool first = (s % TC_CHUNK) == 0;
-            const bool last = (s % TC_CHUNK) == TC_CHUNK - 1 || s == ksteps - 1;
             bool ok = mbar_wait(&bar_tfull[ts], tph) && mbar_wait(&bar_full[slot], ph);
             if (ok && first && q >= 2) ok = mbar_wait(&bar_dempty[b], (uint32_t)((q >> 1) - 1) & 1u);
             if (!ok) {
@@ -236,9 +245,7 @@ stream_tc_kernel(const __grid_constant__ CUtensorMap mapS, const __grid_constant
                     umma_tf32_ts(d, a_t + 32u + (uint32_t)kk * 8u, bd, id2, 1u);
                 }
             }
-            umma_commit(&bar_empty[slot]);
-            umma_commit(&bar_tempty[ts]);
-            if (last) umma_commit(&bar_dfull[b]);
+            umma_commit(&bar_done[s % TC_NDONE]);
         }
         if (abort_sh) {  // MMAs in flight finish before TMEM is freed
             umma_commit(&bar_fin[par]);
@@ -259,7 +266,8 @@ stream_tc_kernel(const __grid_constant__ CUtensorMap mapS, const __grid_constant
         // per accumulate, so TMEM chains are kept to TC_CHUNK stages
         auto drain = [&](int q) -> bool {
             const int b = q & 1;
-            if (!__all_sync(0xffffffffu, mbar_wait(&bar_dfull[b], (uint32_t)(q >> 1) & 1u)))
+            const int ls = min(ksteps, (q + 1) * TC_CHUNK) - 1;   // last stage of chunk q
+            if (!__all_sync(0xffffffffu, mbar_wait(&bar_done[ls % TC_NDONE], (uint32_t)(ls / TC_NDONE) & 1u)))
                 return false;
             tc_fence_after();
             const uint32_t dcol = tbase + lane_off + (uint32_t)b * Cfg::DSTRIDE;
@@ -285,9 +293,9 @@ stream_tc_kernel(const __grid_constant__ CUtensorMap mapS, const __grid_constant
             const int slot = s % TC_NS;
             const uint32_t ph = (uint32_t)(s / TC_NS) & 1u;
             const int ts = s % TC_NT;
-            const uint32_t tph = (uint32_t)(s / TC_NT) & 1u;
             const bool ok = mbar_wait(&bar_full[slot], ph) &&
-                            (s < TC_NT || mbar_wait(&bar_tempty[ts], tph ^ 1u));
+                            (s < TC_NT || mbar_wait(&bar_done[(s - TC_NT) % TC_NDONE],
+                                                    (uint32_t)((s - TC_NT) / TC_NDONE) & 1u));
             if (!__all_sync(0xffffffffu, ok)) {
                 if (lane == 0) tc_fail(err, &abort_sh, 3);
                 alive = false;
