@@ -421,11 +421,15 @@ static int full_pass(FitCtx& c, int mode, int max_evals, bool xt_ready) {
                            c.P->rel_tol, max_evals, c.L.hist, c.L.hist_cap, c.s);
 }
 
+// Replaying the full-batch loop as a CUDA graph is opt-in (SYMNMF_GRAPHS=1):
+// each pass's kernels run for tens of microseconds or more, the loop is not
+// launch-bound, and eager launches measured as fast or faster on B200
+// (n = 5,000: 6.0 ms per 100 iterations eager, 6.4 ms replayed).
 static bool use_graphs() {
     static int v = -1;
     if (v < 0) {
         const char* e = getenv("SYMNMF_GRAPHS");
-        v = (e != nullptr && std::strcmp(e, "0") == 0) ? 0 : 1;
+        v = (e != nullptr && std::strcmp(e, "1") == 0) ? 1 : 0;
     }
     return v == 1;
 }

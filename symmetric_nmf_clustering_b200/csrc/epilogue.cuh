@@ -232,7 +232,7 @@ __device__ void epilogue_tile_cta(const EpiArgs& a, int tile, int tid, float* sm
     float* T1 = T2 + EP_ROWS * KE;                  // H, then H'
     float* As = T1 + EP_ROWS * KE;                  // k x k Gram of the iterate
     double* red = reinterpret_cast<double*>(As + KE * KE);   // 16 doubles
-    double* Hd = reinterpret_cast<double*>(P);      // H' in fp64, aliases P and T2
+    double* Hd = reinterpret_cast<double*>(P);      // H' in fp64 (row stride KE + 2), aliases P, T2, T1
     const bool step = mode == MODE_FULL || mode == MODE_SVRG_INNER || mode == MODE_STEP_SNAP;
 
     // ---- stage the tile: P = sum of partials (or the snapshot product), H, G, A.
@@ -397,35 +397,80 @@ __device__ void epilogue_tile_cta(const EpiArgs& a, int tile, int tid, float* sm
         }
     }
 
-    // ---- Gram partial of the rows in T1, in fp64 (Hd aliases P and T2, both dead)
+    // ---- Gram partial of the rows in T1, in fp64.  The rows go through
+    // registers so that Hd (row stride KE + 2: 16-byte aligned, and eight
+    // consecutive rows fall in distinct banks) can overwrite P, T2 and T1.
+    constexpr int HS = KE + 2;
+    static_assert(EP_ROWS * HS * 2 <= 3 * EP_ROWS * KE, "Hd fits in P, T2 and T1");
     __syncthreads();
-    for (int e = tid; e < EP_ROWS * KE; e += NT) {
-        const int r = e / KE, c = e % KE;
-        Hd[e] = (r < rows && c < k) ? (double)T1[r * k + c] : 0.0;
+    float hreg[EPT];
+#pragma unroll
+    for (int q = 0; q < EPT; ++q) {
+        const int e = tid + q * NT, r = e / KE, c = e % KE;
+        hreg[q] = (r < rows && c < k) ? T1[r * k + c] : 0.f;
     }
     __syncthreads();
-    double* gp = a.gram_part + (int64_t)tile * k * k;
-    const int pairs = k * (k + 1) / 2;
-    for (int q = tid; q < pairs; q += NT) {
-        // q -> (c, d), c <= d, row-major over the upper triangle
-        int c = 0, rem = q;
-        while (rem >= k - c) {
-            rem -= k - c;
-            ++c;
+#pragma unroll
+    for (int q = 0; q < EPT; ++q) {
+        const int e = tid + q * NT, r = e / KE, c = e % KE;
+        Hd[r * HS + c] = (double)hreg[q];
+    }
+    __syncthreads();
+    // 4x4 register blocks of the upper triangle; the rows of the tile are cut
+    // into RG groups whose partial blocks sit in adjacent lanes and are
+    // combined by a fixed xor-shuffle tree (every lane ends with the same sum)
+    constexpr int NB = KE / 4, NBLK = NB * (NB + 1) / 2;
+    constexpr int RG = NBLK * 32 <= NT ? 32 : NBLK * 16 <= NT ? 16 : NBLK * 8 <= NT ? 8
+                     : NBLK * 4 <= NT ? 4 : NBLK * 2 <= NT ? 2 : 1;
+    constexpr int RROWS = EP_ROWS / RG;   // rows grp, grp + RG, grp + 2 RG, ...
+    static_assert(NBLK * RG <= NT && 32 % RG == 0, "one Gram task per thread, groups inside a warp");
+    double gacc[4][4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) gacc[i][j] = 0.0;
+    const int blk = tid / RG, grp = tid % RG;
+    int bi = 0, bj = 0;
+    if (blk < NBLK) {
+        int rem = blk;
+        while (rem >= NB - bi) {
+            rem -= NB - bi;
+            ++bi;
         }
-        const int d = c + rem;
-        double s0 = 0.0, s1 = 0.0, s2 = 0.0, s3 = 0.0;
-        int r = 0;
-        for (; r + 4 <= rows; r += 4) {
-            s0 = fma(Hd[r * KE + c], Hd[r * KE + d], s0);
-            s1 = fma(Hd[(r + 1) * KE + c], Hd[(r + 1) * KE + d], s1);
-            s2 = fma(Hd[(r + 2) * KE + c], Hd[(r + 2) * KE + d], s2);
-            s3 = fma(Hd[(r + 3) * KE + c], Hd[(r + 3) * KE + d], s3);
+        bj = bi + rem;
+        // rows past the tile's end hold zeros, which add exactly nothing
+        for (int t = 0; t < RROWS; ++t) {
+            const double* hr = Hd + (grp + t * RG) * HS;
+            const double2 x01 = *reinterpret_cast<const double2*>(hr + 4 * bi);
+            const double2 x23 = *reinterpret_cast<const double2*>(hr + 4 * bi + 2);
+            const double2 y01 = *reinterpret_cast<const double2*>(hr + 4 * bj);
+            const double2 y23 = *reinterpret_cast<const double2*>(hr + 4 * bj + 2);
+            const double x[4] = {x01.x, x01.y, x23.x, x23.y};
+            const double y[4] = {y01.x, y01.y, y23.x, y23.y};
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int j = 0; j < 4; ++j) gacc[i][j] = fma(x[i], y[j], gacc[i][j]);
         }
-        for (; r < rows; ++r) s0 = fma(Hd[r * KE + c], Hd[r * KE + d], s0);
-        const double v = (s0 + s1) + (s2 + s3);
-        gp[c * k + d] = v;
-        gp[d * k + c] = v;
+    }
+#pragma unroll
+    for (int o = 1; o < RG; o <<= 1)
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) gacc[i][j] += __shfl_xor_sync(0xffffffffu, gacc[i][j], o);
+    if (blk < NBLK && grp == 0) {
+        double* gp = a.gram_part + (int64_t)tile * k * k;
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int c = 4 * bi + i, d = 4 * bj + j;
+                if (c < k && d < k) {
+                    gp[c * k + d] = gacc[i][j];
+                    gp[d * k + c] = gacc[i][j];
+                }
+            }
     }
 }
 

@@ -191,7 +191,7 @@ def test_errors(m):
     assert e.value.status == _lib.SYMNMF_ERR_WORKSPACE
 
 
-_EAGER_SCRIPT = r"""
+_OTHER_MODE_SCRIPT = r"""
 import sys, numpy as np, torch
 sys.path.insert(0, sys.argv[1])
 import symmetric_nmf_clustering_b200 as m
@@ -203,6 +203,7 @@ np.save(sys.argv[4], st["history"])
 
 
 def test_graph_replay_matches_eager_launches(m, tmp_path):
+    # the default is eager launches; the subprocess replays the loop as a graph
     import os
     import subprocess
     import sys
@@ -210,8 +211,8 @@ def test_graph_replay_matches_eager_launches(m, tmp_path):
     Hg, st, _ = _fit(m, S, 8, seed=5, max_iters=70, rel_tol=0.0)
     np.save(tmp_path / "S.npy", S)
     root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
-    env = dict(os.environ, SYMNMF_GRAPHS="0")
-    r = subprocess.run([sys.executable, "-c", _EAGER_SCRIPT, root, str(tmp_path / "S.npy"),
+    env = dict(os.environ, SYMNMF_GRAPHS="1")
+    r = subprocess.run([sys.executable, "-c", _OTHER_MODE_SCRIPT, root, str(tmp_path / "S.npy"),
                         str(tmp_path / "H.npy"), str(tmp_path / "hist.npy")],
                        env=env, capture_output=True, text=True, timeout=300)
     assert r.returncode == 0, r.stderr
