@@ -303,6 +303,70 @@ rank_kernel(const float* __restrict__ R, int64_t T, int64_t n, int64_t ldr, floa
     }
 }
 
+// The same ranks by sorting: the rank of x_t is its 1-based position when the
+// column is ordered by the key (x_t, t), which breaks ties towards the earlier
+// day exactly as the count above does.  Eight columns per block (one 32-byte
+// sector per day on load and store), a bitonic sort of each column's P = 2^m
+// >= T keys in shared memory (padding keys (+inf, t >= T) sort last), then the
+// positions are scattered into a day-major tile and written out.
+constexpr int RS_COLS = 8;
+constexpr int RS_THREADS = 1024;
+constexpr int RS_PER_COL = RS_THREADS / RS_COLS;
+constexpr int64_t RS_MAX_P = 2048;
+
+__device__ __forceinline__ bool rs_before(float va, int ta, float vb, int tb) {
+    return va < vb || (va == vb && ta < tb);
+}
+
+__global__ void __launch_bounds__(RS_THREADS)
+rank_sort_kernel(const float* __restrict__ R, int64_t T, int64_t n, int64_t ldr, float sign,
+                 int P, int32_t* __restrict__ ranks) {
+    extern __shared__ uint8_t rs_smem[];
+    float* kv = reinterpret_cast<float*>(rs_smem);                 // [RS_COLS][P] values
+    int* kt = reinterpret_cast<int*>(kv + (size_t)RS_COLS * P);     // [RS_COLS][P] days
+    int* rt = kt + (size_t)RS_COLS * P;                             // [T][RS_COLS] ranks
+    const int tid = threadIdx.x;
+    const int64_t i0 = (int64_t)blockIdx.x * RS_COLS;
+    const int cols = (int)min64(RS_COLS, n - i0);
+
+    for (int e = tid; e < RS_COLS * P; e += RS_THREADS) {
+        const int t = e / RS_COLS, c = e % RS_COLS;
+        float v = __int_as_float(0x7f800000);                       // +inf
+        if (t < T && c < cols) v = sign * R[(int64_t)t * ldr + i0 + c];
+        kv[c * P + t] = v;
+        kt[c * P + t] = t;
+    }
+    __syncthreads();
+
+    const int c = tid / RS_PER_COL, lt = tid % RS_PER_COL;
+    float* v = kv + c * P;
+    int* tt = kt + c * P;
+    for (int k = 2; k <= P; k <<= 1) {
+        for (int j = k >> 1; j > 0; j >>= 1) {
+            for (int q = lt; q < (P >> 1); q += RS_PER_COL) {
+                const int a = (q / j) * 2 * j + (q % j), b = a + j;
+                const bool up = (a & k) == 0;
+                const float va = v[a], vb = v[b];
+                const int ta = tt[a], tb = tt[b];
+                if (rs_before(vb, tb, va, ta) == up) {   // out of order for this direction
+                    v[a] = vb;
+                    v[b] = va;
+                    tt[a] = tb;
+                    tt[b] = ta;
+                }
+            }
+            __syncthreads();
+        }
+    }
+
+    for (int p = lt; p < T; p += RS_PER_COL) rt[tt[p] * RS_COLS + c] = p + 1;
+    __syncthreads();
+    for (int e = tid; e < T * RS_COLS; e += RS_THREADS) {
+        const int t = e / RS_COLS, cc = e % RS_COLS;
+        if (cc < cols) ranks[(int64_t)t * n + i0 + cc] = rt[e];
+    }
+}
+
 // phi[r] = (-ln(r / (T+1)))^(-1/2): Frechet (alpha = 2) margin of rank r, fp64.
 __global__ void phi_kernel(double* __restrict__ phi, int64_t T) {
     const int64_t r = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
@@ -388,7 +452,20 @@ int launch_tpdm(const float* R, int64_t T, int64_t n, int64_t ldr, int N,
     const unsigned rblocks = (unsigned)((n + RK_COLS - 1) / RK_COLS);
     const int64_t smem = T * RK_COLS * (int64_t)sizeof(float);
     const float sign = tail_sign < 0 ? -1.f : 1.f;
-    if (smem <= RK_SMEM_MAX) {
+    int P = 2;
+    while (P < T) P <<= 1;
+    if (P <= RS_MAX_P) {
+        const size_t rs_smem = (size_t)RS_COLS * P * 8 + (size_t)T * RS_COLS * 4;
+        static bool rs_attr = false;   // once per process
+        if (!rs_attr) {
+            SYMNMF_CUDA_TRY(cudaFuncSetAttribute(rank_sort_kernel,
+                                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 (int)(RS_COLS * RS_MAX_P * 12)));
+            rs_attr = true;
+        }
+        rank_sort_kernel<<<(unsigned)((n + RS_COLS - 1) / RS_COLS), RS_THREADS, rs_smem, s>>>(
+            R, T, n, ldr, sign, P, ranks);
+    } else if (smem <= RK_SMEM_MAX) {
         SYMNMF_CUDA_TRY(cudaFuncSetAttribute(rank_kernel<true>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize,
                                              (int)RK_SMEM_MAX));
