@@ -11,14 +11,20 @@
 //     Z^T Z = ZF.ZF + (ZF.ZL + ZL.ZF) + O(2^-22)
 // accumulated in two TMEM accumulators (main and correction).
 //
-// One CTA per 128 x 128 output tile (I <= J, upper triangle of tiles; the
-// tile is also written transposed), 256 threads:
+// Persistent: one CTA per SM walks its share of the 128 x 128 output tiles
+// (I <= J, the upper triangle of tiles; each tile is also written
+// transposed), 256 threads:
 //   warp 0      TMA producer: per 32-column stage the rows I of ZF and ZL and,
-//               off the diagonal, the rows J of ZF and ZL (16 KB each)
-//   warp 1      MMA issuer (M = N = 128, K = 8, both operands in shared memory)
+//               off the diagonal, the rows J of ZF and ZL (16 KB each), one
+//               stage ring across the CTA's tiles
+//   warp 1      MMA issuer (M = N = 128, K = 8, both operands in shared
+//               memory) into one of two TMEM accumulator sets, so that a
+//               tile's epilogue overlaps the next tile's loads and MMAs
 //   warp 2      TMEM allocator
 //   warps 4-7   epilogue: thread r owns row I0 + r, reads the accumulators in
-//               32-column chunks and writes S[i][J-tile] and S[J-tile][i]
+//               32-column chunks, stages S[I-tile][chunk] (128-byte swizzle)
+//               and its transpose in shared memory and writes both with TMA
+//               bulk stores
 #include <cudaTypedefs.h>
 
 #include <cmath>
@@ -34,47 +40,60 @@ constexpr int GT_NS = 3;                      // pipeline stages
 constexpr int GT_THREADS = 256;
 constexpr uint32_t GT_PLANE = GT_BM * GT_BK * 4;   // 16 KB: 128 rows x 128 B
 constexpr uint32_t GT_STAGE = 4 * GT_PLANE;        // AF, AL, BF, BL
-constexpr uint32_t GT_SMEM = GT_NS * GT_STAGE + 1024;
-constexpr uint32_t GT_TMEM_COLS = 256;             // main [0,128), correction [128,256)
+constexpr uint32_t GT_OUT = GT_BM * 32 * 4;        // 16 KB: one 32-column output chunk
+constexpr uint32_t GT_SMEM = GT_NS * GT_STAGE + 2 * GT_OUT + 1024;
+constexpr uint32_t GT_ACC = 256;                   // one accumulator set: main [0,128), correction [128,256)
+constexpr uint32_t GT_TMEM_COLS = 2 * GT_ACC;      // two sets: a tile drains while the next accumulates
 
 enum GramTcMode { GT_CORR = 0, GT_TPDM = 1 };
 
+// tile (I, J), I <= J, from its linear index over the upper triangle
+__device__ __forceinline__ void gt_tile(int64_t x, int64_t* I, int64_t* J) {
+    int64_t j = (int64_t)((sqrt(8.0 * (double)x + 1.0) - 1.0) * 0.5);
+    while ((j + 1) * (j + 2) / 2 <= x) ++j;
+    while (j * (j + 1) / 2 > x) --j;
+    *J = j;
+    *I = x - j * (j + 1) / 2;
+}
+
+// Persistent: CTA b takes the tiles b, b + grid, b + 2 grid, ...
 template <int MODE>
 __global__ void __launch_bounds__(GT_THREADS, 1)
 gram_tc_kernel(const __grid_constant__ CUtensorMap mapF, const __grid_constant__ CUtensorMap mapL,
-               int64_t n, int Kp, float scale, float* __restrict__ S, int64_t lds,
-               int* __restrict__ err) {
+               const __grid_constant__ CUtensorMap mapD, const __grid_constant__ CUtensorMap mapT,
+               int64_t n, int Kp, int64_t pairs, float scale, int* __restrict__ err) {
     using namespace sm100;
     extern __shared__ uint8_t gt_smem_raw[];
-    __shared__ __align__(8) uint64_t bar_full[GT_NS], bar_empty[GT_NS], bar_acc;
+    __shared__ __align__(8) uint64_t bar_full[GT_NS], bar_empty[GT_NS];
+    __shared__ __align__(8) uint64_t acc_full[2], acc_empty[2], bar_fin;
     __shared__ uint32_t tmem_base_sh;
-    __shared__ volatile int abort_sh;
+    __shared__ volatile int abort_sh, ep_fail_sh, go_sh;
 
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(gt_smem_raw) + 1023) & ~uintptr_t(1023));
+    float* outD = reinterpret_cast<float*>(smem + GT_NS * GT_STAGE);   // [128 rows][32], 128B swizzle
+    float* outT = outD + GT_BM * 32;                                   // [32 rows][128], plain
 
-    // tile (I, J), I <= J, from the linear index over the upper triangle
-    const int64_t x = blockIdx.x;
-    int64_t J = (int64_t)((sqrt(8.0 * (double)x + 1.0) - 1.0) * 0.5);
-    while ((J + 1) * (J + 2) / 2 <= x) ++J;
-    while (J * (J + 1) / 2 > x) --J;
-    const int64_t I = x - J * (J + 1) / 2;
-    const bool diag = I == J;
-    const int64_t I0 = I * GT_BM, J0 = J * GT_BM;
     const int ksteps = Kp / GT_BK;
-    const uint32_t stage_bytes = diag ? 2 * GT_PLANE : 4 * GT_PLANE;
-
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     if (tid == 0) {
         for (int s = 0; s < GT_NS; ++s) {
             mbar_init(&bar_full[s], 1);
             mbar_init(&bar_empty[s], 1);
         }
-        mbar_init(&bar_acc, 1);
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&acc_full[b], 1);
+            mbar_init(&acc_empty[b], 4);   // one arrival per epilogue warp
+        }
+        mbar_init(&bar_fin, 1);
         abort_sh = 0;
+        ep_fail_sh = 0;
+        go_sh = 1;
         fence_mbar_init();
         prefetch_tmap(&mapF);
         prefetch_tmap(&mapL);
+        prefetch_tmap(&mapD);
+        prefetch_tmap(&mapT);
     }
     if (warp == 2) {
         tmem_alloc(&tmem_base_sh, GT_TMEM_COLS);
@@ -88,111 +107,148 @@ gram_tc_kernel(const __grid_constant__ CUtensorMap mapF, const __grid_constant__
     auto plane = [&](int slot, int q) { return smem + slot * GT_STAGE + q * GT_PLANE; };
 
     if (warp == 0 && lane == 0) {
-        // ---------------- TMA producer
-        int issued = 0;
-        for (int s = 0; s < ksteps; ++s) {
-            if (abort_sh) break;
-            const int slot = s % GT_NS;
-            const uint32_t ph = (uint32_t)(s / GT_NS) & 1u;
-            if (s >= GT_NS && !mbar_wait(&bar_empty[slot], ph ^ 1u)) {
-                abort_sh = 1;
-                atomicExch(err, 1);
-                break;
+        // ---------------- TMA producer: one stage ring across all of this CTA's tiles
+        int64_t g = 0;   // stages issued
+        for (int64_t x = blockIdx.x; x < pairs && !abort_sh; x += gridDim.x) {
+            int64_t I, J;
+            gt_tile(x, &I, &J);
+            const bool diag = I == J;
+            const uint32_t stage_bytes = diag ? 2 * GT_PLANE : 4 * GT_PLANE;
+            for (int s = 0; s < ksteps; ++s, ++g) {
+                if (abort_sh) break;
+                const int slot = (int)(g % GT_NS);
+                if (g >= GT_NS && !mbar_wait(&bar_empty[slot], (uint32_t)((g / GT_NS) & 1) ^ 1u)) {
+                    abort_sh = 1;
+                    atomicExch(err, 1);
+                    break;
+                }
+                mbar_arrive_expect_tx(&bar_full[slot], stage_bytes);
+                const int32_t xk = s * GT_BK;
+                tma_load_2d(plane(slot, 0), &mapF, xk, (int32_t)(I * GT_BM), &bar_full[slot]);
+                tma_load_2d(plane(slot, 1), &mapL, xk, (int32_t)(I * GT_BM), &bar_full[slot]);
+                if (!diag) {
+                    tma_load_2d(plane(slot, 2), &mapF, xk, (int32_t)(J * GT_BM), &bar_full[slot]);
+                    tma_load_2d(plane(slot, 3), &mapL, xk, (int32_t)(J * GT_BM), &bar_full[slot]);
+                }
             }
-            mbar_arrive_expect_tx(&bar_full[slot], stage_bytes);
-            const int32_t xk = s * GT_BK;
-            tma_load_2d(plane(slot, 0), &mapF, xk, (int32_t)I0, &bar_full[slot]);
-            tma_load_2d(plane(slot, 1), &mapL, xk, (int32_t)I0, &bar_full[slot]);
-            if (!diag) {
-                tma_load_2d(plane(slot, 2), &mapF, xk, (int32_t)J0, &bar_full[slot]);
-                tma_load_2d(plane(slot, 3), &mapL, xk, (int32_t)J0, &bar_full[slot]);
-            }
-            ++issued;
         }
-        if (abort_sh) {
-            for (int s = max(0, issued - GT_NS); s < issued; ++s)
-                mbar_wait(&bar_full[s % GT_NS], (uint32_t)(s / GT_NS) & 1u);
+        if (abort_sh) {   // let the copies already issued land before the CTA exits
+            for (int64_t q = g > GT_NS ? g - GT_NS : 0; q < g; ++q)
+                mbar_wait(&bar_full[q % GT_NS], (uint32_t)((q / GT_NS) & 1));
         }
     } else if (warp == 1 && lane == 0) {
-        // ---------------- MMA issuer
+        // ---------------- MMA issuer: tile u accumulates into set u % 2
         constexpr uint32_t id = idesc_tf32(GT_BM, GT_BM);
-        for (int s = 0; s < ksteps; ++s) {
-            if (abort_sh) break;
-            const int slot = s % GT_NS;
-            const uint32_t ph = (uint32_t)(s / GT_NS) & 1u;
-            if (!mbar_wait(&bar_full[slot], ph)) {
+        int64_t g = 0;
+        int u = 0;
+        for (int64_t x = blockIdx.x; x < pairs && !abort_sh; x += gridDim.x, ++u) {
+            int64_t I, J;
+            gt_tile(x, &I, &J);
+            const bool diag = I == J;
+            const int b = u & 1;
+            if (u >= 2 && !mbar_wait(&acc_empty[b], (uint32_t)((u >> 1) - 1) & 1u)) {
                 abort_sh = 1;
                 atomicExch(err, 2);
                 break;
             }
             tc_fence_after();
-            const uint32_t af = smem_u32(plane(slot, 0)), al = smem_u32(plane(slot, 1));
-            const uint32_t bf = diag ? af : smem_u32(plane(slot, 2));
-            const uint32_t bl = diag ? al : smem_u32(plane(slot, 3));
+            const uint32_t dm = tbase + (uint32_t)b * GT_ACC, dc = dm + 128u;
+            for (int s = 0; s < ksteps; ++s, ++g) {
+                if (abort_sh) break;
+                const int slot = (int)(g % GT_NS);
+                if (!mbar_wait(&bar_full[slot], (uint32_t)((g / GT_NS) & 1))) {
+                    abort_sh = 1;
+                    atomicExch(err, 2);
+                    break;
+                }
+                tc_fence_after();
+                const uint32_t af = smem_u32(plane(slot, 0)), al = smem_u32(plane(slot, 1));
+                const uint32_t bf = diag ? af : smem_u32(plane(slot, 2));
+                const uint32_t bl = diag ? al : smem_u32(plane(slot, 3));
 #pragma unroll
-            for (int kk = 0; kk < GT_BK / 8; ++kk) {
-                const uint32_t o = (uint32_t)kk * 32u;
-                const uint32_t acc = (s | kk) ? 1u : 0u;
-                umma_tf32_ss(tbase, umma_desc_sw128(af + o), umma_desc_sw128(bf + o), id, acc);
-                umma_tf32_ss(tbase + 128u, umma_desc_sw128(af + o), umma_desc_sw128(bl + o), id, acc);
-                umma_tf32_ss(tbase + 128u, umma_desc_sw128(al + o), umma_desc_sw128(bf + o), id, 1u);
+                for (int kk = 0; kk < GT_BK / 8; ++kk) {
+                    const uint32_t o = (uint32_t)kk * 32u;
+                    const uint32_t acc = (s | kk) ? 1u : 0u;
+                    umma_tf32_ss(dm, umma_desc_sw128(af + o), umma_desc_sw128(bf + o), id, acc);
+                    umma_tf32_ss(dc, umma_desc_sw128(af + o), umma_desc_sw128(bl + o), id, acc);
+                    umma_tf32_ss(dc, umma_desc_sw128(al + o), umma_desc_sw128(bf + o), id, 1u);
+                }
+                umma_commit(&bar_empty[slot]);
             }
-            umma_commit(&bar_empty[slot]);
+            if (abort_sh) break;
+            umma_commit(&acc_full[b]);
         }
-        umma_commit(&bar_acc);
-        mbar_wait(&bar_acc, 0);   // (also when aborting: MMAs finish before TMEM is freed)
+        umma_commit(&bar_fin);
+        mbar_wait(&bar_fin, 0);   // every MMA has finished before TMEM is freed
     } else if (warp >= 4) {
-        // ---------------- epilogue (control flow warp-uniform for tcgen05.ld)
+        // ---------------- epilogue: thread r owns row I0 + r of the tile; the four
+        // warps take every decision together (they share named barrier 1)
         const int wl = warp & 3;
         const int r = wl * 32 + lane;
         const uint32_t lane_off = (uint32_t)(wl * 32) << 16;
-        const bool ok = __all_sync(0xffffffffu, mbar_wait(&bar_acc, 0)) &&
-                        !__any_sync(0xffffffffu, abort_sh != 0);
-        if (!ok) {
-            if (lane == 0) atomicExch(err, 3);
-        } else {
+        int u = 0;
+        for (int64_t x = blockIdx.x; x < pairs; x += gridDim.x, ++u) {
+            int64_t I, J;
+            gt_tile(x, &I, &J);
+            const bool diag = I == J;
+            const int b = u & 1;
+            const int64_t I0 = I * GT_BM, J0 = J * GT_BM;
+            const bool w_ok = __all_sync(0xffffffffu, mbar_wait(&acc_full[b], (uint32_t)(u >> 1) & 1u));
+            if (lane == 0 && !w_ok) atomicOr(const_cast<int*>(&ep_fail_sh), 1);
+            asm volatile("bar.sync 1, 128;" ::: "memory");
+            if (r == 0) go_sh = (ep_fail_sh == 0 && abort_sh == 0) ? 1 : 0;
+            asm volatile("bar.sync 1, 128;" ::: "memory");
+            if (!go_sh) break;
             tc_fence_after();
             const int64_t i = I0 + r;
+            const uint32_t acc_col = tbase + lane_off + (uint32_t)b * GT_ACC;
 #pragma unroll 1
             for (int q = 0; q < GT_BM / 32; ++q) {
                 uint32_t vm[32], vc[32];
-                tmem_ld_32x32b_x32(tbase + lane_off + (uint32_t)q * 32u, vm);
-                tmem_ld_32x32b_x32(tbase + lane_off + 128u + (uint32_t)q * 32u, vc);
+                tmem_ld_32x32b_x32(acc_col + (uint32_t)q * 32u, vm);
+                tmem_ld_32x32b_x32(acc_col + 128u + (uint32_t)q * 32u, vc);
                 tmem_wait_ld();
                 float v[32];
 #pragma unroll
                 for (int e = 0; e < 32; ++e) {
                     float z = __uint_as_float(vm[e]) + __uint_as_float(vc[e]);
-                    const int64_t j = J0 + q * 32 + e;
                     if (MODE == GT_CORR) {
                         z = fabsf(z);
-                        if (i == j) z = 1.f;
+                        if (i == J0 + q * 32 + e) z = 1.f;
                     } else {
                         z *= scale;
                     }
                     v[e] = z;
                 }
-                const int64_t j0 = J0 + q * 32;
-                if (i < n) {
-                    float* dst = S + i * lds + j0;
-                    if (j0 + 32 <= n) {
+                // the staging tiles are free once the last chunk's stores have read them
+                if (r == 0) bulk_wait_read_all();
+                asm volatile("bar.sync 1, 128;" ::: "memory");
+                float* rowp = outD + r * 32;   // row r: 16-byte chunk c sits at c ^ (r & 7)
 #pragma unroll
-                        for (int e = 0; e < 32; e += 4)
-                            *reinterpret_cast<float4*>(dst + e) =
-                                make_float4(v[e], v[e + 1], v[e + 2], v[e + 3]);
-                    } else {
-                        for (int e = 0; e < 32; ++e)
-                            if (j0 + e < n) dst[e] = v[e];
-                    }
+                for (int c = 0; c < 8; ++c)
+                    *reinterpret_cast<float4*>(rowp + ((c ^ (r & 7)) << 2)) =
+                        make_float4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
+                if (!diag) {
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) outT[e * GT_BM + r] = v[e];
                 }
-                if (!diag && i < n) {
-                    // transposed block: lanes write consecutive i of row j (coalesced)
-#pragma unroll
-                    for (int e = 0; e < 32; ++e)
-                        if (j0 + e < n) S[(j0 + e) * lds + i] = v[e];
+                fence_proxy_async_smem();
+                asm volatile("bar.sync 1, 128;" ::: "memory");
+                if (r == 0 && J0 + q * 32 < n) {   // chunks wholly past the end are not stored
+                    tma_store_2d(&mapD, outD, (int32_t)(J0 + q * 32), (int32_t)I0);
+                    if (!diag) tma_store_2d(&mapT, outT, (int32_t)I0, (int32_t)(J0 + q * 32));
+                    bulk_commit_group();
                 }
             }
+            // this accumulator set has been read: the MMA issuer may reuse it
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&acc_empty[b]);
         }
+        if (r == 0 && (ep_fail_sh || !go_sh)) {
+            if (ep_fail_sh) atomicExch(err, 3);
+        }
+        if (r == 0) bulk_wait_all();   // stores complete before the CTA's shared memory goes
     }
 
     tc_fence_before();
@@ -237,28 +293,60 @@ static int gt_map(CUtensorMap* m, const float* base, int64_t Kp, int64_t rows) {
     return SYMNMF_OK;
 }
 
+// Store map over S (n x n, row stride lds floats) with a box of bx x by floats.
+static int gt_store_map(CUtensorMap* m, float* S, int64_t n, int64_t lds, uint32_t bx, uint32_t by,
+                        CUtensorMapSwizzle swz) {
+    auto fn = gt_encode_fn();
+    if (fn == nullptr) {
+        set_error("cuTensorMapEncodeTiled is not available from the driver");
+        return SYMNMF_ERR_NOT_SUPPORTED;
+    }
+    cuuint64_t dims[2] = {(cuuint64_t)n, (cuuint64_t)n};
+    cuuint64_t strides[1] = {(cuuint64_t)lds * sizeof(float)};
+    cuuint32_t box[2] = {bx, by};
+    cuuint32_t estr[2] = {1, 1};
+    const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, S, dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) {
+        set_error("cuTensorMapEncodeTiled (store) failed (%d)", (int)r);
+        return SYMNMF_ERR_CUDA;
+    }
+    return SYMNMF_OK;
+}
+
 // ZF, ZL: n_pad x Kp (n_pad multiple of 128, Kp multiple of 32, zero padding).
 int launch_gram_tc(const float* ZF, const float* ZL, int64_t n, int64_t n_pad, int64_t Kp,
                    bool corr, float scale, float* S, int64_t lds, int* err, cudaStream_t s) {
-    CUtensorMap mapF, mapL;
+    CUtensorMap mapF, mapL, mapD, mapT;
     SYMNMF_TRY(gt_map(&mapF, ZF, Kp, n_pad));
     SYMNMF_TRY(gt_map(&mapL, ZL, Kp, n_pad));
+    SYMNMF_TRY(gt_store_map(&mapD, S, n, lds, 32, GT_BM, CU_TENSOR_MAP_SWIZZLE_128B));
+    SYMNMF_TRY(gt_store_map(&mapT, S, n, lds, GT_BM, 32, CU_TENSOR_MAP_SWIZZLE_NONE));
     const int64_t nt = n_pad / GT_BM;
     const int64_t pairs = nt * (nt + 1) / 2;
-    if (pairs > 0x7fffffffLL) {
-        set_error("n = %lld too large for the Gram tile grid", (long long)n);
-        return SYMNMF_ERR_INVALID_ARG;
-    }
+    int dev = 0, sms = 148;
+    SYMNMF_CUDA_TRY(cudaGetDevice(&dev));
+    SYMNMF_CUDA_TRY(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
+    const unsigned grid = (unsigned)std::min<int64_t>(pairs, sms);   // persistent, one CTA per SM
     if (corr) {
-        SYMNMF_CUDA_TRY(cudaFuncSetAttribute(gram_tc_kernel<GT_CORR>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)GT_SMEM));
-        gram_tc_kernel<GT_CORR><<<(unsigned)pairs, GT_THREADS, GT_SMEM, s>>>(mapF, mapL, n, (int)Kp,
-                                                                            scale, S, lds, err);
+        static bool attr = false;   // once per process
+        if (!attr) {
+            SYMNMF_CUDA_TRY(cudaFuncSetAttribute(gram_tc_kernel<GT_CORR>,
+                                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)GT_SMEM));
+            attr = true;
+        }
+        gram_tc_kernel<GT_CORR><<<grid, GT_THREADS, GT_SMEM, s>>>(mapF, mapL, mapD, mapT, n, (int)Kp,
+                                                                 pairs, scale, err);
     } else {
-        SYMNMF_CUDA_TRY(cudaFuncSetAttribute(gram_tc_kernel<GT_TPDM>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)GT_SMEM));
-        gram_tc_kernel<GT_TPDM><<<(unsigned)pairs, GT_THREADS, GT_SMEM, s>>>(mapF, mapL, n, (int)Kp,
-                                                                            scale, S, lds, err);
+        static bool attr = false;
+        if (!attr) {
+            SYMNMF_CUDA_TRY(cudaFuncSetAttribute(gram_tc_kernel<GT_TPDM>,
+                                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)GT_SMEM));
+            attr = true;
+        }
+        gram_tc_kernel<GT_TPDM><<<grid, GT_THREADS, GT_SMEM, s>>>(mapF, mapL, mapD, mapT, n, (int)Kp,
+                                                                 pairs, scale, err);
     }
     SYMNMF_LAUNCH_CHECK();
     return SYMNMF_OK;
