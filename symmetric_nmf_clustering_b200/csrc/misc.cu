@@ -55,12 +55,22 @@ stats_partial_kernel(const float* __restrict__ S, int64_t n, int64_t lds,
                 const float e[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
 #pragma unroll
                 for (int w = 0; w < 4; ++w) {
-                    if (isfinite(e[w])) {
+                    // widen to fp64 by moving the bit fields (exact for normal
+                    // floats): the conversion instruction's throughput, not
+                    // HBM, limited this pass
+                    const uint32_t b = __float_as_uint(e[w]);
+                    const uint32_t ex = (b >> 23) & 0xFFu;
+                    if (ex - 1u < 254u) {
+                        const uint32_t hi = (b & 0x80000000u) | ((ex + 896u) << 20) | ((b >> 3) & 0x000FFFFFu);
+                        const double d = __hiloint2double((int)hi, (int)(b << 29));
+                        sum += d;
+                        sq = fma(d, d, sq);
+                    } else if (ex == 0xFFu) {
+                        bad += 1.0;
+                    } else {   // zero or subnormal
                         const double d = e[w];
                         sum += d;
                         sq = fma(d, d, sq);
-                    } else {
-                        bad += 1.0;
                     }
                 }
             }
