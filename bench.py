@@ -286,6 +286,32 @@ def measure_rows(m, torch, dev, S, H0, lab, n, k, T, rank, workload):
     return out
 
 
+def row_rooflines(rows, n, k, T, hbm_peak):
+    """Algorithmic traffic (or flops) of each timed row over its time, as a fraction of
+    the measured peaks: HBM copy bandwidth for streams, and for the |corr| Gram the
+    TF32 rate taken as half the measured bf16 rate (the nominal ratio)."""
+    out = {}
+    sbytes = 4.0 * n * n
+    def hbm(name, bytes_, ms):
+        if ms and ms > 0:
+            gbs = bytes_ / (ms / 1e3) / 1e9
+            out[name] = {"bound": "hbm", "GBs": gbs, "frac": gbs / hbm_peak}
+    hbm("stats", sbytes, rows.get("stats_ms"))
+    if "kmeans_steps" in rows:
+        # two S passes per assignment step; the last step stops after its assignment
+        hbm("kmeans_step", 2 * sbytes, rows.get("kmeans_ms_per_step"))
+    if "svrg_epoch_ms" in rows:
+        hbm("svrg_epoch", 2 * sbytes, rows.get("svrg_epoch_ms"))   # snapshot pass + all blocks
+    if "tpdm_build_ms" in rows:
+        hbm("tpdm_build_writes", sbytes, rows.get("tpdm_build_ms"))
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            tf32 = 0.5 * float(json.load(f)["bf16_tflops"])
+    except Exception:
+        tf32 = 0.5 * 1590.0
+    return out, tf32
+
+
 # ----------------------------------------------------------------------------- reference arm
 def run_reference(args):
     world, rank, _ = dist_env()
@@ -427,6 +453,11 @@ def run_ours(args):
     rows = None
     if not args.no_rows:
         rows = measure_rows(m, torch, dev, S, H0, lab, n, k, T, rank, args.workload)
+        rows["roofline"], tf32_peak = row_rooflines(rows, n, k, T, peak)
+        rows["roofline"]["corr_build"] = {
+            "bound": "tensor", "tf32_TFs": 3.0 * n * n * T / (build_ms / 1e3) / 1e12,
+            "peak_TFs": tf32_peak, "frac": 3.0 * n * n * T / (build_ms / 1e3) / 1e12 / tf32_peak,
+            "flops": "3 n^2 T (exact TF32 split, upper triangle of tiles)"}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -455,7 +486,8 @@ def run_ours(args):
             "e2e": e2e,
             "cpu_baseline": cpu,
             "rows": rows,
-            "context": {"corr_build_ms": build_ms, "torch_mm_S_H_ms": mm_ms,
+            "context": {"corr_build_ms": build_ms,
+                        "corr_build_tf32_TFs": 3.0 * n * n * T / (build_ms / 1e3) / 1e12, "torch_mm_S_H_ms": mm_ms,
                         "ARI_vs_planted": oracle.ari(lab.cpu().numpy(), planted),
                         "final_loss": st["loss"], "loop_ms": st["loop_ms"]},
         }
