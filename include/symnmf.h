@@ -34,7 +34,9 @@
  *    caller-provided workspace `ws` of `ws_bytes` bytes (256-byte aligned),
  *    sized by symnmf_workspace_size(); too small gives SYMNMF_ERR_WORKSPACE.
  *  - Streams: work is issued on `stream` (NULL = the legacy default stream).
- *    Builders, symnmf_sh, symnmf_stats and symnmf_labels are asynchronous.
+ *    symnmf_stats and symnmf_labels are asynchronous.  The tensor-core builders,
+ *    symnmf_sh and symnmf_sh_noalloc synchronise `stream` at the end to read
+ *    their device error word (SYMNMF_ERR_TIMEOUT when a bounded wait gave up).
  *    symnmf_fit and symnmf_spectral_probe write host outputs and synchronise
  *    `stream` before they return.
  *  - Errors: every call returns a symnmf_status; SYMNMF_OK = 0.  A failing
@@ -161,7 +163,7 @@ SYMNMF_API int symnmf_workspace_size(int op, int64_t n, int k, int64_t T,
  * S_ij = |sum_t z_ti z_tj| / sqrt(sum_t z_ti^2 sum_t z_tj^2) with z the
  * column-centred returns; S_ii = 1; a zero-variance column gives a zero row
  * and column apart from S_ii = 1.  Column means and norms in fp64.
- * Requires T >= 2.  Asynchronous.
+ * Requires T >= 2.  Synchronises `stream` (reads the device error word).
  */
 SYMNMF_API int symnmf_build_corr(const float* R, int64_t T, int64_t n, int64_t ldr,
                       float* S, int64_t lds, void* ws, size_t ws_bytes,
@@ -175,7 +177,8 @@ SYMNMF_API int symnmf_build_corr(const float* R, int64_t T, int64_t n, int64_t l
  *   rho_t = ||x_t||_2                         (fp64)
  *   E     = the N = max(1, floor(tail_frac*T)) days of largest rho (ties -> earlier day)
  *   S_ij  = (n/N) sum_{t in E} (x_ti/rho_t)(x_tj/rho_t)
- * tail_frac in (0, 1]; tail_sign = +1 or -1.  R must be finite.  Asynchronous.
+ * tail_frac in (0, 1]; tail_sign = +1 or -1.  R must be finite.  Synchronises
+ * `stream` (reads the device error word).
  */
 SYMNMF_API int symnmf_build_tpdm(const float* R, int64_t T, int64_t n, int64_t ldr,
                       double tail_frac, int tail_sign, float* S, int64_t lds,
@@ -192,7 +195,8 @@ SYMNMF_API int symnmf_stats(const float* S, int64_t n, int64_t lds, double* out_
 
 /*
  * Y = S X: one pass of the S-stream ([CaS] "Factorization at scale": the
- * dominant S H products) for X, Y n x k (1 <= k <= 64).  Asynchronous.
+ * dominant S H products) for X, Y n x k (1 <= k <= 64).  Synchronises `stream`
+ * (reads the device error word).
  */
 SYMNMF_API int symnmf_sh(const float* S, int64_t n, int64_t lds, const float* X, int k,
               float* Y, void* ws, size_t ws_bytes, symnmf_stream_t stream);
@@ -362,7 +366,7 @@ SYMNMF_API int symnmf_rolling(const float* R, int64_t days, int64_t n, int64_t l
  * Every call shares the one array and it keeps the last call's contents:
  * calls that overlap on the GPU (on different streams, or from several host
  * threads without ordering) race on it.  S, X, Y as for symnmf_sh.
- * Asynchronous on `stream`.
+ * Synchronises `stream` at the end (reads the error word).
  */
 SYMNMF_API int symnmf_sh_noalloc(const float* S, int64_t n, int64_t lds, const float* X, int k,
                                  float* Y, symnmf_stream_t stream);

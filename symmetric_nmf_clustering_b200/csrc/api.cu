@@ -1383,7 +1383,16 @@ int symnmf_sh(const float* S, int64_t n, int64_t lds, const float* X, int k, flo
     cudaStream_t s = (cudaStream_t)stream;
     SYMNMF_CUDA_TRY(cudaMemsetAsync(sa.err, 0, sizeof(int), s));
     SYMNMF_CUDA_TRY(cudaMemsetAsync(sa.counters, 0, (size_t)epilogue_blocks(n) * sizeof(int), s));
-    return stream_pass(d, sa, X, nullptr, k, 0, n, false, epi_product(n, k, Y), s, nullptr);
+    SYMNMF_TRY(stream_pass(d, sa, X, nullptr, k, 0, n, false, epi_product(n, k, Y), s, nullptr));
+    // a bounded device-side wait that gave up is reported in the error word
+    int h = 0;
+    SYMNMF_CUDA_TRY(cudaMemcpyAsync(&h, sa.err, sizeof(int), cudaMemcpyDeviceToHost, s));
+    SYMNMF_CUDA_TRY(cudaStreamSynchronize(s));
+    if (h != 0) {
+        set_error("an S-stream pipeline wait timed out on the device (code %d)", h);
+        return SYMNMF_ERR_TIMEOUT;
+    }
+    return SYMNMF_OK;
 }
 
 int symnmf_spectral_probe(const float* S, int64_t n, int64_t lds, int n_eig, int block,

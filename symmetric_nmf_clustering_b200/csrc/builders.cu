@@ -219,6 +219,19 @@ __global__ void normalize_t_kernel(const float* __restrict__ R, int64_t T, int64
     }
 }
 
+// The tensor-core Gram reports a bounded device-side wait that gave up in its
+// error word; read it (this synchronises the stream).
+static int gram_status(const int* err, cudaStream_t s) {
+    int h = 0;
+    SYMNMF_CUDA_TRY(cudaMemcpyAsync(&h, err, sizeof(int), cudaMemcpyDeviceToHost, s));
+    SYMNMF_CUDA_TRY(cudaStreamSynchronize(s));
+    if (h != 0) {
+        set_error("a builder pipeline wait timed out on the device (code %d)", h);
+        return SYMNMF_ERR_TIMEOUT;
+    }
+    return SYMNMF_OK;
+}
+
 int launch_corr(const float* R, int64_t T, int64_t n, int64_t ldr, float* S,
                 int64_t lds, double* mu, double* inv, float* Z, int64_t ldz,
                 cudaStream_t s) {
@@ -233,7 +246,8 @@ int launch_corr(const float* R, int64_t T, int64_t n, int64_t ldr, float* S,
         dim3 grid((unsigned)(n_pad / 32), (unsigned)(Kt / 32));
         normalize_t_kernel<<<grid, dim3(32, 8), 0, s>>>(R, T, n, ldr, mu, inv, ZF, ZL, Kt);
         SYMNMF_LAUNCH_CHECK();
-        return launch_gram_tc(ZF, ZL, n, n_pad, Kt, true, 1.f, S, lds, err, s);
+        SYMNMF_TRY(launch_gram_tc(ZF, ZL, n, n_pad, Kt, true, 1.f, S, lds, err, s));
+        return gram_status(err, s);
     }
     const int64_t Kp = round_up(T, GK);
     const int64_t total = Kp * ldz;
@@ -491,7 +505,8 @@ int launch_tpdm(const float* R, int64_t T, int64_t n, int64_t ldr, int N,
         const int64_t blocks = min64((total + 255) / 256, 8192);
         gather_wt_kernel<<<(unsigned)blocks, 256, 0, s>>>(ranks, phi, rho, days, N, n, WF, WL, n_pad, Kt);
         SYMNMF_LAUNCH_CHECK();
-        return launch_gram_tc(WF, WL, n, n_pad, Kt, false, scale, S, lds, err, s);
+        SYMNMF_TRY(launch_gram_tc(WF, WL, n, n_pad, Kt, false, scale, S, lds, err, s));
+        return gram_status(err, s);
     }
     const int64_t Np = round_up(N, GK);
     const int64_t total = Np * ldw;

@@ -47,13 +47,44 @@ constexpr uint32_t GT_TMEM_COLS = 2 * GT_ACC;      // two sets: a tile drains wh
 
 enum GramTcMode { GT_CORR = 0, GT_TPDM = 1 };
 
-// tile (I, J), I <= J, from its linear index over the upper triangle
-__device__ __forceinline__ void gt_tile(int64_t x, int64_t* I, int64_t* J) {
+// (a, b), a <= b, from a linear index over an upper triangle, b-major
+__device__ __forceinline__ void gt_tri(int64_t x, int64_t* a, int64_t* b) {
     int64_t j = (int64_t)((sqrt(8.0 * (double)x + 1.0) - 1.0) * 0.5);
     while ((j + 1) * (j + 2) / 2 <= x) ++j;
     while (j * (j + 1) / 2 > x) --j;
-    *J = j;
-    *I = x - j * (j + 1) / 2;
+    *b = j;
+    *a = x - j * (j + 1) / 2;
+}
+
+// The tiles are visited in groups of GT_GROUP x GT_GROUP (the tile grid padded
+// to whole groups, groups column-major over the upper triangle), so that the
+// CTAs running at the same time share GT_GROUP row blocks of each operand in
+// L2 instead of each fetching its own.  Tiles in the padding are skipped, by
+// every role alike.
+constexpr int64_t GT_GROUP = 16;
+constexpr int64_t GT_G2 = GT_GROUP * GT_GROUP, GT_GD = GT_GROUP * (GT_GROUP + 1) / 2;
+__host__ __device__ __forceinline__ int64_t gt_before(int64_t c) {   // tiles in group columns < c
+    return GT_G2 * c * (c - 1) / 2 + c * GT_GD;
+}
+int64_t gt_virtual_tiles(int64_t nt) { return gt_before((nt + GT_GROUP - 1) / GT_GROUP); }
+
+// tile (I, J), I <= J, of virtual index v; false for a tile in the padding
+__device__ __forceinline__ bool gt_tile(int64_t v, int64_t nt, int64_t* I, int64_t* J) {
+    int64_t c = (int64_t)(sqrt(2.0 * (double)v) / (double)GT_GROUP);
+    while (c > 0 && gt_before(c) > v) --c;
+    while (gt_before(c + 1) <= v) ++c;
+    const int64_t off = v - gt_before(c);
+    if (off < c * GT_G2) {   // off-diagonal group (gi, c), gi < c
+        const int64_t gi = off / GT_G2, l = off % GT_G2;
+        *I = gi * GT_GROUP + l / GT_GROUP;
+        *J = c * GT_GROUP + l % GT_GROUP;
+    } else {                 // diagonal group (c, c)
+        int64_t a, b;
+        gt_tri(off - c * GT_G2, &a, &b);
+        *I = c * GT_GROUP + a;
+        *J = c * GT_GROUP + b;
+    }
+    return *J < nt;
 }
 
 // Persistent: CTA b takes the tiles b, b + grid, b + 2 grid, ...
@@ -61,7 +92,7 @@ template <int MODE>
 __global__ void __launch_bounds__(GT_THREADS, 1)
 gram_tc_kernel(const __grid_constant__ CUtensorMap mapF, const __grid_constant__ CUtensorMap mapL,
                const __grid_constant__ CUtensorMap mapD, const __grid_constant__ CUtensorMap mapT,
-               int64_t n, int Kp, int64_t pairs, float scale, int* __restrict__ err) {
+               int64_t n, int Kp, int64_t vtiles, float scale, int* __restrict__ err) {
     using namespace sm100;
     extern __shared__ uint8_t gt_smem_raw[];
     __shared__ __align__(8) uint64_t bar_full[GT_NS], bar_empty[GT_NS];
@@ -75,6 +106,7 @@ gram_tc_kernel(const __grid_constant__ CUtensorMap mapF, const __grid_constant__
     float* outT = outD + GT_BM * 32;                                   // [32 rows][128], plain
 
     const int ksteps = Kp / GT_BK;
+    const int64_t nt = (n + GT_BM - 1) / GT_BM;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     if (tid == 0) {
         for (int s = 0; s < GT_NS; ++s) {
@@ -109,9 +141,9 @@ gram_tc_kernel(const __grid_constant__ CUtensorMap mapF, const __grid_constant__
     if (warp == 0 && lane == 0) {
         // ---------------- TMA producer: one stage ring across all of this CTA's tiles
         int64_t g = 0;   // stages issued
-        for (int64_t x = blockIdx.x; x < pairs && !abort_sh; x += gridDim.x) {
+        for (int64_t x = blockIdx.x; x < vtiles && !abort_sh; x += gridDim.x) {
             int64_t I, J;
-            gt_tile(x, &I, &J);
+            if (!gt_tile(x, nt, &I, &J)) continue;
             const bool diag = I == J;
             const uint32_t stage_bytes = diag ? 2 * GT_PLANE : 4 * GT_PLANE;
             for (int s = 0; s < ksteps; ++s, ++g) {
@@ -141,9 +173,9 @@ gram_tc_kernel(const __grid_constant__ CUtensorMap mapF, const __grid_constant__
         constexpr uint32_t id = idesc_tf32(GT_BM, GT_BM);
         int64_t g = 0;
         int u = 0;
-        for (int64_t x = blockIdx.x; x < pairs && !abort_sh; x += gridDim.x, ++u) {
+        for (int64_t x = blockIdx.x; x < vtiles && !abort_sh; x += gridDim.x) {
             int64_t I, J;
-            gt_tile(x, &I, &J);
+            if (!gt_tile(x, nt, &I, &J)) continue;
             const bool diag = I == J;
             const int b = u & 1;
             if (u >= 2 && !mbar_wait(&acc_empty[b], (uint32_t)((u >> 1) - 1) & 1u)) {
@@ -177,6 +209,7 @@ gram_tc_kernel(const __grid_constant__ CUtensorMap mapF, const __grid_constant__
             }
             if (abort_sh) break;
             umma_commit(&acc_full[b]);
+            ++u;
         }
         umma_commit(&bar_fin);
         mbar_wait(&bar_fin, 0);   // every MMA has finished before TMEM is freed
@@ -187,13 +220,15 @@ gram_tc_kernel(const __grid_constant__ CUtensorMap mapF, const __grid_constant__
         const int r = wl * 32 + lane;
         const uint32_t lane_off = (uint32_t)(wl * 32) << 16;
         int u = 0;
-        for (int64_t x = blockIdx.x; x < pairs; x += gridDim.x, ++u) {
+        for (int64_t x = blockIdx.x; x < vtiles; x += gridDim.x) {
             int64_t I, J;
-            gt_tile(x, &I, &J);
+            if (!gt_tile(x, nt, &I, &J)) continue;
             const bool diag = I == J;
             const int b = u & 1;
+            const uint32_t par = (uint32_t)(u >> 1) & 1u;   // this tile's use of set b
+            ++u;
             const int64_t I0 = I * GT_BM, J0 = J * GT_BM;
-            const bool w_ok = __all_sync(0xffffffffu, mbar_wait(&acc_full[b], (uint32_t)(u >> 1) & 1u));
+            const bool w_ok = __all_sync(0xffffffffu, mbar_wait(&acc_full[b], par));
             if (lane == 0 && !w_ok) atomicOr(const_cast<int*>(&ep_fail_sh), 1);
             asm volatile("bar.sync 1, 128;" ::: "memory");
             if (r == 0) go_sh = (ep_fail_sh == 0 && abort_sh == 0) ? 1 : 0;
@@ -324,11 +359,11 @@ int launch_gram_tc(const float* ZF, const float* ZL, int64_t n, int64_t n_pad, i
     SYMNMF_TRY(gt_store_map(&mapD, S, n, lds, 32, GT_BM, CU_TENSOR_MAP_SWIZZLE_128B));
     SYMNMF_TRY(gt_store_map(&mapT, S, n, lds, GT_BM, 32, CU_TENSOR_MAP_SWIZZLE_NONE));
     const int64_t nt = n_pad / GT_BM;
-    const int64_t pairs = nt * (nt + 1) / 2;
+    const int64_t vtiles = gt_virtual_tiles(nt);
     int dev = 0, sms = 148;
     SYMNMF_CUDA_TRY(cudaGetDevice(&dev));
     SYMNMF_CUDA_TRY(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
-    const unsigned grid = (unsigned)std::min<int64_t>(pairs, sms);   // persistent, one CTA per SM
+    const unsigned grid = (unsigned)std::min<int64_t>(nt * (nt + 1) / 2, sms);   // persistent, one CTA per SM
     if (corr) {
         static bool attr = false;   // once per process
         if (!attr) {
@@ -337,7 +372,7 @@ int launch_gram_tc(const float* ZF, const float* ZL, int64_t n, int64_t n_pad, i
             attr = true;
         }
         gram_tc_kernel<GT_CORR><<<grid, GT_THREADS, GT_SMEM, s>>>(mapF, mapL, mapD, mapT, n, (int)Kp,
-                                                                 pairs, scale, err);
+                                                                 vtiles, scale, err);
     } else {
         static bool attr = false;
         if (!attr) {
@@ -346,7 +381,7 @@ int launch_gram_tc(const float* ZF, const float* ZL, int64_t n, int64_t n_pad, i
             attr = true;
         }
         gram_tc_kernel<GT_TPDM><<<grid, GT_THREADS, GT_SMEM, s>>>(mapF, mapL, mapD, mapT, n, (int)Kp,
-                                                                 pairs, scale, err);
+                                                                 vtiles, scale, err);
     }
     SYMNMF_LAUNCH_CHECK();
     return SYMNMF_OK;

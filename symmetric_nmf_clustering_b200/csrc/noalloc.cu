@@ -99,5 +99,14 @@ extern "C" int symnmf_sh_noalloc(const float* S, int64_t n, int64_t lds, const f
     // the array keeps the previous call's contents: the error word starts at zero
     SYMNMF_CUDA_TRY(cudaMemsetAsync(err, 0, sizeof(int), s));
     SYMNMF_TRY(launch_split(X, nullptr, k, k, 0, n, p.j0, p.j1, XT, ldxt, s));
-    return launch_stream_tc(p, S, lds, XT, ldxt, Y, err, nullptr, s);
+    SYMNMF_TRY(launch_stream_tc(p, S, lds, XT, ldxt, Y, err, nullptr, s));
+    // a bounded device-side wait that gave up is reported in the error word
+    int h = 0;
+    SYMNMF_CUDA_TRY(cudaMemcpyAsync(&h, err, sizeof(int), cudaMemcpyDeviceToHost, s));
+    SYMNMF_CUDA_TRY(cudaStreamSynchronize(s));
+    if (h != 0) {
+        set_error("an S-stream pipeline wait timed out on the device (code %d)", h);
+        return SYMNMF_ERR_TIMEOUT;
+    }
+    return SYMNMF_OK;
 }

@@ -65,7 +65,9 @@ def test_sh_matches_oracle(m, n, k):
     assert rel_fro(Y, ref) <= 2e-6   # regression guard: fp32-class error, far inside the bound
 
 
-@pytest.mark.parametrize("T,n", [(250, 2000), (250, 1999), (2, 37), (17, 130), (1000, 600)])
+# n = 4,100: 561 tiles, several per CTA of the persistent Gram (both TMEM
+# accumulator sets and their barrier phases in use)
+@pytest.mark.parametrize("T,n", [(250, 2000), (250, 1999), (2, 37), (17, 130), (1000, 600), (60, 4100)])
 def test_corr_builder(m, T, n):
     R, _, _ = synth.workload("corr_n2000_k8", seed=T + n, n=n, T=T)
     S = m.build_corr(to_dev(R, DEV, pad4=True)).cpu().numpy()
@@ -83,8 +85,12 @@ def test_corr_builder_zero_variance_column(m):
     assert S[5, 5] == 1.0 and np.all(S[5, np.arange(64) != 5] == 0.0)
 
 
+# T <= 2048 ranks by sorting (2048 is the largest sort); T = 2100 takes the
+# counting kernel
 @pytest.mark.parametrize("T,n,frac,sign", [(250, 2000, 0.05, 1), (1000, 1999, 0.05, 1),
-                                           (100, 130, 0.1, -1), (20, 2, 0.1, 1), (1, 5, 1.0, 1)])
+                                           (100, 130, 0.1, -1), (20, 2, 0.1, 1), (1, 5, 1.0, 1),
+                                           (2048, 45, 0.05, -1), (2100, 37, 0.05, 1),
+                                           (80, 4100, 0.1, 1)])
 def test_tpdm_builder(m, T, n, frac, sign):
     R, _, _ = synth.workload("tpdm_n20000_k24", seed=T + n, n=n, T=T)
     S = m.build_tpdm(to_dev(R, DEV, pad4=True), frac, sign).cpu().numpy()
