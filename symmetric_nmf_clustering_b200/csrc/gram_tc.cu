@@ -36,16 +36,25 @@ namespace symnmf {
 
 constexpr int GT_BM = 128;                    // tile rows and columns
 constexpr int GT_BK = 32;                     // contraction columns per stage
-constexpr int GT_NS = 3;                      // pipeline stages
+constexpr int GT_NS_MAX = 3;                  // pipeline stages (|corr|; TPDM uses 2)
 constexpr int GT_THREADS = 256;
 constexpr uint32_t GT_PLANE = GT_BM * GT_BK * 4;   // 16 KB: 128 rows x 128 B
 constexpr uint32_t GT_STAGE = 4 * GT_PLANE;        // AF, AL, BF, BL
 constexpr uint32_t GT_OUT = GT_BM * 32 * 4;        // 16 KB: one 32-column output chunk
-constexpr uint32_t GT_SMEM = GT_NS * GT_STAGE + 2 * GT_OUT + 1024;
+// |corr| (long contraction): a 3-stage ring, one staging pair for the output;
+// TPDM (2 stages per tile, bound by the writes): a 2-stage ring and two staging
+// pairs, so a chunk is written while the previous chunk's stores still read
+template <int MODE> struct GtShape;
 constexpr uint32_t GT_ACC = 256;                   // one accumulator set: main [0,128), correction [128,256)
 constexpr uint32_t GT_TMEM_COLS = 2 * GT_ACC;      // two sets: a tile drains while the next accumulates
 
 enum GramTcMode { GT_CORR = 0, GT_TPDM = 1 };
+template <> struct GtShape<GT_CORR> { static constexpr int NS = 3, NOUT = 1; };
+template <> struct GtShape<GT_TPDM> { static constexpr int NS = 2, NOUT = 2; };
+template <int MODE>
+constexpr uint32_t gt_smem() {
+    return GtShape<MODE>::NS * GT_STAGE + GtShape<MODE>::NOUT * 2 * GT_OUT + 1024;
+}
 
 // (a, b), a <= b, from a linear index over an upper triangle, b-major
 __device__ __forceinline__ void gt_tri(int64_t x, int64_t* a, int64_t* b) {
@@ -95,15 +104,17 @@ gram_tc_kernel(const __grid_constant__ CUtensorMap mapF, const __grid_constant__
                int64_t n, int Kp, int64_t vtiles, float scale, int* __restrict__ err) {
     using namespace sm100;
     extern __shared__ uint8_t gt_smem_raw[];
-    __shared__ __align__(8) uint64_t bar_full[GT_NS], bar_empty[GT_NS];
+    constexpr int GT_NS = GtShape<MODE>::NS, NOUT = GtShape<MODE>::NOUT;
+    static_assert(gt_smem<MODE>() <= 227 * 1024, "shared memory per block");
+    __shared__ __align__(8) uint64_t bar_full[GT_NS_MAX], bar_empty[GT_NS_MAX];
     __shared__ __align__(8) uint64_t acc_full[2], acc_empty[2], bar_fin;
     __shared__ uint32_t tmem_base_sh;
     __shared__ volatile int abort_sh, ep_fail_sh, go_sh;
 
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(gt_smem_raw) + 1023) & ~uintptr_t(1023));
-    float* outD = reinterpret_cast<float*>(smem + GT_NS * GT_STAGE);   // [128 rows][32], 128B swizzle
-    float* outT = outD + GT_BM * 32;                                   // [32 rows][128], plain
+    // staging pair p: outD(p) [128 rows][32] with 128-byte swizzle, then outT(p) [32 rows][128]
+    float* outBase = reinterpret_cast<float*>(smem + GT_NS * GT_STAGE);
 
     const int ksteps = Kp / GT_BK;
     const int64_t nt = (n + GT_BM - 1) / GT_BM;
@@ -219,7 +230,7 @@ gram_tc_kernel(const __grid_constant__ CUtensorMap mapF, const __grid_constant__
         const int wl = warp & 3;
         const int r = wl * 32 + lane;
         const uint32_t lane_off = (uint32_t)(wl * 32) << 16;
-        int u = 0;
+        int u = 0, cq = 0;   // tiles and output chunks handled
         for (int64_t x = blockIdx.x; x < vtiles; x += gridDim.x) {
             int64_t I, J;
             if (!gt_tile(x, nt, &I, &J)) continue;
@@ -256,7 +267,13 @@ gram_tc_kernel(const __grid_constant__ CUtensorMap mapF, const __grid_constant__
                     v[e] = z;
                 }
                 // the staging tiles are free once the last chunk's stores have read them
-                if (r == 0) bulk_wait_read_all();
+                float* outD = outBase + (size_t)(cq % NOUT) * 2 * GT_BM * 32;
+                float* outT = outD + GT_BM * 32;
+                ++cq;
+                if (r == 0) {
+                    if (NOUT == 2) bulk_wait_read_but_one();   // the pair written two chunks ago is free
+                    else bulk_wait_read_all();
+                }
                 asm volatile("bar.sync 1, 128;" ::: "memory");
                 float* rowp = outD + r * 32;   // row r: 16-byte chunk c sits at c ^ (r & 7)
 #pragma unroll
@@ -269,10 +286,12 @@ gram_tc_kernel(const __grid_constant__ CUtensorMap mapF, const __grid_constant__
                 }
                 fence_proxy_async_smem();
                 asm volatile("bar.sync 1, 128;" ::: "memory");
-                if (r == 0 && J0 + q * 32 < n) {   // chunks wholly past the end are not stored
-                    tma_store_2d(&mapD, outD, (int32_t)(J0 + q * 32), (int32_t)I0);
-                    if (!diag) tma_store_2d(&mapT, outT, (int32_t)I0, (int32_t)(J0 + q * 32));
-                    bulk_commit_group();
+                if (r == 0) {
+                    if (J0 + q * 32 < n) {   // chunks wholly past the end are not stored
+                        tma_store_2d(&mapD, outD, (int32_t)(J0 + q * 32), (int32_t)I0);
+                        if (!diag) tma_store_2d(&mapT, outT, (int32_t)I0, (int32_t)(J0 + q * 32));
+                    }
+                    bulk_commit_group();   // one group per chunk (possibly empty): the waits count chunks
                 }
             }
             // this accumulator set has been read: the MMA issuer may reuse it
@@ -368,19 +387,19 @@ int launch_gram_tc(const float* ZF, const float* ZL, int64_t n, int64_t n_pad, i
         static bool attr = false;   // once per process
         if (!attr) {
             SYMNMF_CUDA_TRY(cudaFuncSetAttribute(gram_tc_kernel<GT_CORR>,
-                                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)GT_SMEM));
+                                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)gt_smem<GT_CORR>()));
             attr = true;
         }
-        gram_tc_kernel<GT_CORR><<<grid, GT_THREADS, GT_SMEM, s>>>(mapF, mapL, mapD, mapT, n, (int)Kp,
+        gram_tc_kernel<GT_CORR><<<grid, GT_THREADS, gt_smem<GT_CORR>(), s>>>(mapF, mapL, mapD, mapT, n, (int)Kp,
                                                                  vtiles, scale, err);
     } else {
         static bool attr = false;
         if (!attr) {
             SYMNMF_CUDA_TRY(cudaFuncSetAttribute(gram_tc_kernel<GT_TPDM>,
-                                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)GT_SMEM));
+                                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)gt_smem<GT_TPDM>()));
             attr = true;
         }
-        gram_tc_kernel<GT_TPDM><<<grid, GT_THREADS, GT_SMEM, s>>>(mapF, mapL, mapD, mapT, n, (int)Kp,
+        gram_tc_kernel<GT_TPDM><<<grid, GT_THREADS, gt_smem<GT_TPDM>(), s>>>(mapF, mapL, mapD, mapT, n, (int)Kp,
                                                                  vtiles, scale, err);
     }
     SYMNMF_LAUNCH_CHECK();
