@@ -371,6 +371,15 @@ SYMNMF_API int symnmf_rolling(const float* R, int64_t days, int64_t n, int64_t l
 SYMNMF_API int symnmf_sh_noalloc(const float* S, int64_t n, int64_t lds, const float* X, int k,
                                  float* Y, symnmf_stream_t stream);
 
+/*
+ * Test hook for failure detection (no counterpart on the pages).  on != 0:
+ * the S-stream kernel's TMA producer issues no loads on the current device,
+ * so every bounded pipeline wait of the next S-stream launches runs out
+ * (about 2 s) and those calls return SYMNMF_ERR_TIMEOUT with the CUDA context
+ * intact; on = 0 restores normal operation.  Synchronous.
+ */
+SYMNMF_API int symnmf_test_stall_pipeline(int on);
+
 #ifdef __cplusplus
 }
 #endif

@@ -140,6 +140,7 @@ SIGNATURES = {
     "symnmf_ari": (_int, [_vp, _vp, _i64, _int, C.POINTER(C.c_double), C.POINTER(C.c_int64), _vp,
                           _sz, _vp]),
     "symnmf_rolling_params_default": (None, [C.POINTER(RollingParams)]),
+    "symnmf_test_stall_pipeline": (_int, [_int]),
     "symnmf_rolling": (_int, [_vp, _i64, _i64, _i64, _vp, _vp, _i64, C.POINTER(RollingParams),
                               C.POINTER(RollingOut), _vp, _sz, _vp]),
 }

@@ -235,6 +235,10 @@ reduce_finalize_kernel(int mode, int nblk, int k, const double* __restrict__ tr_
                        FinalScratch* fs, double rel_tol, int max_evals,
                        double* history, int history_cap) {
     if (st->done) return;
+    if (st->kerr != 0) {   // the S-stream gave up waiting: stop the loop, no result this pass
+        if (blockIdx.x == 0 && threadIdx.x == 0) st->done = 1;
+        return;
+    }
     __shared__ double sh[8][32];
     __shared__ bool last;
     const int kk = k * k;

@@ -41,6 +41,11 @@
 
 namespace symnmf {
 
+// Test hook (symnmf_test_stall_pipeline): when set, the TMA producer issues no
+// loads, so the consumers' bounded waits run out and the launch returns its
+// error word instead of a result.
+__device__ int g_stall_producer = 0;
+
 // Pipeline shape (compile-time).  SYMNMF_TC_A_SMEM = 1: the first MMA reads S
 // straight from shared memory; the tensor core truncates fp32 operands to
 // TF32, which is exactly S_hi (measured on B200: bit-identical results to
@@ -177,7 +182,7 @@ stream_tc_kernel(const __grid_constant__ CUtensorMap mapS, const __grid_constant
     tc_fence_after();
     const uint32_t tbase = tmem_base_sh;
 
-    if (warp == 0 && lane == 0 && ksteps > 0) {
+    if (warp == 0 && lane == 0 && ksteps > 0 && *(volatile int*)&g_stall_producer == 0) {
         // ---------------- TMA producer
         int issued = 0;
         const uint64_t pol_s = SYMNMF_TC_L2HINT ? policy_evict_first() : 0;
@@ -519,3 +524,14 @@ int launch_stream_tc(const TcPlan& p, const float* S, int64_t lds, const float* 
 }
 
 }  // namespace symnmf
+
+extern "C" int symnmf_test_stall_pipeline(int on) {
+    symnmf::clear_error();
+    const int v = on ? 1 : 0;
+    const cudaError_t e = cudaMemcpyToSymbol(symnmf::g_stall_producer, &v, sizeof(int));
+    if (e != cudaSuccess) {
+        symnmf::set_error("cudaMemcpyToSymbol failed: %s", cudaGetErrorString(e));
+        return SYMNMF_ERR_CUDA;
+    }
+    return SYMNMF_OK;
+}
