@@ -320,7 +320,7 @@ static int read_state(const FitState* st, HostState* h, cudaStream_t s) {
     h->rel = tmp.rel;
     h->t = tmp.t;
     h->t_stop = tmp.t_stop;
-    h->done = tmp.done;
+    h->done = tmp.done || tmp.kerr != 0;   // a pass that gave up waiting ends the loop
     h->converged = tmp.converged;
     h->nonfinite = tmp.nonfinite;
     return SYMNMF_OK;
@@ -535,6 +535,10 @@ static int run_full(FitCtx& c, int max_evals, HostState* hs) {
             SYMNMF_TRY(read_state(c.L.st, hs, c.s));
             SYMNMF_TRY(c.tm.harvest());
             if (hs->done) break;
+            if (launched + 1 >= max_evals + 2 * check) {   // the device should have stopped by now
+                set_error("the full-batch loop did not stop after %d passes", launched + 1);
+                return SYMNMF_ERR_CUDA;
+            }
             // after the first (eager) pass, replay graphs while enough passes remain
             if (!graphed && use_graphs() && max_evals - hs->t > G) {
                 bool used = false;

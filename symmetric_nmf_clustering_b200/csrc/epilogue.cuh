@@ -41,6 +41,41 @@ struct EpiArgs {
     int64_t ldxt;
 };
 
+// The evaluation's scalar step (one thread): f_t = ||S||^2 - 2 tr + ||A||^2,
+// history, relative change, stopping test ([CaS] "Factorizing with SymNMF";
+// the trace identity of "Factorization at scale").
+__device__ __forceinline__ void finalize_scalar(int mode, FitState* st, double tr, double rel_tol,
+                                                int max_evals, double* history, int history_cap) {
+    const bool eval = mode == MODE_FULL || mode == MODE_SNAPSHOT;
+    const int t = st->t;
+    bool stop = false;
+    if (eval) {
+        const double L = st->s_sqnorm - 2.0 * tr + st->a_sqnorm;
+        if (t < history_cap && history != nullptr) history[t] = L;
+        if (!isfinite(L)) {
+            st->nonfinite = 1;
+            stop = true;
+        }
+        if (t > 0) {
+            const double Lp = st->loss;
+            double rel;
+            if (Lp != 0.0) rel = fabs(L - Lp) / fabs(Lp);
+            else rel = (L == Lp) ? 0.0 : INFINITY;
+            st->rel = rel;
+            if (rel_tol > 0.0 && rel < rel_tol) {
+                st->converged = 1;
+                stop = true;
+            }
+        }
+        st->loss_prev = st->loss;
+        st->loss = L;
+        st->t_stop = t;
+        if (t >= max_evals - 1) stop = true;
+        st->t = t + 1;
+    }
+    if (stop) st->done = 1;
+}
+
 // Barrier over the 128 threads that run one tile's epilogue.
 template <bool FUSED>
 __device__ __forceinline__ void ep_sync() {
@@ -475,3 +510,4 @@ __device__ void epilogue_tile_cta(const EpiArgs& a, int tile, int tid, float* sm
 }
 
 }  // namespace symnmf
+

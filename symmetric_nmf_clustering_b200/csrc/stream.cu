@@ -244,7 +244,6 @@ reduce_finalize_kernel(int mode, int nblk, int k, const double* __restrict__ tr_
     const int kk = k * k;
     const int w = threadIdx.x >> 5, l = threadIdx.x & 31;
     const bool gram = mode != MODE_SNAPSHOT;
-    const bool eval = mode == MODE_FULL || mode == MODE_SNAPSHOT;
     const int gram_blocks = gram ? (kk + 31) / 32 : 0;
 
     if ((int)blockIdx.x < gram_blocks) {
@@ -291,33 +290,7 @@ reduce_finalize_kernel(int mode, int nblk, int k, const double* __restrict__ tr_
     __threadfence();
 
     if (threadIdx.x == 0) {
-        const int t = st->t;
-        bool stop = false;
-        if (eval) {
-            const double L = st->s_sqnorm - 2.0 * __ldcg(&fs->tr) + st->a_sqnorm;
-            if (t < history_cap && history != nullptr) history[t] = L;
-            if (!isfinite(L)) {
-                st->nonfinite = 1;
-                stop = true;
-            }
-            if (t > 0) {
-                const double Lp = st->loss;
-                double rel;
-                if (Lp != 0.0) rel = fabs(L - Lp) / fabs(Lp);
-                else rel = (L == Lp) ? 0.0 : INFINITY;
-                st->rel = rel;
-                if (rel_tol > 0.0 && rel < rel_tol) {
-                    st->converged = 1;
-                    stop = true;
-                }
-            }
-            st->loss_prev = st->loss;
-            st->loss = L;
-            st->t_stop = t;
-            if (t >= max_evals - 1) stop = true;
-            st->t = t + 1;
-        }
-        if (stop) st->done = 1;
+        finalize_scalar(mode, st, __ldcg(&fs->tr), rel_tol, max_evals, history, history_cap);
         fs->arrived = 0u;
     }
     __syncthreads();
