@@ -1,6 +1,7 @@
-// The per-tile epilogue of an S-stream pass, shared by the standalone
-// epilogue kernel and the tensor-core stream kernel (where the last split CTA
-// of each 128-row tile runs it in place).
+// The per-tile epilogue of an S-stream pass, in two forms: epilogue_tile (128
+// threads, the standalone epilogue kernel of the CUDA-core path and of the
+// passes without a stream) and epilogue_tile_cta (all 256 threads of the last
+// split CTA of each 128-row tile in the tensor-core stream kernel).
 //
 // For the rows i of one tile, with P_i = sum over splits of the partial rows
 // (fixed split order), by mode:
@@ -76,34 +77,28 @@ __device__ __forceinline__ void finalize_scalar(int mode, FitState* st, double t
     if (stop) st->done = 1;
 }
 
-// Barrier over the 128 threads that run one tile's epilogue.
-template <bool FUSED>
-__device__ __forceinline__ void ep_sync() {
-    if (FUSED) asm volatile("bar.sync 1, 128;" ::: "memory");
-    else __syncthreads();
-}
+
 
 // Fixed-shape sum over the 128 threads (warp shuffles, then warp 0); the
 // result is valid in tid 0.
-template <bool FUSED>
 __device__ __forceinline__ double ep_sum(double v, int tid, double* red) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) v += __shfl_down_sync(0xffffffffu, v, o);
     const int w = tid >> 5, l = tid & 31;
     if (l == 0) red[w] = v;
-    ep_sync<FUSED>();
+    __syncthreads();
     double r = 0.0;
     if (w == 0) {
         r = l < EP_ROWS / 32 ? red[l] : 0.0;
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) r += __shfl_down_sync(0xffffffffu, r, o);
     }
-    ep_sync<FUSED>();
+    __syncthreads();
     return r;
 }
 
 // smem: at least max(KE*KE, EP_ROWS*(KE+1)) floats; red: EP_ROWS/32 doubles.
-template <int KE, bool FUSED>
+template <int KE>
 __device__ void epilogue_tile(const EpiArgs& a, int tile, int tid, float* smem, double* red) {
     const int mode = a.mode;
     const int64_t n = a.n;
@@ -117,7 +112,7 @@ __device__ void epilogue_tile(const EpiArgs& a, int tile, int tid, float* smem, 
 
     if (step) {
         for (int e = tid; e < k * k; e += EP_ROWS) As[(e / k) * KE + (e % k)] = a.st->A32[e];
-        ep_sync<FUSED>();
+        __syncthreads();
     }
 
     float p[KE], h[KE];
@@ -167,7 +162,7 @@ __device__ void epilogue_tile(const EpiArgs& a, int tile, int tid, float* smem, 
         double tr = 0.0;
 #pragma unroll
         for (int c = 0; c < KE; ++c) tr += (double)h[c] * (double)p[c];
-        const double tot = ep_sum<FUSED>(tr, tid, red);
+        const double tot = ep_sum(tr, tid, red);
         if (tid == 0) a.tr_part[tile] = tot;
     }
     if (mode == MODE_SNAPSHOT) return;
@@ -210,10 +205,10 @@ __device__ void epilogue_tile(const EpiArgs& a, int tile, int tid, float* smem, 
     }
 
     // Gram partial of the rows now in h (new iterate, or the given H for GRAM)
-    ep_sync<FUSED>();  // every thread is done reading As
+    __syncthreads();  // every thread is done reading As
 #pragma unroll
     for (int c = 0; c < KE; ++c) hs[tid][c] = valid ? h[c] : 0.f;
-    ep_sync<FUSED>();
+    __syncthreads();
     const int rows = (int)min64(EP_ROWS, n - (int64_t)tile * EP_ROWS);
     double* gp = a.gram_part + (int64_t)tile * k * k;
     for (int e = tid; e < k * k; e += EP_ROWS) {

@@ -177,7 +177,7 @@ __global__ void __launch_bounds__(EP_ROWS) epilogue_kernel(const EpiArgs a) {
     constexpr int SM_FLOATS = KE * KE > EP_ROWS * (KE + 1) ? KE * KE : EP_ROWS * (KE + 1);
     __shared__ float smem[SM_FLOATS];
     __shared__ double red[EP_ROWS / 32];
-    epilogue_tile<KE, false>(a, blockIdx.x, threadIdx.x, smem, red);
+    epilogue_tile<KE>(a, blockIdx.x, threadIdx.x, smem, red);
 }
 
 int launch_epilogue(int mode, int64_t n, int k, const float* part, int splits,
