@@ -312,6 +312,14 @@ def row_rooflines(rows, n, k, T, hbm_peak):
     return out, tf32
 
 
+def bench_config(workload, world):
+    """The workload description both arms print."""
+    spec = synth.WORKLOADS[workload]
+    return {"workload": workload, "n": spec["n"], "k": spec["k"], "T": spec["T"], "solver": "adagrad",
+            "lr": 0.1, "eps": 1e-10, "l2": "inputs larger than L2 (S is 4n^2 bytes)",
+            "parallelism": f"independent windows x{world}" if world > 1 else "single"}
+
+
 # ----------------------------------------------------------------------------- reference arm
 def run_reference(args):
     world, rank, _ = dist_env()
@@ -324,7 +332,7 @@ def run_reference(args):
         "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": 1000.0 / res["value"], "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": args.workload, "n": spec["n"], "k": spec["k"], "T": spec["T"]},
+        "config": bench_config(args.workload, args.gpus),
         "impl": "reference",
         "cpu_baseline": {k2: res[k2] for k2 in ("value", "unit", "cores", "kind", "sample")},
         "e2e": {"value": res["value"], "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -472,9 +480,7 @@ def run_ours(args):
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
             "warmup": W, "ms_per_step": t_max / K, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-            "config": {"workload": args.workload, "n": n, "k": k, "T": T, "solver": "adagrad",
-                       "lr": 0.1, "eps": 1e-10, "l2": "inputs larger than L2 (S is 4n^2 bytes)",
-                       "parallelism": f"independent windows x{world}" if world > 1 else "single"},
+            "config": bench_config(args.workload, world),
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak, "traffic": None,
                          "kernel": "stream_tc_kernel", "peak_source": peak_src,
