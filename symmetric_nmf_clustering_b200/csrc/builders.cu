@@ -381,6 +381,98 @@ rank_sort_kernel(const float* __restrict__ R, int64_t T, int64_t n, int64_t ldr,
     }
 }
 
+// The same ranks with the sort held in registers: one warp per column and
+// RPL = P / 32 keys per lane, P = 2^m >= max(T, 32) <= 1024.  A key packs the
+// day under an order-preserving image of the value (the float's bits, with
+// -0 folded onto +0 so that the two stay a tie), so one unsigned 64-bit
+// comparison orders by (x_t, t).  Key slot e = lane * RPL + r: bitonic steps
+// of span < RPL swap registers inside a lane, wider ones trade with the lane
+// at distance span / RPL by shuffle.  The keys enter in any order (each
+// carries its day), so the load reads day r * 32 + lane from a day-major tile
+// of the block's columns without bank conflicts; positions leave through
+// the same tile.  Padding keys are all ones and sort last.
+constexpr int RW_COLS = 8;                  // columns per block, one per warp
+constexpr int RW_THREADS = 32 * RW_COLS;
+constexpr int RW_LD = RW_COLS + 1;          // tile row stride (odd: no bank conflicts)
+constexpr int64_t RW_MAX_P = 1024;
+
+__device__ __forceinline__ uint64_t rw_key(float x, int t) {
+    uint32_t u = __float_as_uint(x);
+    if ((u & 0x7fffffffu) == 0u) u = 0u;                   // -0 -> +0
+    u = (u & 0x80000000u) ? ~u : (u | 0x80000000u);        // monotone in x
+    return ((uint64_t)u << 32) | (uint32_t)t;
+}
+
+template <int RPL>
+__device__ __forceinline__ void rw_bitonic(uint64_t (&key)[RPL], int lane) {
+#pragma unroll
+    for (int k = 2; k <= 32 * RPL; k <<= 1) {
+#pragma unroll
+        for (int j = k >> 1; j > 0; j >>= 1) {
+            if (j >= RPL) {
+                // partner slot e ^ j lives in lane ^ (j / RPL), same register
+                const int lm = j / RPL;
+                const bool up = ((lane * RPL) & k) == 0;
+                const bool keep_min = ((lane & lm) == 0) == up;
+#pragma unroll
+                for (int r = 0; r < RPL; ++r) {
+                    const uint64_t o = __shfl_xor_sync(0xffffffffu, key[r], lm);
+                    key[r] = ((o < key[r]) == keep_min) ? o : key[r];
+                }
+            } else {
+#pragma unroll
+                for (int r = 0; r < RPL; ++r) {
+                    if (r & j) continue;
+                    const bool up = ((lane * RPL + r) & k) == 0;
+                    const uint64_t a = key[r], b = key[r + j];
+                    const bool sw = (b < a) == up;
+                    key[r] = sw ? b : a;
+                    key[r + j] = sw ? a : b;
+                }
+            }
+        }
+    }
+}
+
+template <int RPL>
+__global__ void __launch_bounds__(RW_THREADS)
+rank_warp_kernel(const float* __restrict__ R, int64_t T, int64_t n, int64_t ldr, float sign,
+                 int32_t* __restrict__ ranks) {
+    __shared__ uint32_t tile[RW_MAX_P * RW_LD];             // [day][column]
+    const int tid = threadIdx.x, lane = tid & 31, c = tid >> 5;
+    const int64_t i0 = (int64_t)blockIdx.x * RW_COLS;
+    const int cols = (int)min64(RW_COLS, n - i0);
+    const int Ti = (int)T;
+
+    for (int e = tid; e < Ti * RW_COLS; e += RW_THREADS) {
+        const int t = e / RW_COLS, cc = e % RW_COLS;
+        const float x = cc < cols ? sign * R[(int64_t)t * ldr + i0 + cc] : 0.f;
+        tile[t * RW_LD + cc] = __float_as_uint(x);
+    }
+    __syncthreads();
+
+    uint64_t key[RPL];
+#pragma unroll
+    for (int r = 0; r < RPL; ++r) {
+        const int t = r * 32 + lane;
+        key[r] = t < Ti ? rw_key(__uint_as_float(tile[t * RW_LD + c]), t) : ~0ull;
+    }
+    __syncthreads();                                        // the tile now takes ranks
+
+    rw_bitonic<RPL>(key, lane);
+
+#pragma unroll
+    for (int r = 0; r < RPL; ++r) {
+        const uint32_t t = (uint32_t)key[r];                // padding: 0xffffffff
+        if (t < (uint32_t)Ti) tile[t * RW_LD + c] = (uint32_t)(lane * RPL + r + 1);
+    }
+    __syncthreads();
+    for (int e = tid; e < Ti * RW_COLS; e += RW_THREADS) {
+        const int t = e / RW_COLS, cc = e % RW_COLS;
+        if (cc < cols) ranks[(int64_t)t * n + i0 + cc] = (int32_t)tile[t * RW_LD + cc];
+    }
+}
+
 // phi[r] = (-ln(r / (T+1)))^(-1/2): Frechet (alpha = 2) margin of rank r, fp64.
 __global__ void phi_kernel(double* __restrict__ phi, int64_t T) {
     const int64_t r = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
@@ -468,7 +560,17 @@ int launch_tpdm(const float* R, int64_t T, int64_t n, int64_t ldr, int N,
     const float sign = tail_sign < 0 ? -1.f : 1.f;
     int P = 2;
     while (P < T) P <<= 1;
-    if (P <= RS_MAX_P) {
+    if (P <= RW_MAX_P) {
+        const unsigned wblocks = (unsigned)((n + RW_COLS - 1) / RW_COLS);
+        switch (P <= 32 ? 1 : P / 32) {
+            case 1: rank_warp_kernel<1><<<wblocks, RW_THREADS, 0, s>>>(R, T, n, ldr, sign, ranks); break;
+            case 2: rank_warp_kernel<2><<<wblocks, RW_THREADS, 0, s>>>(R, T, n, ldr, sign, ranks); break;
+            case 4: rank_warp_kernel<4><<<wblocks, RW_THREADS, 0, s>>>(R, T, n, ldr, sign, ranks); break;
+            case 8: rank_warp_kernel<8><<<wblocks, RW_THREADS, 0, s>>>(R, T, n, ldr, sign, ranks); break;
+            case 16: rank_warp_kernel<16><<<wblocks, RW_THREADS, 0, s>>>(R, T, n, ldr, sign, ranks); break;
+            default: rank_warp_kernel<32><<<wblocks, RW_THREADS, 0, s>>>(R, T, n, ldr, sign, ranks); break;
+        }
+    } else if (P <= RS_MAX_P) {
         const size_t rs_smem = (size_t)RS_COLS * P * 8 + (size_t)T * RS_COLS * 4;
         static bool rs_attr = false;   // once per process
         if (!rs_attr) {

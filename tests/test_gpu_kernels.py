@@ -85,10 +85,13 @@ def test_corr_builder_zero_variance_column(m):
     assert S[5, 5] == 1.0 and np.all(S[5, np.arange(64) != 5] == 0.0)
 
 
-# T <= 2048 ranks by sorting (2048 is the largest sort); T = 2100 takes the
-# counting kernel
+# T <= 1024 ranks by a sort held in registers (32 keys per lane at most;
+# T = 20, 33, 400, 1024 fill 1, 2, 16, 32 keys per lane), T <= 2048 by a sort
+# in shared memory, larger T by the counting kernel
 @pytest.mark.parametrize("T,n,frac,sign", [(250, 2000, 0.05, 1), (1000, 1999, 0.05, 1),
                                            (100, 130, 0.1, -1), (20, 2, 0.1, 1), (1, 5, 1.0, 1),
+                                           (33, 500, 0.1, -1), (400, 333, 0.05, 1),
+                                           (1024, 300, 0.05, -1), (1025, 70, 0.05, 1),
                                            (2048, 45, 0.05, -1), (2100, 37, 0.05, 1),
                                            (80, 4100, 0.1, 1)])
 def test_tpdm_builder(m, T, n, frac, sign):
@@ -99,11 +102,15 @@ def test_tpdm_builder(m, T, n, frac, sign):
     assert abs(np.trace(S.astype(np.float64)) - n) <= 1e-5 * n
 
 
-def test_tpdm_builder_with_ties(m):
-    rng = np.random.default_rng(3)
-    R = rng.integers(-3, 4, size=(64, 40)).astype(np.float32)
-    S = m.build_tpdm(to_dev(R, DEV), 0.125, 1).cpu().numpy()
-    ref = oracle.tpdm(R, 0.125, 1)
+@pytest.mark.parametrize("T,n,sign", [(64, 40, 1), (64, 40, -1), (1000, 24, -1), (1500, 16, 1)])
+def test_tpdm_builder_with_ties(m, T, n, sign):
+    # integer returns: long runs of equal values, ranked towards the earlier
+    # day; a third of the zeros are -0.0, which ties with +0.0
+    rng = np.random.default_rng(T + n)
+    R = rng.integers(-3, 4, size=(T, n)).astype(np.float32)
+    R[(R == 0) & (rng.random((T, n)) < 0.33)] = -0.0
+    S = m.build_tpdm(to_dev(R, DEV), 0.125, sign).cpu().numpy()
+    ref = oracle.tpdm(R, 0.125, sign)
     assert np.max(np.abs(S - ref)) <= 1e-5 * np.max(np.abs(ref))
 
 
