@@ -53,24 +53,36 @@ stats_partial_kernel(const float* __restrict__ S, int64_t n, int64_t lds,
 #pragma unroll
             for (int u = 0; u < U; ++u) {
                 const float e[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+                // all four normal (false for zero, subnormal, inf and NaN)
+                bool normal = true;
 #pragma unroll
-                for (int w = 0; w < 4; ++w) {
-                    // widen to fp64 by moving the bit fields (exact for normal
-                    // floats): the conversion instruction's throughput, not
-                    // HBM, limited this pass
-                    const uint32_t b = __float_as_uint(e[w]);
-                    const uint32_t ex = (b >> 23) & 0xFFu;
-                    if (ex - 1u < 254u) {
-                        const uint32_t hi = (b & 0x80000000u) | ((ex + 896u) << 20) | ((b >> 3) & 0x000FFFFFu);
+                for (int w = 0; w < 4; ++w)
+                    normal &= (fabsf(e[w]) >= 0x1p-126f) & (fabsf(e[w]) <= 0x1.fffffep127f);
+                if (normal) {
+                    // widen to fp64 by moving the bit fields, exact for normal
+                    // floats: the arithmetic shift puts the sign in bits 31..28
+                    // and the exponent in 27..20, the mask clears bits 30..28
+                    // and the add rebiases the exponent by 1023 - 127 = 896
+                    // (no carry reaches bit 31); the conversion instruction's
+                    // throughput, not HBM, limited this pass
+#pragma unroll
+                    for (int w = 0; w < 4; ++w) {
+                        const uint32_t b = __float_as_uint(e[w]);
+                        const uint32_t hi = ((uint32_t)((int32_t)b >> 3) & 0x8FFFFFFFu) + 0x38000000u;
                         const double d = __hiloint2double((int)hi, (int)(b << 29));
                         sum += d;
                         sq = fma(d, d, sq);
-                    } else if (ex == 0xFFu) {
-                        bad += 1.0;
-                    } else {   // zero or subnormal
-                        const double d = e[w];
-                        sum += d;
-                        sq = fma(d, d, sq);
+                    }
+                } else {
+#pragma unroll
+                    for (int w = 0; w < 4; ++w) {
+                        if (isfinite(e[w])) {
+                            const double d = e[w];
+                            sum += d;
+                            sq = fma(d, d, sq);
+                        } else {
+                            bad += 1.0;
+                        }
                     }
                 }
             }
