@@ -7,6 +7,7 @@
 #include <algorithm>
 #include <cstdio>
 #include <string>
+#include <utility>
 
 #include "symnmf.h"
 
@@ -202,5 +203,32 @@ int launch_gemm_nn_sub(float* W, int64_t n, int64_t ldw, int cw, const float* V,
                        int64_t ldv, int cv, const float* C, cudaStream_t s);
 int launch_trsm_right(float* W, int64_t n, int64_t ldw, int cw, const float* Rinv,
                       cudaStream_t s);
+
+// Programmatic dependent launch.  A kernel launched with programmatic stream
+// serialization may start before the previous kernel in its stream has
+// finished; it calls pdl_wait() before it reads anything that kernel wrote
+// (a no-op when it was launched the ordinary way).  pdl_trigger() lets the
+// next such kernel be scheduled once every CTA of this grid has triggered or
+// exited.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+// Launches kern<<<grid, block, smem, s>>>(args...) with programmatic stream
+// serialization.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                       Args&&... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
 
 }  // namespace symnmf

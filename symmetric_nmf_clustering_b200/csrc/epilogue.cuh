@@ -22,6 +22,16 @@ namespace symnmf {
 
 constexpr int EP_ROWS = 128;
 
+// 16-byte global -> shared copy that bypasses L1 (the data were written by
+// other CTAs of the same kernel), and the wait for all of this thread's copies
+__device__ __forceinline__ void cp_async_cg16(float* dst_smem, const float* src) {
+    const uint32_t d = (uint32_t)__cvta_generic_to_shared(dst_smem);
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+    asm volatile("cp.async.wait_all;" ::: "memory");
+}
+
 struct EpiArgs {
     int mode;
     int64_t n;
@@ -245,9 +255,10 @@ constexpr size_t epilogue_cta_floats() {
 // the same four-chain fp64 sum (products of fp32 values are exact in fp64, so
 // entry (c, d) equals entry (d, c) and is computed once).  The trace partial
 // is summed in a different, fixed order.
-// smem: epilogue_cta_floats<KE>() floats.  Callers: every thread of the CTA.
+// smem: stage_floats >= epilogue_cta_floats<KE>() floats, 16-byte aligned.
+// Callers: every thread of the CTA.
 template <int KE>
-__device__ void epilogue_tile_cta(const EpiArgs& a, int tile, int tid, float* smem) {
+__device__ void epilogue_tile_cta(const EpiArgs& a, int tile, int tid, float* smem, int stage_floats) {
     constexpr int NT = 256;
     static_assert(EP_ROWS * KE % NT == 0, "whole elements per thread");
     const int mode = a.mode;
@@ -293,7 +304,33 @@ __device__ void epilogue_tile_cta(const EpiArgs& a, int tile, int tid, float* sm
     float acc[EPT];
 #pragma unroll
     for (int q = 0; q < EPT; ++q) acc[q] = 0.f;
-    if (mode != MODE_GRAM && mode != MODE_STEP_SNAP) {
+    // the partial tiles are contiguous runs of 16-byte pieces when n k and the
+    // tile's element count are multiples of 4: they then go to shared memory
+    // (all of it is free until P, H, G and A are stored below) with cp.async,
+    // as many tiles per batch as fit, one L2 round trip per batch
+    constexpr int TS = EP_ROWS * KE;
+    const int nbt = stage_floats / TS;
+    const bool staged = nbt >= 1 && (n * k) % 4 == 0 && tot % 4 == 0;
+    if (staged && mode != MODE_GRAM && mode != MODE_STEP_SNAP) {
+        for (int s0 = 0; s0 < a.splits; s0 += nbt) {
+            const int sb = min(nbt, a.splits - s0);
+            for (int t = 0; t < sb; ++t) {
+                const float* src = a.part + (int64_t)(s0 + t) * n * k + base;
+                for (int e4 = tid; e4 < tot / 4; e4 += NT)
+                    cp_async_cg16(smem + t * TS + 4 * e4, src + 4 * e4);
+            }
+            cp_async_wait_all();
+            __syncthreads();
+            for (int t = 0; t < sb; ++t) {
+#pragma unroll
+                for (int q = 0; q < EPT; ++q) {
+                    const int e = tid + q * NT;
+                    if (e < tot) acc[q] += smem[t * TS + e];
+                }
+            }
+            __syncthreads();   // read before the next batch (or P, H, G) overwrites
+        }
+    } else if (mode != MODE_GRAM && mode != MODE_STEP_SNAP) {
         int s = 0;
         if constexpr (EPT <= 16) {
             for (; s + 1 < a.splits; s += 2) {
@@ -372,27 +409,83 @@ __device__ void epilogue_tile_cta(const EpiArgs& a, int tile, int tid, float* sm
 
     // ---- projected AdaGrad step: two threads per row, KE/2 columns each
     if (step) {
-        constexpr int HALF = KE / 2;
+        constexpr int HALF = KE / 2;   // a multiple of 4
         const int r = tid >> 1, c0 = (tid & 1) * HALF;
-        float h[KE], hn[HALF], gn[HALF];
+        float hn[HALF], gn[HALF];
         const bool valid = r < rows;
+        if ((k & 3) == 0) {
+            // rows of H, P, G and of A read as 16-byte pieces (r k, c0 and KE
+            // are multiples of 4), H A accumulated in the same d order
+            float h[KE], ha[HALF];
 #pragma unroll
-        for (int d = 0; d < KE; ++d) h[d] = (valid && d < k) ? T1[r * k + d] : 0.f;
+            for (int m = 0; m < KE / 4; ++m) {
+                float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (valid && 4 * m < k) x = *reinterpret_cast<const float4*>(T1 + r * k + 4 * m);
+                h[4 * m] = x.x;
+                h[4 * m + 1] = x.y;
+                h[4 * m + 2] = x.z;
+                h[4 * m + 3] = x.w;
+            }
 #pragma unroll
-        for (int j = 0; j < HALF; ++j) {
-            const int c = c0 + j;
-            hn[j] = 0.f;
-            gn[j] = 0.f;
-            if (valid && c < k) {
-                float ha = 0.f;
+            for (int j = 0; j < HALF; ++j) ha[j] = 0.f;
 #pragma unroll
-                for (int d = 0; d < KE; ++d)
-                    if (d < k) ha = fmaf(h[d], As[d * KE + c], ha);
-                const float g = 4.f * (ha - P[r * k + c]);
-                const float gg = fmaf(g, g, T2[r * k + c]);
-                const float stepv = __fdiv_rn(a.lr * g, __fadd_rn(__fsqrt_rn(gg), a.eps));
-                hn[j] = fmaxf(T1[r * k + c] - stepv, 0.f);   // = h[c]
-                gn[j] = gg;
+            for (int d = 0; d < KE; ++d) {
+                if (d < k) {
+#pragma unroll
+                    for (int m = 0; m < HALF / 4; ++m) {
+                        const float4 a4 = *reinterpret_cast<const float4*>(As + d * KE + c0 + 4 * m);
+                        ha[4 * m] = fmaf(h[d], a4.x, ha[4 * m]);
+                        ha[4 * m + 1] = fmaf(h[d], a4.y, ha[4 * m + 1]);
+                        ha[4 * m + 2] = fmaf(h[d], a4.z, ha[4 * m + 2]);
+                        ha[4 * m + 3] = fmaf(h[d], a4.w, ha[4 * m + 3]);
+                    }
+                }
+            }
+#pragma unroll
+            for (int m = 0; m < HALF / 4; ++m) {
+                float4 p4 = make_float4(0.f, 0.f, 0.f, 0.f), g4 = p4, h4 = p4;
+                if (valid && c0 + 4 * m < k) {
+                    p4 = *reinterpret_cast<const float4*>(P + r * k + c0 + 4 * m);
+                    g4 = *reinterpret_cast<const float4*>(T2 + r * k + c0 + 4 * m);
+                    h4 = *reinterpret_cast<const float4*>(T1 + r * k + c0 + 4 * m);
+                }
+                const float pv[4] = {p4.x, p4.y, p4.z, p4.w};
+                const float gv4[4] = {g4.x, g4.y, g4.z, g4.w};
+                const float hv4[4] = {h4.x, h4.y, h4.z, h4.w};
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int j = 4 * m + u;
+                    hn[j] = 0.f;
+                    gn[j] = 0.f;
+                    if (valid && c0 + j < k) {
+                        const float g = 4.f * (ha[j] - pv[u]);
+                        const float gg = fmaf(g, g, gv4[u]);
+                        const float stepv = __fdiv_rn(a.lr * g, __fadd_rn(__fsqrt_rn(gg), a.eps));
+                        hn[j] = fmaxf(hv4[u] - stepv, 0.f);
+                        gn[j] = gg;
+                    }
+                }
+            }
+        } else {
+            float h[KE];
+#pragma unroll
+            for (int d = 0; d < KE; ++d) h[d] = (valid && d < k) ? T1[r * k + d] : 0.f;
+#pragma unroll
+            for (int j = 0; j < HALF; ++j) {
+                const int c = c0 + j;
+                hn[j] = 0.f;
+                gn[j] = 0.f;
+                if (valid && c < k) {
+                    float ha = 0.f;
+#pragma unroll
+                    for (int d = 0; d < KE; ++d)
+                        if (d < k) ha = fmaf(h[d], As[d * KE + c], ha);
+                    const float g = 4.f * (ha - P[r * k + c]);
+                    const float gg = fmaf(g, g, T2[r * k + c]);
+                    const float stepv = __fdiv_rn(a.lr * g, __fadd_rn(__fsqrt_rn(gg), a.eps));
+                    hn[j] = fmaxf(T1[r * k + c] - stepv, 0.f);   // = h[c]
+                    gn[j] = gg;
+                }
             }
         }
         __syncthreads();   // every thread holds its row of H: T1, T2 may be overwritten

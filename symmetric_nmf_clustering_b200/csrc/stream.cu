@@ -234,6 +234,8 @@ reduce_finalize_kernel(int mode, int nblk, int k, const double* __restrict__ tr_
                        const double* __restrict__ gram_part, FitState* st,
                        FinalScratch* fs, double rel_tol, int max_evals,
                        double* history, int history_cap) {
+    pdl_wait();
+    pdl_trigger();   // the next pass's CTAs may start their setup meanwhile
     if (st->done) return;
     if (st->kerr != 0) {   // the S-stream gave up waiting: stop the loop, no result this pass
         if (blockIdx.x == 0 && threadIdx.x == 0) st->done = 1;
@@ -324,8 +326,9 @@ int launch_finalize(int mode, int nblk, int k, const double* tr_part,
     const int kk = k * k;
     const int gram_blocks = mode != MODE_SNAPSHOT ? (kk + 31) / 32 : 0;
     const int grid = gram_blocks + 1;
-    reduce_finalize_kernel<<<grid, RF_THREADS, 0, s>>>(mode, nblk, k, tr_part, gram_part, st, fs,
-                                                      rel_tol, max_evals, history, history_cap);
+    SYMNMF_CUDA_TRY(launch_pdl(reduce_finalize_kernel, dim3(grid), dim3(RF_THREADS), 0, s, mode, nblk, k,
+                               tr_part, gram_part, st, fs, rel_tol, max_evals, history,
+                               history_cap));
     SYMNMF_LAUNCH_CHECK();
     return SYMNMF_OK;
 }

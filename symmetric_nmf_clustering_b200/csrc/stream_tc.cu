@@ -128,6 +128,7 @@ stream_tc_kernel(const __grid_constant__ CUtensorMap mapS, const __grid_constant
                  const EpiArgs epi, int* __restrict__ counters) {
     using Cfg = TcCfg<KP>;
     using namespace sm100;
+    pdl_wait();   // everything below may read what the previous kernel wrote
     if (st != nullptr && st->done) return;
 
     extern __shared__ uint8_t tc_smem_raw[];
@@ -374,8 +375,12 @@ stream_tc_kernel(const __grid_constant__ CUtensorMap mapS, const __grid_constant
     // every stage has landed and been consumed: the pipeline's shared memory is
     // free, and all eight warps run the tile's epilogue
     if (last_sh) {
+        // this CTA holds no TMEM any more and the CTAs without an epilogue
+        // have exited: the next kernel may be scheduled
+        pdl_trigger();
         __threadfence();
-        epilogue_tile_cta<KP>(epi, (int)blockIdx.x, tid, reinterpret_cast<float*>(smem));
+        epilogue_tile_cta<KP>(epi, (int)blockIdx.x, tid, reinterpret_cast<float*>(smem),
+                              (int)((Cfg::SMEM - 1024) / sizeof(float)));
         if (tid == 0) counters[blockIdx.x] = 0;   // ready for the next pass
     }
 }
@@ -505,8 +510,8 @@ int launch_stream_tc(const TcPlan& p, const float* S, int64_t lds, const float* 
                                                  (int)TcCfg<KP>::SMEM));                      \
             attr_set = true;                                                                  \
         }                                                                                     \
-        kern<<<grid, TC_THREADS, TcCfg<KP>::SMEM, s>>>(mapS, mapX, p.n, p.k, p.j0, p.j1,      \
-                                                       p.jspan, part, err, st, ea, cnt);      \
+        SYMNMF_CUDA_TRY(launch_pdl(kern, grid, dim3(TC_THREADS), TcCfg<KP>::SMEM, s, mapS, mapX, \
+                                   p.n, p.k, p.j0, p.j1, p.jspan, part, err, st, ea, cnt));   \
     } while (0)
     switch (p.KP) {
         case 8: SYMNMF_TC(8); break;
