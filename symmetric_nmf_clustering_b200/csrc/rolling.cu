@@ -6,11 +6,17 @@
 // and the window delta earlier; a 3-sigma control limit on the latter.
 //
 // The driver composes the library's own entry points (builders, fit, labels,
-// S-stream product) on one stream; this file adds the contingency-table
-// kernel behind the ARI and the monitor's reduction kernels.
+// S-stream product); with both kinds selected it runs the |corr| chain on the
+// caller's stream and the TPDM chain on a second stream from a second host
+// thread, each window's passes being latency-bound at this size.  This file
+// adds the contingency-table kernel behind the ARI and the monitor's
+// reduction kernels.
 #include <cmath>
 #include <cstring>
+#include <cstdlib>
 #include <limits>
+#include <string>
+#include <thread>
 #include <vector>
 
 #include "common.cuh"
@@ -193,16 +199,24 @@ __global__ void cross_final_kernel(const double* __restrict__ part, int nblk,
 
 // ---------------------------------------------------------------- workspace
 
-struct RollingLayout {
+// One chain's buffers: a chain is one dependence matrix over every window
+// (build, monitor, fit, labels, ARI on its own stream).
+struct ChainLayout {
     void* shared = nullptr;      // builders, fit and the monitor's product take turns here
     size_t shared_bytes = 0;
     float* H = nullptr;
     AriLayout ari;
-    float* Z = nullptr;          // n x 8 indicator of the stressed groups
     float* Y = nullptr;          // n x 8 product S Z
-    int* counts = nullptr;
     double* part = nullptr;
     double* cross = nullptr;     // the current window's monitor value
+};
+
+struct RollingLayout {
+    ChainLayout chain[2];        // chain[1] only when the two kinds run concurrently
+    float* S2 = nullptr;         // the second chain's n x n matrix, row stride lds2
+    int64_t lds2 = 0;
+    float* Z = nullptr;          // n x 8 indicator of the stressed groups (read-only)
+    int* counts = nullptr;
 };
 
 static int cross_blocks(const Dev& d) { return 2 * d.sms; }
@@ -211,22 +225,34 @@ static int sub_ws(int op, int64_t n, int k, int64_t T, const symnmf_fit_params* 
     return symnmf_workspace_size(op, n, k, T, P, b);
 }
 
+static void chain_plan(const Dev& d, Arena& a, int64_t n, int k, size_t shared_bytes,
+                       ChainLayout* C) {
+    C->shared_bytes = shared_bytes;
+    C->shared = a.take<char>(shared_bytes);
+    C->H = a.take<float>((size_t)n * k);
+    ari_plan(a, &C->ari);
+    C->Y = a.take<float>((size_t)n * RL_MAX_STRESSED);
+    C->part = a.take<double>((size_t)cross_blocks(d));
+    C->cross = a.take<double>(64);
+}
+
+// concurrent: room for both chains and the second n x n matrix
 int rolling_plan(const Dev& d, Arena& a, int64_t n, int k, int64_t T, const symnmf_fit_params& P,
-                 RollingLayout* L) {
+                 bool concurrent, RollingLayout* L) {
     size_t b_corr = 0, b_tpdm = 0, b_fit = 0, b_sh = 0;
     SYMNMF_TRY(sub_ws(SYMNMF_OP_BUILD_CORR, n, k, T, &P, &b_corr));
     SYMNMF_TRY(sub_ws(SYMNMF_OP_BUILD_TPDM, n, k, T, &P, &b_tpdm));
     SYMNMF_TRY(sub_ws(SYMNMF_OP_FIT, n, k, T, &P, &b_fit));
     SYMNMF_TRY(sub_ws(SYMNMF_OP_SH, n, RL_MAX_STRESSED, T, &P, &b_sh));
-    L->shared_bytes = std::max(std::max(b_corr, b_tpdm), std::max(b_fit, b_sh));
-    L->shared = a.take<char>(L->shared_bytes);
-    L->H = a.take<float>((size_t)n * k);
-    ari_plan(a, &L->ari);
+    const size_t shared = std::max(std::max(b_corr, b_tpdm), std::max(b_fit, b_sh));
     L->Z = a.take<float>((size_t)n * RL_MAX_STRESSED);
-    L->Y = a.take<float>((size_t)n * RL_MAX_STRESSED);
     L->counts = a.take<int>(64);
-    L->part = a.take<double>((size_t)cross_blocks(d));
-    L->cross = a.take<double>(64);
+    chain_plan(d, a, n, k, shared, &L->chain[0]);
+    if (concurrent) {
+        chain_plan(d, a, n, k, shared, &L->chain[1]);
+        L->lds2 = (n + 3) / 4 * 4;
+        L->S2 = a.take<float>((size_t)n * (size_t)L->lds2);
+    }
     return SYMNMF_OK;
 }
 
@@ -243,7 +269,7 @@ int rolling_workspace_bytes(const Dev& d, int64_t n, int k, int64_t T, const sym
     Arena a;
     a.dry = true;
     RollingLayout L;
-    SYMNMF_TRY(rolling_plan(d, a, n, k, T, P, &L));
+    SYMNMF_TRY(rolling_plan(d, a, n, k, T, P, true, &L));
     *bytes = a.used + 256;
     return SYMNMF_OK;
 }
@@ -268,6 +294,102 @@ struct EventPair {
     }
 };
 
+// What one chain needs and what it reports.
+struct ChainRun {
+    int kind = 0;                // 0 = |corr|, 1 = TPDM
+    const ChainLayout* C = nullptr;
+    float* S = nullptr;
+    int64_t lds = 0;
+    cudaStream_t s = nullptr;
+    double build_ms = 0.0, fit_ms = 0.0;
+    std::vector<double> ari_delta;
+    int launches = 0;
+    int rc = SYMNMF_OK;
+    std::string err;
+};
+
+struct StudyArgs {
+    const Dev* d;
+    const float* R;
+    int64_t n, ldr, T, W;
+    const symnmf_rolling_params* p;
+    bool monitor;
+    int G;
+    const float* Z;
+    const int* counts;
+    symnmf_rolling_out* out;
+};
+
+// Every window of one kind on r.s: build, monitor, fit, labels, the two ARIs.
+static int run_chain(const StudyArgs& A, ChainRun& r) {
+    const symnmf_rolling_params& p = *A.p;
+    const ChainLayout& L = *r.C;
+    const int64_t n = A.n;
+    const int c = r.kind;
+    const double nan = std::numeric_limits<double>::quiet_NaN();
+    r.ari_delta.assign((size_t)A.W, nan);
+    EventPair ev_build, ev_fit;
+    SYMNMF_TRY(ev_build.create());
+    SYMNMF_TRY(ev_fit.create());
+    auto count = [&]() {
+        r.launches += launches();
+        reset_launches();
+    };
+    reset_launches();
+    for (int64_t w = 0; w < A.W; ++w) {
+        const float* Rw = A.R + (size_t)(w * p.stride) * (size_t)A.ldr;
+        SYMNMF_CUDA_TRY(cudaEventRecord(ev_build.a, r.s));
+        if (c == 0)
+            SYMNMF_TRY(symnmf_build_corr(Rw, A.T, n, A.ldr, r.S, r.lds, L.shared, L.shared_bytes, r.s));
+        else
+            SYMNMF_TRY(symnmf_build_tpdm(Rw, A.T, n, A.ldr, p.tail_frac, p.tail_sign, r.S, r.lds,
+                                         L.shared, L.shared_bytes, r.s));
+        count();
+        SYMNMF_CUDA_TRY(cudaEventRecord(ev_build.b, r.s));
+        double cross = nan;
+        if (A.monitor) {
+            SYMNMF_TRY(symnmf_sh(r.S, n, r.lds, A.Z, A.G, L.Y, L.shared, L.shared_bytes, r.s));
+            cross_partial_kernel<<<cross_blocks(*A.d), RL_THREADS, 0, r.s>>>(L.Y, A.Z, n, A.G, L.part);
+            SYMNMF_LAUNCH_CHECK();
+            cross_final_kernel<<<1, RL_THREADS, 0, r.s>>>(L.part, cross_blocks(*A.d), A.counts, A.G,
+                                                          L.cross);
+            SYMNMF_LAUNCH_CHECK();
+            SYMNMF_CUDA_TRY(cudaMemcpyAsync(&cross, L.cross, sizeof(double), cudaMemcpyDeviceToHost,
+                                            r.s));
+            count();
+        }
+        SYMNMF_CUDA_TRY(cudaEventRecord(ev_fit.a, r.s));
+        symnmf_fit_stats st;
+        SYMNMF_TRY(symnmf_fit(r.S, n, r.lds, p.k, &p.fit, L.H, &st, L.shared, L.shared_bytes, r.s));
+        count();
+        int32_t* lab = A.out->labels[c] + (size_t)w * (size_t)n;
+        SYMNMF_TRY(symnmf_labels(L.H, n, p.k, lab, r.s));
+        count();
+        SYMNMF_CUDA_TRY(cudaEventRecord(ev_fit.b, r.s));
+        double prev = nan, dl = nan;
+        if (w >= 1) SYMNMF_TRY(ari_run(*A.d, L.ari, lab - n, lab, n, p.k, &prev, nullptr, r.s));
+        if (w >= p.delta)
+            SYMNMF_TRY(ari_run(*A.d, L.ari, lab - (size_t)p.delta * n, lab, n, p.k, &dl, nullptr, r.s));
+        count();
+        // the fit and the ARI synchronised the stream: both event pairs are complete
+        SYMNMF_CUDA_TRY(cudaStreamSynchronize(r.s));
+        r.build_ms += ev_build.ms();
+        r.fit_ms += ev_fit.ms();
+        r.ari_delta[(size_t)w] = dl;
+        if (A.out->ari_prev[c]) A.out->ari_prev[c][w] = prev;
+        if (A.out->ari_delta[c]) A.out->ari_delta[c][w] = dl;
+        if (A.out->cross[c]) A.out->cross[c][w] = cross;
+        if (A.out->loss[c]) A.out->loss[c][w] = st.loss;
+    }
+    return SYMNMF_OK;
+}
+
+// Two kinds side by side unless SYMNMF_ROLLING_SERIAL=1 (read at each call).
+static bool rolling_serial() {
+    const char* e = getenv("SYMNMF_ROLLING_SERIAL");
+    return e != nullptr && std::strcmp(e, "1") == 0;
+}
+
 static int rolling_impl(const float* R, int64_t days, int64_t n, int64_t ldr, const int32_t* groups,
                         float* S, int64_t lds, const symnmf_rolling_params& p,
                         symnmf_rolling_out* out, void* ws, size_t ws_bytes, cudaStream_t s) {
@@ -280,39 +402,42 @@ static int rolling_impl(const float* R, int64_t days, int64_t n, int64_t ldr, co
                   (long long)W, (long long)T, (long long)p.stride, (long long)days);
         return SYMNMF_ERR_INVALID_ARG;
     }
-    Arena a;
-    a.base = static_cast<char*>(ws);
-    a.cap = ws_bytes;
-    RollingLayout L;
-    SYMNMF_TRY(rolling_plan(d, a, n, p.k, T, p.fit, &L));
-    if (!a.ok()) {
-        set_error("workspace too small: %zu given, %zu needed", ws_bytes, a.used);
-        return SYMNMF_ERR_WORKSPACE;
-    }
     const bool kind_on[2] = {(p.kinds & SYMNMF_KIND_CORR) != 0, (p.kinds & SYMNMF_KIND_TPDM) != 0};
     for (int c = 0; c < 2; ++c)
         if (kind_on[c] && out->labels[c] == nullptr) {
             set_error("labels[%d] must be a device buffer of n_windows x n int32", c);
             return SYMNMF_ERR_INVALID_ARG;
         }
+    // the two chains run concurrently when both kinds are on and the workspace
+    // holds the second chain; otherwise one after the other
+    RollingLayout L;
+    bool concurrent = kind_on[0] && kind_on[1] && !rolling_serial();
+    {
+        Arena a;
+        a.base = static_cast<char*>(ws);
+        a.cap = ws_bytes;
+        SYMNMF_TRY(rolling_plan(d, a, n, p.k, T, p.fit, concurrent, &L));
+        if (!a.ok() && concurrent) {
+            concurrent = false;
+            L = RollingLayout();
+            a.used = 0;
+            SYMNMF_TRY(rolling_plan(d, a, n, p.k, T, p.fit, false, &L));
+        }
+        if (!a.ok()) {
+            set_error("workspace too small: %zu given, %zu needed", ws_bytes, a.used);
+            return SYMNMF_ERR_WORKSPACE;
+        }
+    }
     const bool monitor = p.n_stressed >= 2;
     const int G = p.n_stressed;
     StressedList sl{};
     sl.count = G;
     for (int g = 0; g < G; ++g) sl.g[g] = p.stressed[g];
 
-    int launches_total = 0;
-    auto count_launches = [&]() {
-        launches_total += launches();
-        reset_launches();
-    };
     reset_launches();
-    EventPair whole, ev_build, ev_fit;
+    EventPair whole;
     SYMNMF_TRY(whole.create());
-    SYMNMF_TRY(ev_build.create());
-    SYMNMF_TRY(ev_fit.create());
     SYMNMF_CUDA_TRY(cudaEventRecord(whole.a, s));
-
     if (monitor) {
         SYMNMF_CUDA_TRY(cudaMemsetAsync(L.counts, 0, sizeof(int) * RL_MAX_STRESSED, s));
         const int blocks = (int)std::max<int64_t>(
@@ -320,60 +445,80 @@ static int rolling_impl(const float* R, int64_t days, int64_t n, int64_t ldr, co
         stressed_indicator_kernel<<<blocks, RL_THREADS, 0, s>>>(groups, n, sl, L.Z, L.counts);
         SYMNMF_LAUNCH_CHECK();
     }
+    int launches_total = launches();
+    reset_launches();
+
     const double nan = std::numeric_limits<double>::quiet_NaN();
-    std::vector<double> ari_delta[2];
     for (int c = 0; c < 2; ++c) {
         out->build_ms[c] = 0.0;
         out->fit_ms[c] = 0.0;
         out->mean[c] = out->std[c] = out->limit[c] = nan;
-        ari_delta[c].assign((size_t)W, nan);
     }
     out->n_windows = W;
-
-    for (int64_t w = 0; w < W; ++w) {
-        const float* Rw = R + (size_t)(w * p.stride) * (size_t)ldr;
-        for (int c = 0; c < 2; ++c) {
-            if (!kind_on[c]) continue;
-            SYMNMF_CUDA_TRY(cudaEventRecord(ev_build.a, s));
-            if (c == 0)
-                SYMNMF_TRY(symnmf_build_corr(Rw, T, n, ldr, S, lds, L.shared, L.shared_bytes, s));
-            else
-                SYMNMF_TRY(symnmf_build_tpdm(Rw, T, n, ldr, p.tail_frac, p.tail_sign, S, lds,
-                                             L.shared, L.shared_bytes, s));
-            SYMNMF_CUDA_TRY(cudaEventRecord(ev_build.b, s));
-            double cross = nan;
-            if (monitor) {
-                SYMNMF_TRY(symnmf_sh(S, n, lds, L.Z, G, L.Y, L.shared, L.shared_bytes, s));
-                cross_partial_kernel<<<cross_blocks(d), RL_THREADS, 0, s>>>(L.Y, L.Z, n, G, L.part);
-                SYMNMF_LAUNCH_CHECK();
-                cross_final_kernel<<<1, RL_THREADS, 0, s>>>(L.part, cross_blocks(d), L.counts, G,
-                                                            L.cross);
-                SYMNMF_LAUNCH_CHECK();
-                SYMNMF_CUDA_TRY(cudaMemcpyAsync(&cross, L.cross, sizeof(double),
-                                                cudaMemcpyDeviceToHost, s));
-            }
-            count_launches();
-            SYMNMF_CUDA_TRY(cudaEventRecord(ev_fit.a, s));
-            symnmf_fit_stats st;
-            SYMNMF_TRY(symnmf_fit(S, n, lds, p.k, &p.fit, L.H, &st, L.shared, L.shared_bytes, s));
-            int32_t* lab = out->labels[c] + (size_t)w * (size_t)n;
-            SYMNMF_TRY(symnmf_labels(L.H, n, p.k, lab, s));
-            SYMNMF_CUDA_TRY(cudaEventRecord(ev_fit.b, s));
-            count_launches();
-            double prev = nan, dl = nan;
-            if (w >= 1) SYMNMF_TRY(ari_run(d, L.ari, lab - n, lab, n, p.k, &prev, nullptr, s));
-            if (w >= p.delta)
-                SYMNMF_TRY(ari_run(d, L.ari, lab - (size_t)p.delta * n, lab, n, p.k, &dl, nullptr, s));
-            count_launches();
-            // the fit and the ARI synchronised the stream: both event pairs are complete
-            out->build_ms[c] += ev_build.ms();
-            out->fit_ms[c] += ev_fit.ms();
-            ari_delta[c][(size_t)w] = dl;
-            if (out->ari_prev[c]) out->ari_prev[c][w] = prev;
-            if (out->ari_delta[c]) out->ari_delta[c][w] = dl;
-            if (out->cross[c]) out->cross[c][w] = cross;
-            if (out->loss[c]) out->loss[c][w] = st.loss;
+    StudyArgs A{&d, R, n, ldr, T, W, &p, monitor, G, L.Z, L.counts, out};
+    ChainRun run[2];
+    for (int c = 0; c < 2; ++c) {
+        run[c].kind = c;
+        run[c].C = &L.chain[0];
+        run[c].S = S;
+        run[c].lds = lds;
+        run[c].s = s;
+    }
+    if (concurrent) {
+        // the TPDM chain: its own stream (after the setup above on s), buffers,
+        // matrix and host thread; s waits for it before the call returns
+        int dev = 0;
+        SYMNMF_CUDA_TRY(cudaGetDevice(&dev));
+        cudaStream_t s2 = nullptr;
+        cudaEvent_t e_in = nullptr, e_out = nullptr;
+        SYMNMF_CUDA_TRY(cudaStreamCreateWithFlags(&s2, cudaStreamNonBlocking));
+        auto release = [&]() {
+            if (e_in) cudaEventDestroy(e_in);
+            if (e_out) cudaEventDestroy(e_out);
+            cudaStreamDestroy(s2);
+        };
+        if (cudaEventCreateWithFlags(&e_in, cudaEventDisableTiming) != cudaSuccess ||
+            cudaEventCreateWithFlags(&e_out, cudaEventDisableTiming) != cudaSuccess ||
+            cudaEventRecord(e_in, s) != cudaSuccess || cudaStreamWaitEvent(s2, e_in, 0) != cudaSuccess) {
+            release();
+            set_error("could not order the second rolling stream");
+            return SYMNMF_ERR_CUDA;
         }
+        run[1].C = &L.chain[1];
+        run[1].S = L.S2;
+        run[1].lds = L.lds2;
+        run[1].s = s2;
+        std::thread worker([&]() {
+            ChainRun& r = run[1];
+            if (cudaSetDevice(dev) != cudaSuccess) {
+                r.rc = SYMNMF_ERR_CUDA;
+                r.err = "cudaSetDevice failed in the second rolling chain";
+                return;
+            }
+            r.rc = run_chain(A, r);
+            if (r.rc != SYMNMF_OK) r.err = symnmf_last_error();
+        });
+        run[0].rc = run_chain(A, run[0]);
+        const std::string err0 = run[0].rc != SYMNMF_OK ? std::string(symnmf_last_error()) : "";
+        worker.join();
+        const bool joined = cudaEventRecord(e_out, s2) == cudaSuccess &&
+                            cudaStreamWaitEvent(s, e_out, 0) == cudaSuccess;
+        release();
+        if (run[0].rc != SYMNMF_OK) {
+            set_error("%s", err0.c_str());
+            return run[0].rc;
+        }
+        if (run[1].rc != SYMNMF_OK) {
+            set_error("%s", run[1].err.c_str());
+            return run[1].rc;
+        }
+        if (!joined) {
+            set_error("could not order the caller's stream after the second rolling chain");
+            return SYMNMF_ERR_CUDA;
+        }
+    } else {
+        for (int c = 0; c < 2; ++c)
+            if (kind_on[c]) SYMNMF_TRY(run_chain(A, run[c]));
     }
     SYMNMF_CUDA_TRY(cudaEventRecord(whole.b, s));
     SYMNMF_CUDA_TRY(cudaEventSynchronize(whole.b));
@@ -384,19 +529,23 @@ static int rolling_impl(const float* R, int64_t days, int64_t n, int64_t ldr, co
     const int64_t c1 = p.calib_end > 0 ? std::min<int64_t>(p.calib_end, W) : W;
     for (int c = 0; c < 2; ++c) {
         if (!kind_on[c]) continue;
+        out->build_ms[c] = run[c].build_ms;
+        out->fit_ms[c] = run[c].fit_ms;
+        launches_total += run[c].launches;
+        const std::vector<double>& ad = run[c].ari_delta;
         double sum = 0.0;
         int64_t m = 0;
         for (int64_t t = c0; t < c1; ++t)
-            if (std::isfinite(ari_delta[c][(size_t)t])) {
-                sum += ari_delta[c][(size_t)t];
+            if (std::isfinite(ad[(size_t)t])) {
+                sum += ad[(size_t)t];
                 ++m;
             }
         if (m >= 2) {
             const double mu = sum / (double)m;
             double ss = 0.0;
             for (int64_t t = c0; t < c1; ++t)
-                if (std::isfinite(ari_delta[c][(size_t)t])) {
-                    const double dv = ari_delta[c][(size_t)t] - mu;
+                if (std::isfinite(ad[(size_t)t])) {
+                    const double dv = ad[(size_t)t] - mu;
                     ss += dv * dv;
                 }
             out->mean[c] = mu;
@@ -405,7 +554,7 @@ static int rolling_impl(const float* R, int64_t days, int64_t n, int64_t ldr, co
         }
         if (out->flag[c])
             for (int64_t t = 0; t < W; ++t) {
-                const double v = ari_delta[c][(size_t)t];
+                const double v = ad[(size_t)t];
                 out->flag[c][t] = (std::isfinite(v) && std::isfinite(out->limit[c]) &&
                                    v < out->limit[c]) ? 1 : 0;
             }

@@ -55,6 +55,28 @@ def test_stats_matches_oracle(m, n):
     assert abs(got[1] - sq) <= 1e-12 * sq
 
 
+@pytest.mark.parametrize("n", [513, 1024])
+def test_stats_full_float_range(m, n):
+    # the pass widens a group of four values by moving bit fields when all four
+    # are normal and through the conversion otherwise: mix every class into the
+    # groups -- both signs over the whole normal range, the extreme normals,
+    # signed zeros, subnormals, infinities and NaN (n = 513 adds a ragged tail)
+    rng = np.random.default_rng(n)
+    mag = 10.0 ** rng.uniform(-37.0, 37.0, size=(n, n))
+    S = (rng.choice([-1.0, 1.0], size=(n, n)) * mag).astype(np.float32)
+    specials = np.array([0.0, -0.0, 1e-40, -3e-42, 1.4e-45, np.float32(2.0 ** -126),
+                         -np.float32(2.0 ** -126), np.finfo(np.float32).max,
+                         -np.finfo(np.float32).max, np.inf, -np.inf, np.nan], dtype=np.float32)
+    pick = rng.random((n, n)) < 0.05
+    S[pick] = rng.choice(specials, size=int(pick.sum()))
+    got = m.stats(to_dev(S, DEV, pad4=True)).cpu().numpy()
+    s, sq, bad = oracle.stats(S)
+    absum = float(np.abs(np.where(np.isfinite(S), S, 0.0).astype(np.float64)).sum())
+    assert got[2] == bad
+    assert abs(got[0] - s) <= 1e-12 * absum   # relative to sum |S|: the signs cancel
+    assert abs(got[1] - sq) <= 1e-12 * sq
+
+
 @pytest.mark.parametrize("n,k", [(2000, 24), (2000, 8), (1999, 7), (2001, 33), (1500, 64), (3, 1), (1, 1)])
 def test_sh_matches_oracle(m, n, k):
     _, _, S = corr_problem(n, 60, seed=n)

@@ -168,3 +168,41 @@ def test_rolling_full_size_sampled_windows(m):
             assert got[kind]["ari_delta"][174] == ref[kind]["ari_delta"][174]
         a = got[kind]["ari_delta"]
         assert np.all(np.isnan(a[:50])) and np.all((a[50:] >= -1.0) & (a[50:] <= 1.0))
+
+
+def _same(x, y):
+    return np.array_equal(np.asarray(x), np.asarray(y), equal_nan=True)
+
+
+def test_rolling_concurrent_chains_match_serial(m, monkeypatch):
+    # with both kinds the TPDM windows run on a second stream and host thread;
+    # every output must equal the one-after-the-other run bit for bit, and so
+    # must a run whose workspace is one second matrix short of the full size
+    import ctypes as C
+    import torch
+    from symmetric_nmf_clustering_b200 import _lib as L
+    st = _stream_small()
+    R = to_dev(st.R, DEV, pad4=True)
+    groups = to_dev(st.groups_before.astype(np.int32), DEV)
+    kw = dict(groups=groups, window=60, k=6, delta=10, calib_begin=10, calib_end=20,
+              tail_frac=0.05, tail_sign=-1, stressed=list(st.stressed),
+              fit=dict(max_iters=60, seed=3))
+    conc = m.rolling(R, **kw)
+    monkeypatch.setenv("SYMNMF_ROLLING_SERIAL", "1")
+    serial = m.rolling(R, **kw)
+    monkeypatch.delenv("SYMNMF_ROLLING_SERIAL")
+    n = st.R.shape[1]
+    p = m.rolling_params(window=60, k=6, fit=dict(max_iters=60, seed=3))
+    size = C.c_size_t(0)
+    L.check("symnmf_workspace_size", L.load().symnmf_workspace_size(
+        L.OP_ROLLING, n, p.k, p.window, C.byref(p.fit), C.byref(size)))
+    short = size.value - n * ((n + 3) // 4 * 4) * 4
+    small = m.rolling(R, ws=torch.empty(short, dtype=torch.uint8, device=DEV), **kw)
+    for other in (serial, small):
+        for kind in ("corr", "tpdm"):
+            a, b = conc[kind], other[kind]
+            assert torch.equal(a["labels"], b["labels"]), kind
+            for key in ("loss", "cross", "ari_prev", "ari_delta", "flags"):
+                assert _same(a[key], b[key]), (kind, key)
+            for key in ("mean", "std", "limit"):
+                assert _same(a[key], b[key]), (kind, key)
