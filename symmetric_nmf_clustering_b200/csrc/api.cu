@@ -960,12 +960,11 @@ static int probe_impl(const Dev& d, const float* S, int64_t n, int64_t lds, int 
                                       cudaMemcpyDeviceToDevice, s));
     SYMNMF_TRY(orthonormalize(L, L.Q, n, ldq, b, L.Q, ldq, 0, seed + 1, B, s));
     bool converged = false;
-    int have = 0;  // columns of T resolved
+    // W = S Q_0 (one S pass)
+    SYMNMF_TRY(stream_pass(d, sa, L.Q, nullptr, ldq, 0, n, false, epi_product(n, b, L.W), s, nullptr));
     for (int j = 0; j < steps; ++j) {
-        // W = S Q_j (one S pass)
-        SYMNMF_TRY(stream_pass(d, sa, L.Q + (size_t)j * b, nullptr, ldq, 0, n, false,
-                               epi_product(n, b, L.W), s, nullptr));
-        // full reorthogonalisation against Q_0..Q_j, twice; the Q_j coefficients are A_j
+        // W holds S Q_j: full reorthogonalisation against Q_0..Q_j, twice; the
+        // Q_j coefficients are A_j
         const int nq = (j + 1) * b;
         coef.assign((size_t)nq * b, 0.0);
         for (int pass = 0; pass < 2; ++pass)
@@ -975,8 +974,27 @@ static int probe_impl(const Dev& d, const float* S, int64_t n, int64_t lds, int 
                 const double v = 0.5 * (coef[(size_t)(j * b + r) * b + c2] + coef[(size_t)(j * b + c2) * b + r]);
                 T[(size_t)(j * b + r) * mtot + j * b + c2] = v;
             }
-        have = nq;
-        // Rayleigh-Ritz on the block tridiagonal T of the basis so far
+        // next block W = Q_{j+1} B_{j+1}, and its S pass goes out before the
+        // Rayleigh-Ritz step below, so that the host's eigenvalue work runs
+        // while the GPU streams S (one pass is wasted when this block
+        // converges)
+        const bool more = j + 1 < steps;
+        if (more) {
+            float* Qn = L.Q + (size_t)(j + 1) * b;
+            SYMNMF_CUDA_TRY(cudaMemcpy2DAsync(Qn, ldq * sizeof(float), L.W, b * sizeof(float),
+                                              (size_t)b * sizeof(float), (size_t)n,
+                                              cudaMemcpyDeviceToDevice, s));
+            SYMNMF_TRY(orthonormalize(L, Qn, n, ldq, b, L.Q, ldq, nq, seed + 2 + j, B, s));
+            for (int r = 0; r < b; ++r)
+                for (int c2 = 0; c2 < b; ++c2) {
+                    const double v = B[(size_t)r * b + c2];
+                    T[(size_t)((j + 1) * b + r) * mtot + j * b + c2] = v;
+                    T[(size_t)(j * b + c2) * mtot + (j + 1) * b + r] = v;
+                }
+            SYMNMF_TRY(stream_pass(d, sa, Qn, nullptr, ldq, 0, n, false, epi_product(n, b, L.W), s,
+                                   nullptr));
+        }
+        // Rayleigh-Ritz on the leading nq x nq block of the block tridiagonal T
         if (nq >= n_eig) {
             std::vector<double> sub((size_t)nq * nq);
             for (int r = 0; r < nq; ++r)
@@ -989,21 +1007,8 @@ static int probe_impl(const Dev& d, const float* S, int64_t n, int64_t lds, int 
             }
             prev = theta;
         }
-        if (converged || j + 1 >= steps) break;
-        // next block: W = Q_{j+1} B_{j+1}
-        float* Qn = L.Q + (size_t)(j + 1) * b;
-        SYMNMF_CUDA_TRY(cudaMemcpy2DAsync(Qn, ldq * sizeof(float), L.W, b * sizeof(float),
-                                          (size_t)b * sizeof(float), (size_t)n,
-                                          cudaMemcpyDeviceToDevice, s));
-        SYMNMF_TRY(orthonormalize(L, Qn, n, ldq, b, L.Q, ldq, nq, seed + 2 + j, B, s));
-        for (int r = 0; r < b; ++r)
-            for (int c2 = 0; c2 < b; ++c2) {
-                const double v = B[(size_t)r * b + c2];
-                T[(size_t)((j + 1) * b + r) * mtot + j * b + c2] = v;
-                T[(size_t)(j * b + c2) * mtot + (j + 1) * b + r] = v;
-            }
+        if (converged || !more) break;
     }
-    (void)have;
     {
         int kerr = 0;
         SYMNMF_CUDA_TRY(cudaMemcpyAsync(&kerr, L.err, sizeof(int), cudaMemcpyDeviceToHost, s));
