@@ -206,3 +206,18 @@ def test_rolling_concurrent_chains_match_serial(m, monkeypatch):
                 assert _same(a[key], b[key]), (kind, key)
             for key in ("mean", "std", "limit"):
                 assert _same(a[key], b[key]), (kind, key)
+
+
+def test_rolling_error_in_the_second_chain_is_reported(m):
+    # tail_frac is checked by the TPDM builder only: the TPDM chain (second
+    # stream and host thread) fails at its first window while the |corr| chain
+    # runs on, and the call reports the TPDM builder's error
+    from symmetric_nmf_clustering_b200 import _lib as L
+    st = _stream_small()
+    R = to_dev(st.R, DEV, pad4=True)
+    with pytest.raises(L.SymNMFError) as e:
+        m.rolling(R, window=60, k=6, kinds=3, delta=5, tail_frac=0.0, fit=dict(max_iters=5))
+    assert "tail_frac" in str(e.value)
+    # the library is still usable afterwards
+    ok = m.rolling(R, window=60, k=6, kinds=3, delta=5, n_windows=3, fit=dict(max_iters=5))
+    assert ok["n_windows"] == 3
