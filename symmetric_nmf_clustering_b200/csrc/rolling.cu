@@ -488,7 +488,7 @@ static int rolling_impl(const float* R, int64_t days, int64_t n, int64_t ldr, co
         run[1].S = L.S2;
         run[1].lds = L.lds2;
         run[1].s = s2;
-        std::thread worker([&]() {
+        auto second = [&]() {
             ChainRun& r = run[1];
             if (cudaSetDevice(dev) != cudaSuccess) {
                 r.rc = SYMNMF_ERR_CUDA;
@@ -497,10 +497,18 @@ static int rolling_impl(const float* R, int64_t days, int64_t n, int64_t ldr, co
             }
             r.rc = run_chain(A, r);
             if (r.rc != SYMNMF_OK) r.err = symnmf_last_error();
-        });
+        };
+        std::thread worker;
+        bool threaded = true;
+        try {
+            worker = std::thread(second);
+        } catch (...) {   // no thread to be had: the second chain follows the first
+            threaded = false;
+        }
         run[0].rc = run_chain(A, run[0]);
         const std::string err0 = run[0].rc != SYMNMF_OK ? std::string(symnmf_last_error()) : "";
-        worker.join();
+        if (threaded) worker.join();
+        else if (run[0].rc == SYMNMF_OK) second();
         const bool joined = cudaEventRecord(e_out, s2) == cudaSuccess &&
                             cudaStreamWaitEvent(s, e_out, 0) == cudaSuccess;
         release();
