@@ -89,9 +89,18 @@ static void householder_tridiag(int m, std::vector<double>& A, std::vector<doubl
         const double beta = 2.0 / vnorm2;
         // trailing block B = A[k+1:, k+1:]: B <- (I - beta v v^T) B (I - beta v v^T)
         for (int i = k + 1; i < m; ++i) {
-            double s = 0.0;
-            for (int j = k + 1; j < m; ++j) s += a(i, j) * v[j];
-            p[i] = beta * s;
+            // four independent partial sums (latency, not flops, bounds this loop)
+            const double* ai = &a(i, 0);
+            double s0 = 0.0, s1 = 0.0, s2 = 0.0, s3 = 0.0;
+            int j = k + 1;
+            for (; j + 3 < m; j += 4) {
+                s0 += ai[j] * v[j];
+                s1 += ai[j + 1] * v[j + 1];
+                s2 += ai[j + 2] * v[j + 2];
+                s3 += ai[j + 3] * v[j + 3];
+            }
+            for (; j < m; ++j) s0 += ai[j] * v[j];
+            p[i] = beta * ((s0 + s1) + (s2 + s3));
         }
         double K = 0.0;
         for (int i = k + 1; i < m; ++i) K += v[i] * p[i];
@@ -107,20 +116,25 @@ static void householder_tridiag(int m, std::vector<double>& A, std::vector<doubl
     d[m - 1] = a(m - 1, m - 1);
 }
 
-// Number of eigenvalues of the tridiagonal (d, e) that are < x (Sturm count
-// through the pivots of the LDL^T factorisation of T - x I).
-static int sturm_below(const std::vector<double>& d, const std::vector<double>& e, double x) {
+// Number of eigenvalues of the tridiagonal (d, e) below each of four shifts
+// x[r] (Sturm counts through the pivots of the LDL^T factorisations of
+// T - x[r] I), as four independent recurrences so that their divisions overlap.
+static void sturm_below4(const std::vector<double>& d, const std::vector<double>& e,
+                         const double x[4], int c[4]) {
     const int m = (int)d.size();
-    int count = 0;
-    double q = 1.0;
     const double tiny = std::numeric_limits<double>::min();
+    double q[4] = {1.0, 1.0, 1.0, 1.0};
+    int cnt[4] = {0, 0, 0, 0};
     for (int i = 0; i < m; ++i) {
         const double e2 = i > 0 ? e[i - 1] * e[i - 1] : 0.0;
-        q = (d[i] - x) - (i > 0 ? e2 / q : 0.0);
-        if (q == 0.0) q = -tiny;
-        if (q < 0.0) ++count;
+        for (int r = 0; r < 4; ++r) {
+            double v = (d[i] - x[r]) - (i > 0 ? e2 / q[r] : 0.0);
+            if (v == 0.0) v = -tiny;
+            cnt[r] += v < 0.0 ? 1 : 0;
+            q[r] = v;
+        }
     }
-    return count;
+    for (int r = 0; r < 4; ++r) c[r] = cnt[r];
 }
 
 void sym_top_eigvals(int m, std::vector<double> A, int count, std::vector<double>& out) {
@@ -138,18 +152,39 @@ void sym_top_eigvals(int m, std::vector<double> A, int count, std::vector<double
     hi += 1e-6 * span;
     count = std::min(count, m);
     out.assign(count, 0.0);
-    for (int j = 0; j < count; ++j) {
-        // the (j+1)-th largest eigenvalue = the (m-j)-th smallest: find x with
-        // sturm_below(x) <= m-j-1 < sturm_below(x') for the tightest bracket
-        const int idx = m - 1 - j;  // 0-based ascending index
-        double a = lo, b = hi;
+    // brackets [blo, bhi] of every target; every Sturm count narrows the
+    // brackets of all targets.  Four targets are bisected in lockstep so that
+    // their Sturm recurrences (chains of dependent divisions) overlap.
+    std::vector<double> blo(count, lo), bhi(count, hi);
+    constexpr int G = 4;
+    for (int j0 = 0; j0 < count; j0 += G) {
+        const int g = std::min(G, count - j0);
+        bool done[G] = {false, false, false, false};
         for (int it = 0; it < 200; ++it) {
-            const double mid = 0.5 * (a + b);
-            if (mid == a || mid == b) break;
-            if (sturm_below(d, e, mid) <= idx) a = mid;
-            else b = mid;
+            double mid[G];
+            bool any = false;
+            for (int q = 0; q < G; ++q) {
+                mid[q] = 0.0;
+                if (q >= g || done[q]) continue;
+                const double a = blo[j0 + q], b = bhi[j0 + q];
+                mid[q] = 0.5 * (a + b);
+                if (mid[q] == a || mid[q] == b) done[q] = true;
+                else any = true;
+            }
+            if (!any) break;
+            int c[G];
+            sturm_below4(d, e, mid, c);
+            for (int q = 0; q < g; ++q) {
+                if (done[q]) continue;
+                // eigenvalues below mid[q]: c[q]; the target of ascending index
+                // m-1-j lies at or above mid[q] iff c[q] <= m-1-j
+                for (int j = j0; j < count; ++j) {
+                    if (c[q] <= m - 1 - j) blo[j] = std::max(blo[j], mid[q]);
+                    else bhi[j] = std::min(bhi[j], mid[q]);
+                }
+            }
         }
-        out[j] = 0.5 * (a + b);
+        for (int q = 0; q < g; ++q) out[j0 + q] = 0.5 * (blo[j0 + q] + bhi[j0 + q]);
     }
 }
 
