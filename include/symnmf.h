@@ -339,13 +339,15 @@ SYMNMF_API void symnmf_rolling_params_default(symnmf_rolling_params* p);
 /*
  * Runs the study above.  S: the caller's n x n fp32 buffer (lds a multiple of
  * 4), overwritten window by window.  groups may be NULL when n_stressed = 0.
- * Workspace: SYMNMF_OP_ROLLING with T = window and params = &p->fit; that size
- * holds a second chain (its own n x n matrix and buffers), and with both kinds
- * selected the TPDM windows then run on a stream and host thread of their own,
- * beside the |corr| windows on `stream` (ordered after `stream`'s earlier work;
- * `stream` waits for them before the call returns).  A smaller workspace that
- * still holds one chain, or the environment variable SYMNMF_ROLLING_SERIAL=1,
- * runs the kinds one after the other; the results are the same.  Synchronises
+ * Workspace: SYMNMF_OP_ROLLING with T = window and params = &p->fit.  That
+ * size holds four chains: each selected kind's windows are split between two
+ * chains (alternate windows), each chain after the first with its own n x n
+ * matrix and buffers, running on a stream and host thread of its own (the
+ * chains are ordered after `stream`'s earlier work and `stream` waits for
+ * them before the call returns); the ARI series is computed from the stored
+ * labels afterwards.  A smaller workspace runs one chain per kind, or a
+ * single chain that takes the kinds in turn (also forced by the environment
+ * variable SYMNMF_ROLLING_SERIAL=1); the results are the same.  Synchronises
  * the streams once per window and kind (the fit reads its state).
  */
 SYMNMF_API int symnmf_rolling(const float* R, int64_t days, int64_t n, int64_t ldr,

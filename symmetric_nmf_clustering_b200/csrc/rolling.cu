@@ -6,11 +6,12 @@
 // and the window delta earlier; a 3-sigma control limit on the latter.
 //
 // The driver composes the library's own entry points (builders, fit, labels,
-// S-stream product); with both kinds selected it runs the |corr| chain on the
-// caller's stream and the TPDM chain on a second stream from a second host
-// thread, each window's passes being latency-bound at this size.  This file
-// adds the contingency-table kernel behind the ARI and the monitor's
-// reduction kernels.
+// S-stream product).  The windows are independent fits, each pass of which is
+// latency-bound at the workload's size, so the driver runs up to four chains
+// side by side -- two per dependence matrix, taking alternate windows -- each
+// on its own stream and host thread with its own matrix and buffers; the ARI
+// series follows from the stored labels.  This file adds the contingency-table
+// kernel behind the ARI and the monitor's reduction kernels.
 #include <cmath>
 #include <cstring>
 #include <cstdlib>
@@ -199,24 +200,27 @@ __global__ void cross_final_kernel(const double* __restrict__ part, int nblk,
 
 // ---------------------------------------------------------------- workspace
 
-// One chain's buffers: a chain is one dependence matrix over every window
-// (build, monitor, fit, labels, ARI on its own stream).
+// One chain's buffers.  A chain runs every P-th window of one dependence
+// matrix (build, monitor, fit, labels) on its own stream.
 struct ChainLayout {
     void* shared = nullptr;      // builders, fit and the monitor's product take turns here
     size_t shared_bytes = 0;
     float* H = nullptr;
-    AriLayout ari;
     float* Y = nullptr;          // n x 8 product S Z
     double* part = nullptr;
     double* cross = nullptr;     // the current window's monitor value
 };
 
+constexpr int RL_MAX_CHAINS = 4;    // two per kind
+
 struct RollingLayout {
-    ChainLayout chain[2];        // chain[1] only when the two kinds run concurrently
-    float* S2 = nullptr;         // the second chain's n x n matrix, row stride lds2
-    int64_t lds2 = 0;
+    ChainLayout chain[RL_MAX_CHAINS];
+    float* S_own[RL_MAX_CHAINS] = {};   // matrices of chains 1.. (chain 0 uses the caller's S)
+    int64_t lds_own = 0;
+    int nchains = 1;
     float* Z = nullptr;          // n x 8 indicator of the stressed groups (read-only)
     int* counts = nullptr;
+    AriLayout ari;               // the ARI series, computed after the fits
 };
 
 static int cross_blocks(const Dev& d) { return 2 * d.sms; }
@@ -230,28 +234,28 @@ static void chain_plan(const Dev& d, Arena& a, int64_t n, int k, size_t shared_b
     C->shared_bytes = shared_bytes;
     C->shared = a.take<char>(shared_bytes);
     C->H = a.take<float>((size_t)n * k);
-    ari_plan(a, &C->ari);
     C->Y = a.take<float>((size_t)n * RL_MAX_STRESSED);
     C->part = a.take<double>((size_t)cross_blocks(d));
     C->cross = a.take<double>(64);
 }
 
-// concurrent: room for both chains and the second n x n matrix
+// nchains chains: each after the first gets its own n x n matrix
 int rolling_plan(const Dev& d, Arena& a, int64_t n, int k, int64_t T, const symnmf_fit_params& P,
-                 bool concurrent, RollingLayout* L) {
+                 int nchains, RollingLayout* L) {
     size_t b_corr = 0, b_tpdm = 0, b_fit = 0, b_sh = 0;
     SYMNMF_TRY(sub_ws(SYMNMF_OP_BUILD_CORR, n, k, T, &P, &b_corr));
     SYMNMF_TRY(sub_ws(SYMNMF_OP_BUILD_TPDM, n, k, T, &P, &b_tpdm));
     SYMNMF_TRY(sub_ws(SYMNMF_OP_FIT, n, k, T, &P, &b_fit));
     SYMNMF_TRY(sub_ws(SYMNMF_OP_SH, n, RL_MAX_STRESSED, T, &P, &b_sh));
     const size_t shared = std::max(std::max(b_corr, b_tpdm), std::max(b_fit, b_sh));
+    L->nchains = nchains;
     L->Z = a.take<float>((size_t)n * RL_MAX_STRESSED);
     L->counts = a.take<int>(64);
-    chain_plan(d, a, n, k, shared, &L->chain[0]);
-    if (concurrent) {
-        chain_plan(d, a, n, k, shared, &L->chain[1]);
-        L->lds2 = (n + 3) / 4 * 4;
-        L->S2 = a.take<float>((size_t)n * (size_t)L->lds2);
+    ari_plan(a, &L->ari);
+    L->lds_own = (n + 3) / 4 * 4;
+    for (int c = 0; c < nchains; ++c) {
+        chain_plan(d, a, n, k, shared, &L->chain[c]);
+        if (c > 0) L->S_own[c] = a.take<float>((size_t)n * (size_t)L->lds_own);
     }
     return SYMNMF_OK;
 }
@@ -269,7 +273,7 @@ int rolling_workspace_bytes(const Dev& d, int64_t n, int k, int64_t T, const sym
     Arena a;
     a.dry = true;
     RollingLayout L;
-    SYMNMF_TRY(rolling_plan(d, a, n, k, T, P, true, &L));
+    SYMNMF_TRY(rolling_plan(d, a, n, k, T, P, RL_MAX_CHAINS, &L));
     *bytes = a.used + 256;
     return SYMNMF_OK;
 }
@@ -297,12 +301,12 @@ struct EventPair {
 // What one chain needs and what it reports.
 struct ChainRun {
     int kind = 0;                // 0 = |corr|, 1 = TPDM
+    int64_t first = 0, step = 1; // windows first, first + step, ...
     const ChainLayout* C = nullptr;
     float* S = nullptr;
     int64_t lds = 0;
     cudaStream_t s = nullptr;
     double build_ms = 0.0, fit_ms = 0.0;
-    std::vector<double> ari_delta;
     int launches = 0;
     int rc = SYMNMF_OK;
     std::string err;
@@ -320,14 +324,13 @@ struct StudyArgs {
     symnmf_rolling_out* out;
 };
 
-// Every window of one kind on r.s: build, monitor, fit, labels, the two ARIs.
+// The chain's windows on r.s: build, monitor, fit, labels (the ARIs come after).
 static int run_chain(const StudyArgs& A, ChainRun& r) {
     const symnmf_rolling_params& p = *A.p;
     const ChainLayout& L = *r.C;
     const int64_t n = A.n;
     const int c = r.kind;
     const double nan = std::numeric_limits<double>::quiet_NaN();
-    r.ari_delta.assign((size_t)A.W, nan);
     EventPair ev_build, ev_fit;
     SYMNMF_TRY(ev_build.create());
     SYMNMF_TRY(ev_fit.create());
@@ -336,7 +339,7 @@ static int run_chain(const StudyArgs& A, ChainRun& r) {
         reset_launches();
     };
     reset_launches();
-    for (int64_t w = 0; w < A.W; ++w) {
+    for (int64_t w = r.first; w < A.W; w += r.step) {
         const float* Rw = A.R + (size_t)(w * p.stride) * (size_t)A.ldr;
         SYMNMF_CUDA_TRY(cudaEventRecord(ev_build.a, r.s));
         if (c == 0)
@@ -366,28 +369,90 @@ static int run_chain(const StudyArgs& A, ChainRun& r) {
         SYMNMF_TRY(symnmf_labels(L.H, n, p.k, lab, r.s));
         count();
         SYMNMF_CUDA_TRY(cudaEventRecord(ev_fit.b, r.s));
-        double prev = nan, dl = nan;
-        if (w >= 1) SYMNMF_TRY(ari_run(*A.d, L.ari, lab - n, lab, n, p.k, &prev, nullptr, r.s));
-        if (w >= p.delta)
-            SYMNMF_TRY(ari_run(*A.d, L.ari, lab - (size_t)p.delta * n, lab, n, p.k, &dl, nullptr, r.s));
-        count();
-        // the fit and the ARI synchronised the stream: both event pairs are complete
-        SYMNMF_CUDA_TRY(cudaStreamSynchronize(r.s));
+        SYMNMF_CUDA_TRY(cudaStreamSynchronize(r.s));   // both event pairs complete, cross read
         r.build_ms += ev_build.ms();
         r.fit_ms += ev_fit.ms();
-        r.ari_delta[(size_t)w] = dl;
-        if (A.out->ari_prev[c]) A.out->ari_prev[c][w] = prev;
-        if (A.out->ari_delta[c]) A.out->ari_delta[c][w] = dl;
         if (A.out->cross[c]) A.out->cross[c][w] = cross;
         if (A.out->loss[c]) A.out->loss[c][w] = st.loss;
     }
     return SYMNMF_OK;
 }
 
-// Two kinds side by side unless SYMNMF_ROLLING_SERIAL=1 (read at each call).
+// Chains side by side unless SYMNMF_ROLLING_SERIAL=1 (read at each call).
 static bool rolling_serial() {
     const char* e = getenv("SYMNMF_ROLLING_SERIAL");
     return e != nullptr && std::strcmp(e, "1") == 0;
+}
+
+// Runs run[1..nc-1] on their own host threads (each on its own stream,
+// ordered after s) and run[0] on this thread and s; s then waits for them.
+// A chain whose thread cannot be started runs here after run[0].
+static int run_chains(const StudyArgs& A, ChainRun* run, int nc, cudaStream_t s) {
+    int dev = 0;
+    SYMNMF_CUDA_TRY(cudaGetDevice(&dev));
+    cudaEvent_t e_in = nullptr;
+    cudaStream_t streams[RL_MAX_CHAINS] = {};
+    cudaEvent_t e_out[RL_MAX_CHAINS] = {};
+    auto release = [&]() {
+        if (e_in) cudaEventDestroy(e_in);
+        for (int i = 1; i < nc; ++i) {
+            if (e_out[i]) cudaEventDestroy(e_out[i]);
+            if (streams[i]) cudaStreamDestroy(streams[i]);
+        }
+    };
+    bool ok = cudaEventCreateWithFlags(&e_in, cudaEventDisableTiming) == cudaSuccess &&
+              cudaEventRecord(e_in, s) == cudaSuccess;
+    for (int i = 1; ok && i < nc; ++i)
+        ok = cudaStreamCreateWithFlags(&streams[i], cudaStreamNonBlocking) == cudaSuccess &&
+             cudaEventCreateWithFlags(&e_out[i], cudaEventDisableTiming) == cudaSuccess &&
+             cudaStreamWaitEvent(streams[i], e_in, 0) == cudaSuccess;
+    if (!ok) {
+        release();
+        set_error("could not set up the rolling study's streams");
+        return SYMNMF_ERR_CUDA;
+    }
+    auto body = [&](int i) {
+        ChainRun& r = run[i];
+        if (cudaSetDevice(dev) != cudaSuccess) {
+            r.rc = SYMNMF_ERR_CUDA;
+            r.err = "cudaSetDevice failed in a rolling chain";
+            return;
+        }
+        r.rc = run_chain(A, r);
+        if (r.rc != SYMNMF_OK) r.err = symnmf_last_error();
+    };
+    std::thread workers[RL_MAX_CHAINS];
+    bool threaded[RL_MAX_CHAINS] = {};
+    for (int i = 1; i < nc; ++i) {
+        run[i].s = streams[i];
+        try {
+            workers[i] = std::thread(body, i);
+            threaded[i] = true;
+        } catch (...) {   // no thread to be had: this chain runs here after chain 0
+            threaded[i] = false;
+        }
+    }
+    run[0].rc = run_chain(A, run[0]);
+    if (run[0].rc != SYMNMF_OK) run[0].err = symnmf_last_error();
+    for (int i = 1; i < nc; ++i) {
+        if (threaded[i]) workers[i].join();
+        else body(i);
+    }
+    bool joined = true;
+    for (int i = 1; i < nc; ++i)
+        joined = joined && cudaEventRecord(e_out[i], streams[i]) == cudaSuccess &&
+                 cudaStreamWaitEvent(s, e_out[i], 0) == cudaSuccess;
+    release();
+    for (int i = 0; i < nc; ++i)
+        if (run[i].rc != SYMNMF_OK) {
+            set_error("%s", run[i].err.c_str());
+            return run[i].rc;
+        }
+    if (!joined) {
+        set_error("could not order the caller's stream after the rolling chains");
+        return SYMNMF_ERR_CUDA;
+    }
+    return SYMNMF_OK;
 }
 
 static int rolling_impl(const float* R, int64_t days, int64_t n, int64_t ldr, const int32_t* groups,
@@ -408,24 +473,31 @@ static int rolling_impl(const float* R, int64_t days, int64_t n, int64_t ldr, co
             set_error("labels[%d] must be a device buffer of n_windows x n int32", c);
             return SYMNMF_ERR_INVALID_ARG;
         }
-    // the two chains run concurrently when both kinds are on and the workspace
-    // holds the second chain; otherwise one after the other
+    int kinds[2], nk = 0;
+    for (int c = 0; c < 2; ++c)
+        if (kind_on[c]) kinds[nk++] = c;
+    // chains: two per kind when the workspace holds them, else one per kind,
+    // else a single chain that runs the kinds in turn
     RollingLayout L;
-    bool concurrent = kind_on[0] && kind_on[1] && !rolling_serial();
+    int per_kind = 1, nc = 1;
     {
-        Arena a;
-        a.base = static_cast<char*>(ws);
-        a.cap = ws_bytes;
-        SYMNMF_TRY(rolling_plan(d, a, n, p.k, T, p.fit, concurrent, &L));
-        if (!a.ok() && concurrent) {
-            concurrent = false;
+        const int tries[3][2] = {{2, 2 * nk}, {1, nk}, {1, 1}};
+        bool fit = false;
+        for (int t = rolling_serial() ? 2 : 0; t < 3 && !fit; ++t) {
+            if (tries[t][1] > RL_MAX_CHAINS) continue;
+            Arena a;
+            a.base = static_cast<char*>(ws);
+            a.cap = ws_bytes;
             L = RollingLayout();
-            a.used = 0;
-            SYMNMF_TRY(rolling_plan(d, a, n, p.k, T, p.fit, false, &L));
-        }
-        if (!a.ok()) {
-            set_error("workspace too small: %zu given, %zu needed", ws_bytes, a.used);
-            return SYMNMF_ERR_WORKSPACE;
+            SYMNMF_TRY(rolling_plan(d, a, n, p.k, T, p.fit, tries[t][1], &L));
+            if (a.ok()) {
+                fit = true;
+                per_kind = tries[t][0];
+                nc = tries[t][1];
+            } else if (t == 2) {
+                set_error("workspace too small: %zu given, %zu needed", ws_bytes, a.used);
+                return SYMNMF_ERR_WORKSPACE;
+            }
         }
     }
     const bool monitor = p.n_stressed >= 2;
@@ -456,78 +528,56 @@ static int rolling_impl(const float* R, int64_t days, int64_t n, int64_t ldr, co
     }
     out->n_windows = W;
     StudyArgs A{&d, R, n, ldr, T, W, &p, monitor, G, L.Z, L.counts, out};
-    ChainRun run[2];
-    for (int c = 0; c < 2; ++c) {
-        run[c].kind = c;
-        run[c].C = &L.chain[0];
-        run[c].S = S;
-        run[c].lds = lds;
-        run[c].s = s;
+    ChainRun run[RL_MAX_CHAINS];
+    for (int i = 0; i < nc; ++i) {
+        run[i].C = &L.chain[i];
+        run[i].S = i == 0 ? S : L.S_own[i];
+        run[i].lds = i == 0 ? lds : L.lds_own;
+        run[i].s = s;
     }
-    if (concurrent) {
-        // the TPDM chain: its own stream (after the setup above on s), buffers,
-        // matrix and host thread; s waits for it before the call returns
-        int dev = 0;
-        SYMNMF_CUDA_TRY(cudaGetDevice(&dev));
-        cudaStream_t s2 = nullptr;
-        cudaEvent_t e_in = nullptr, e_out = nullptr;
-        SYMNMF_CUDA_TRY(cudaStreamCreateWithFlags(&s2, cudaStreamNonBlocking));
-        auto release = [&]() {
-            if (e_in) cudaEventDestroy(e_in);
-            if (e_out) cudaEventDestroy(e_out);
-            cudaStreamDestroy(s2);
-        };
-        if (cudaEventCreateWithFlags(&e_in, cudaEventDisableTiming) != cudaSuccess ||
-            cudaEventCreateWithFlags(&e_out, cudaEventDisableTiming) != cudaSuccess ||
-            cudaEventRecord(e_in, s) != cudaSuccess || cudaStreamWaitEvent(s2, e_in, 0) != cudaSuccess) {
-            release();
-            set_error("could not order the second rolling stream");
-            return SYMNMF_ERR_CUDA;
-        }
-        run[1].C = &L.chain[1];
-        run[1].S = L.S2;
-        run[1].lds = L.lds2;
-        run[1].s = s2;
-        auto second = [&]() {
-            ChainRun& r = run[1];
-            if (cudaSetDevice(dev) != cudaSuccess) {
-                r.rc = SYMNMF_ERR_CUDA;
-                r.err = "cudaSetDevice failed in the second rolling chain";
-                return;
-            }
-            r.rc = run_chain(A, r);
-            if (r.rc != SYMNMF_OK) r.err = symnmf_last_error();
-        };
-        std::thread worker;
-        bool threaded = true;
-        try {
-            worker = std::thread(second);
-        } catch (...) {   // no thread to be had: the second chain follows the first
-            threaded = false;
-        }
-        run[0].rc = run_chain(A, run[0]);
-        const std::string err0 = run[0].rc != SYMNMF_OK ? std::string(symnmf_last_error()) : "";
-        if (threaded) worker.join();
-        else if (run[0].rc == SYMNMF_OK) second();
-        const bool joined = cudaEventRecord(e_out, s2) == cudaSuccess &&
-                            cudaStreamWaitEvent(s, e_out, 0) == cudaSuccess;
-        release();
-        if (run[0].rc != SYMNMF_OK) {
-            set_error("%s", err0.c_str());
-            return run[0].rc;
-        }
-        if (run[1].rc != SYMNMF_OK) {
-            set_error("%s", run[1].err.c_str());
-            return run[1].rc;
-        }
-        if (!joined) {
-            set_error("could not order the caller's stream after the second rolling chain");
-            return SYMNMF_ERR_CUDA;
+    if (nc == 1) {
+        for (int q = 0; q < nk; ++q) {   // the kinds in turn on one chain
+            run[0].kind = kinds[q];
+            SYMNMF_TRY(run_chain(A, run[0]));
+            out->build_ms[kinds[q]] = run[0].build_ms;
+            out->fit_ms[kinds[q]] = run[0].fit_ms;
+            launches_total += run[0].launches;
+            run[0].build_ms = run[0].fit_ms = 0.0;
+            run[0].launches = 0;
         }
     } else {
-        for (int c = 0; c < 2; ++c)
-            if (kind_on[c]) SYMNMF_TRY(run_chain(A, run[c]));
+        for (int i = 0; i < nc; ++i) {
+            run[i].kind = kinds[i / per_kind];
+            run[i].first = i % per_kind;
+            run[i].step = per_kind;
+        }
+        SYMNMF_TRY(run_chains(A, run, nc, s));
+        for (int i = 0; i < nc; ++i) {
+            out->build_ms[run[i].kind] += run[i].build_ms;
+            out->fit_ms[run[i].kind] += run[i].fit_ms;
+            launches_total += run[i].launches;
+        }
     }
+
+    // ARI(t - 1, t) and ARI(t - delta, t) from the stored labels
+    std::vector<double> ari_delta[2];
+    reset_launches();
+    for (int c = 0; c < 2; ++c) {
+        if (!kind_on[c]) continue;
+        ari_delta[c].assign((size_t)W, nan);
+        const int32_t* lab = out->labels[c];
+        for (int64_t w = 0; w < W; ++w) {
+            double prev = nan, dl = nan;
+            const int32_t* lw = lab + (size_t)w * (size_t)n;
+            if (w >= 1) SYMNMF_TRY(ari_run(d, L.ari, lw - n, lw, n, p.k, &prev, nullptr, s));
+            if (w >= p.delta)
+                SYMNMF_TRY(ari_run(d, L.ari, lw - (size_t)p.delta * n, lw, n, p.k, &dl, nullptr, s));
+            ari_delta[c][(size_t)w] = dl;
+            if (out->ari_prev[c]) out->ari_prev[c][w] = prev;
+            if (out->ari_delta[c]) out->ari_delta[c][w] = dl;
+        }
+    }
+    launches_total += launches();
     SYMNMF_CUDA_TRY(cudaEventRecord(whole.b, s));
     SYMNMF_CUDA_TRY(cudaEventSynchronize(whole.b));
     out->total_ms = whole.ms();
@@ -537,10 +587,7 @@ static int rolling_impl(const float* R, int64_t days, int64_t n, int64_t ldr, co
     const int64_t c1 = p.calib_end > 0 ? std::min<int64_t>(p.calib_end, W) : W;
     for (int c = 0; c < 2; ++c) {
         if (!kind_on[c]) continue;
-        out->build_ms[c] = run[c].build_ms;
-        out->fit_ms[c] = run[c].fit_ms;
-        launches_total += run[c].launches;
-        const std::vector<double>& ad = run[c].ari_delta;
+        const std::vector<double>& ad = ari_delta[c];
         double sum = 0.0;
         int64_t m = 0;
         for (int64_t t = c0; t < c1; ++t)

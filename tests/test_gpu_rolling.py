@@ -175,9 +175,10 @@ def _same(x, y):
 
 
 def test_rolling_concurrent_chains_match_serial(m, monkeypatch):
-    # with both kinds the TPDM windows run on a second stream and host thread;
-    # every output must equal the one-after-the-other run bit for bit, and so
-    # must a run whose workspace is one second matrix short of the full size
+    # the full workspace runs four chains (two per kind, alternate windows) on
+    # their own streams and host threads; every output must equal the single-
+    # chain run bit for bit, and so must a run whose workspace is one matrix
+    # short of the full size (one chain per kind)
     import ctypes as C
     import torch
     from symmetric_nmf_clustering_b200 import _lib as L
