@@ -78,12 +78,11 @@ static int check_S(const float* S, int64_t n, int64_t lds) {
 // The tensor-core kernel is the S-stream; SYMNMF_STREAM=cuda_core selects the
 // CUDA-core kernel instead (same result within fp32 rounding), for comparison.
 static bool use_tc() {
-    static int v = -1;
-    if (v < 0) {
+    static const bool v = [] {   // read once (thread-safe static initialisation)
         const char* e = getenv("SYMNMF_STREAM");
-        v = (e != nullptr && std::strcmp(e, "cuda_core") == 0) ? 0 : 1;
-    }
-    return v == 1;
+        return !(e != nullptr && std::strcmp(e, "cuda_core") == 0);
+    }();
+    return v;
 }
 
 static size_t stream_partials(const Dev& d, int64_t n, int k, int64_t r0, int64_t r1) {
@@ -426,12 +425,11 @@ static int full_pass(FitCtx& c, int mode, int max_evals, bool xt_ready) {
 // launch-bound, and eager launches measured as fast or faster on B200
 // (n = 5,000: 6.0 ms per 100 iterations eager, 6.4 ms replayed).
 static bool use_graphs() {
-    static int v = -1;
-    if (v < 0) {
+    static const bool v = [] {   // read once (thread-safe static initialisation)
         const char* e = getenv("SYMNMF_GRAPHS");
-        v = (e != nullptr && std::strcmp(e, "1") == 0) ? 1 : 0;
-    }
-    return v == 1;
+        return e != nullptr && std::strcmp(e, "1") == 0;
+    }();
+    return v;
 }
 
 // Replays a captured graph of G full-batch passes on a private stream (ordered

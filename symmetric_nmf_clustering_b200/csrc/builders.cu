@@ -17,12 +17,11 @@ int launch_gram_tc(const float* ZF, const float* ZL, int64_t n, int64_t n_pad, i
 
 // Tensor-core Gram by default; SYMNMF_STREAM=cuda_core selects the CUDA-core one.
 static bool builders_tc() {
-    static int v = -1;
-    if (v < 0) {
+    static const bool v = [] {   // read once (thread-safe static initialisation)
         const char* e = getenv("SYMNMF_STREAM");
-        v = (e != nullptr && std::strcmp(e, "cuda_core") == 0) ? 0 : 1;
-    }
-    return v == 1;
+        return !(e != nullptr && std::strcmp(e, "cuda_core") == 0);
+    }();
+    return v;
 }
 constexpr int TCB_ROWS = 128;   // row padding of the transposed operands
 constexpr int TCB_K = 32;       // contraction padding of the transposed operands
@@ -572,13 +571,10 @@ int launch_tpdm(const float* R, int64_t T, int64_t n, int64_t ldr, int N,
         }
     } else if (P <= RS_MAX_P) {
         const size_t rs_smem = (size_t)RS_COLS * P * 8 + (size_t)T * RS_COLS * 4;
-        static bool rs_attr = false;   // once per process
-        if (!rs_attr) {
-            SYMNMF_CUDA_TRY(cudaFuncSetAttribute(rank_sort_kernel,
-                                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                 (int)(RS_COLS * RS_MAX_P * 12)));
-            rs_attr = true;
-        }
+        // once per process (thread-safe static initialisation)
+        static const cudaError_t rs_attr = cudaFuncSetAttribute(
+            rank_sort_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)(RS_COLS * RS_MAX_P * 12));
+        SYMNMF_CUDA_TRY(rs_attr);
         rank_sort_kernel<<<(unsigned)((n + RS_COLS - 1) / RS_COLS), RS_THREADS, rs_smem, s>>>(
             R, T, n, ldr, sign, P, ranks);
     } else if (smem <= RK_SMEM_MAX) {

@@ -314,15 +314,16 @@ gram_tc_kernel(const __grid_constant__ CUtensorMap mapF, const __grid_constant__
 }
 
 static PFN_cuTensorMapEncodeTiled_v12000 gt_encode_fn() {
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    if (fn == nullptr) {
+    // looked up once (thread-safe static initialisation)
+    static const PFN_cuTensorMapEncodeTiled_v12000 fn = []() -> PFN_cuTensorMapEncodeTiled_v12000 {
         void* p = nullptr;
         cudaDriverEntryPointQueryResult q;
         if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
                 cudaSuccess &&
             q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-    }
+            return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+        return nullptr;
+    }();
     return fn;
 }
 
@@ -384,21 +385,16 @@ int launch_gram_tc(const float* ZF, const float* ZL, int64_t n, int64_t n_pad, i
     SYMNMF_CUDA_TRY(cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev));
     const unsigned grid = (unsigned)std::min<int64_t>(nt * (nt + 1) / 2, sms);   // persistent, one CTA per SM
     if (corr) {
-        static bool attr = false;   // once per process
-        if (!attr) {
-            SYMNMF_CUDA_TRY(cudaFuncSetAttribute(gram_tc_kernel<GT_CORR>,
-                                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)gt_smem<GT_CORR>()));
-            attr = true;
-        }
+        // once per process (thread-safe static initialisation)
+        static const cudaError_t attr = cudaFuncSetAttribute(
+            gram_tc_kernel<GT_CORR>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)gt_smem<GT_CORR>());
+        SYMNMF_CUDA_TRY(attr);
         gram_tc_kernel<GT_CORR><<<grid, GT_THREADS, gt_smem<GT_CORR>(), s>>>(mapF, mapL, mapD, mapT, n, (int)Kp,
                                                                  vtiles, scale, err);
     } else {
-        static bool attr = false;
-        if (!attr) {
-            SYMNMF_CUDA_TRY(cudaFuncSetAttribute(gram_tc_kernel<GT_TPDM>,
-                                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)gt_smem<GT_TPDM>()));
-            attr = true;
-        }
+        static const cudaError_t attr = cudaFuncSetAttribute(
+            gram_tc_kernel<GT_TPDM>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)gt_smem<GT_TPDM>());
+        SYMNMF_CUDA_TRY(attr);
         gram_tc_kernel<GT_TPDM><<<grid, GT_THREADS, gt_smem<GT_TPDM>(), s>>>(mapF, mapL, mapD, mapT, n, (int)Kp,
                                                                  vtiles, scale, err);
     }

@@ -423,15 +423,16 @@ int launch_split(const float* Xa, const float* Xb, int64_t ldx, int k, int64_t r
 // host side
 // ----------------------------------------------------------------------------
 static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    if (fn == nullptr) {
+    // looked up once (thread-safe static initialisation)
+    static const PFN_cuTensorMapEncodeTiled_v12000 fn = []() -> PFN_cuTensorMapEncodeTiled_v12000 {
         void* p = nullptr;
         cudaDriverEntryPointQueryResult q;
         if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
                 cudaSuccess &&
             q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-    }
+            return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+        return nullptr;
+    }();
     return fn;
 }
 
@@ -504,12 +505,10 @@ int launch_stream_tc(const TcPlan& p, const float* S, int64_t lds, const float* 
 #define SYMNMF_TC(KP)                                                                         \
     do {                                                                                      \
         auto kern = stream_tc_kernel<KP>;                                                     \
-        static bool attr_set = false; /* once per process: keeps graph capture clean */        \
-        if (!attr_set) {                                                                      \
-            SYMNMF_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, \
-                                                 (int)TcCfg<KP>::SMEM));                      \
-            attr_set = true;                                                                  \
-        }                                                                                     \
+        /* once per process (thread-safe static initialisation): keeps graph capture clean */ \
+        static const cudaError_t attr_rc = cudaFuncSetAttribute(                              \
+            kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)TcCfg<KP>::SMEM);         \
+        SYMNMF_CUDA_TRY(attr_rc);                                                             \
         SYMNMF_CUDA_TRY(launch_pdl(kern, grid, dim3(TC_THREADS), TcCfg<KP>::SMEM, s, mapS, mapX, \
                                    p.n, p.k, p.j0, p.j1, p.jspan, part, err, st, ea, cnt));   \
     } while (0)
