@@ -422,8 +422,9 @@ static int full_pass(FitCtx& c, int mode, int max_evals, bool xt_ready) {
 
 // Replaying the full-batch loop as a CUDA graph is opt-in (SYMNMF_GRAPHS=1):
 // each pass's kernels run for tens of microseconds or more, the loop is not
-// launch-bound, and eager launches measured as fast or faster on B200
-// (n = 5,000: 6.0 ms per 100 iterations eager, 6.4 ms replayed).
+// launch-bound, and eager (programmatically serialised) launches measured as
+// fast or faster on B200 (n = 5,000: 4.85 ms per 100 iterations eager, 5.2 ms
+// replayed).
 static bool use_graphs() {
     static const bool v = [] {   // read once (thread-safe static initialisation)
         const char* e = getenv("SYMNMF_GRAPHS");
