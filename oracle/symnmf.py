@@ -25,6 +25,11 @@ the library stores them, so that trajectories stay comparable.
 
 Where the pages leave a step open, the reading taken is stated at the
 function.  Parity status per function is listed in ``PINS`` at the bottom.
+Three such readings have nothing on the pages to check them against and are
+parity unpinned (both sides implement the written reading, and GPU/oracle
+parity is still tested): the Block-SVRG stall rule (``stall_tol`` on the
+snapshot loss), the seeding of the starting block size (the power of two
+nearest n/10), and the TPDM tail sign.
 """
 from __future__ import annotations
 
@@ -728,4 +733,5 @@ PINS = {
     "cross_sector_mean": "pair loop brute force; planted constant blocks",
     "control_limit": "hand values",
     "rolling_pipeline": "windows equal standalone window runs; planted switch flagged, calm windows not",
+    "stall rule, starting block size, TPDM tail sign": "parity unpinned (readings of silent passages)",
 }
