@@ -145,6 +145,17 @@ def test_spectral_probe_matches_lapack(m, n, k, block):
     assert (oracle.gap_ratio(ev, k) >= 5.0) == (oracle.gap_ratio(ref, k) >= 5.0)
 
 
+def test_spectral_probe_64_eigenvalues_planted_rank_24(m):
+    # the 64-eigenvalue probe on the planted rank-24 workload (24 groups, 10%
+    # boundary instruments, T = 500), at a size LAPACK answers in seconds:
+    # 24 leading eigenvalues and 40 from the noise bulk
+    _, _, S = corr_problem(4000, 500, seed=11, name="corr_n20000_k24")
+    ev = m.spectral_probe(to_dev(S, DEV, pad4=True), 64, block=16, max_iter=60, tol=1e-9)
+    ref = oracle.top_eigenvalues(S, 64)
+    assert np.max(np.abs(ev - ref)) <= 1e-5 * ref[0]
+    assert (oracle.gap_ratio(ev, 24) >= 5.0) == (oracle.gap_ratio(ref, 24) >= 5.0)
+
+
 def test_spectral_probe_low_rank_block_matrix(m):
     # rank 3 < block: the first Krylov block is rank deficient
     S, _ = synth.planted_block_matrix([50, 30, 20], order_seed=2)
