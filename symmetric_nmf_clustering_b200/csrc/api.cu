@@ -525,12 +525,16 @@ static int run_full(FitCtx& c, int max_evals, HostState* hs) {
     const int iters_begin = c.iters;
     const int check = c.P->check_every;
     const int G = std::max(2, (check + 1) / 2 * 2);   // passes per graph: even, so parity returns
+    // with rel_tol = 0 the loop cannot stop early (a non-finite loss turns the
+    // remaining passes into no-ops on the device), so the host reads the state
+    // only after the first pass and after the last
+    const int poll = c.P->rel_tol > 0.0 ? check : std::max(check, max_evals);
     bool graphed = false;
     for (int launched = 0;; ++launched) {
         SYMNMF_TRY(full_pass(c, MODE_FULL, max_evals, true));
         c.cur ^= 1;
         const bool last = t_begin + launched + 1 >= max_evals;
-        if ((launched + 1) % check == 0 || last || launched == 0) {
+        if ((launched + 1) % poll == 0 || last || launched == 0) {
             SYMNMF_TRY(read_state(c.L.st, hs, c.s));
             SYMNMF_TRY(c.tm.harvest());
             if (hs->done) break;
