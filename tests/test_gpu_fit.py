@@ -169,6 +169,21 @@ def test_deterministic_bitwise(m):
     assert np.array_equal(sa["history"], sb["history"])
 
 
+def test_resume_from_returned_h_and_g(m):
+    # a fit resumed from the (H, G) another fit returned continues it exactly:
+    # 40 updates, then 30 more from there, equal 70 updates in one call (the
+    # Gram of the resumed iterate is recomputed in the same fixed order)
+    n, k = 1200, 8
+    _, _, S = corr_problem(n, 150, seed=21)
+    zeros = np.zeros((n, k), np.float32)
+    H70, s70, G70 = _fit(m, S, k, seed=9, G=zeros, max_iters=70, rel_tol=0.0)
+    H40, s40, G40 = _fit(m, S, k, seed=9, G=zeros, max_iters=40, rel_tol=0.0)
+    Hr, sr, Gr = _fit(m, S, k, H0=H40, G=G40, max_iters=30, rel_tol=0.0)
+    assert np.array_equal(Hr, H70) and np.array_equal(Gr, G70)
+    assert np.array_equal(sr["history"], s70["history"][40:])
+    assert np.array_equal(s40["history"], s70["history"][:41])
+
+
 def test_planted_blocks_recovered_on_gpu(m):
     S, planted = synth.planted_block_matrix([60] * 5, order_seed=3)
     Hg, st, _ = _fit(m, S, 5, seed=1003, max_iters=600, rel_tol=0.0)
