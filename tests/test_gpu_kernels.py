@@ -87,6 +87,19 @@ def test_sh_matches_oracle(m, n, k):
     assert rel_fro(Y, ref) <= 2e-6   # regression guard: fp32-class error, far inside the bound
 
 
+def test_sh_partials_staged_in_several_batches(m):
+    # k = 64 at n = 4,000: 9 contraction splits, while the epilogue's shared
+    # memory holds 5 partial tiles, so each tile's partials arrive in two
+    # batches (summed in split order either way)
+    rng = np.random.default_rng(5)
+    A = rng.random((4000, 4000), dtype=np.float32)
+    S = ((A + A.T) * np.float32(0.5)).astype(np.float32)
+    X = synth.uniform_h0(4000, 64, 0.5, seed=3)
+    Y = m.sh(to_dev(S, DEV), to_dev(X, DEV)).cpu().numpy()
+    ref = S.astype(np.float64) @ X.astype(np.float64)
+    assert rel_fro(Y, ref) <= 2e-6
+
+
 # n = 4,100: 561 tiles, several per CTA of the persistent Gram (both TMEM
 # accumulator sets and their barrier phases in use)
 @pytest.mark.parametrize("T,n", [(250, 2000), (250, 1999), (2, 37), (17, 130), (1000, 600), (60, 4100)])
