@@ -30,7 +30,13 @@
 //               memory, stores its lo plane into TMEM lane r, folds the
 //               finished accumulator into fp32 registers every TC_CHUNK
 //               stages and writes the partial row
-//   all warps   in the last split CTA of the tile, the epilogue (epilogue.cuh)
+//   all warps   in the last split CTA of the tile, the epilogue (epilogue.cuh):
+//               the tile's split partials staged in shared memory by
+//               cp.async, then loss terms, gradient, AdaGrad step, Gram
+//
+// Launch: with programmatic stream serialisation; every CTA waits for the
+// previous kernel (griddepcontrol.wait) before it reads anything, and the
+// epilogue CTAs, which no longer hold TMEM, let the next kernel be scheduled.
 #include <cudaTypedefs.h>
 
 #include <cstring>
