@@ -296,7 +296,10 @@ SYMNMF_API int symnmf_ari(const int32_t* a, const int32_t* b, int64_t n, int k, 
  * pairs of instruments in two different stressed groups (group ids from
  * `groups`, n int32 device); an independent fit from the same seeded start
  * ("Factorizing with SymNMF": fixed-seed initialisation, no warm start) with
- * the `fit` parameters; argmax labels into labels[kind] + w*n; ARI against
+ * the `fit` parameters -- or, with warm_start = 1, the workload recipe's
+ * warm start: window 0 from the seeded start and every later window from
+ * the previous window's factor of the same kind, with the AdaGrad
+ * accumulator reset; argmax labels into labels[kind] + w*n; ARI against
  * window w-1 and window w-delta.  Then the 3-sigma control limit of
  * ARI(t-delta, t): mean and sample standard deviation (n-1) over the
  * calibration windows [calib_begin, calib_end) where it is defined,
@@ -316,6 +319,8 @@ typedef struct {
     int64_t calib_end;       /*   default 0, 0 = every window with ARI(t - delta, t) */
     int n_stressed;          /* groups in the cross-sector monitor: 0 = off, else 2..8 */
     int stressed[8];         /* their group ids */
+    int warm_start;          /* 0 (default): every window from the seeded start; 1: window
+                                w > 0 from window w-1's H of the same kind, G reset to 0 */
     symnmf_fit_params fit;   /* per-window fit; default ADAGRAD, 100 iterations, rel_tol 0 */
 } symnmf_rolling_params;
 

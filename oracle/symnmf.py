@@ -645,7 +645,7 @@ def rolling_pipeline(R, T: int, k: int, n_windows: int | None = None, stride: in
                      kinds=("corr", "tpdm"), tail_frac: float = 0.05, tail_sign: int = -1,
                      delta: int = 50, calib=None, groups=None, stressed=(), iters: int = 100,
                      lr: float = 0.1, eps: float = 1e-10, seed: int = 0, only=None,
-                     keep_H: bool = False) -> dict:
+                     keep_H: bool = False, warm_start: bool = False) -> dict:
     """The rolling-window study ([CaS] "The temporal setup", "Tracking
     stability through time", "Stability and break detection").
 
@@ -663,12 +663,20 @@ def rolling_pipeline(R, T: int, k: int, n_windows: int | None = None, stride: in
     ``only`` (a set of window indices) restricts the work to those windows:
     the others keep label -1 and NaN entries, and an ARI needs both of its
     windows.  ``keep_H`` also returns each window's factor (float32).
+
+    ``warm_start`` takes the workload recipe's reading instead ("warm-started
+    100-iteration fit", AdaGrad accumulator reset per window): the first
+    window starts from the seeded start, every later window from the
+    previous window's factor of the same kind (rounded to float32 as the
+    library stores it), with G = 0.  It needs every window, so not ``only``.
     """
     R = np.asarray(R)
     days, n = R.shape
     W = (days - T) // stride + 1 if n_windows is None else n_windows
     if W < 1 or (W - 1) * stride + T > days:
         raise ValueError("windows do not fit in the stream")
+    if warm_start and only is not None:
+        raise ValueError("a warm start needs every window")
     todo = set(range(W)) if only is None else {int(w) for w in only if 0 <= w < W}
     out = {}
     for kind in kinds:
@@ -677,6 +685,7 @@ def rolling_pipeline(R, T: int, k: int, n_windows: int | None = None, stride: in
         cross = np.full(W, np.nan)
         smax = np.full(W, np.nan)
         Hs = {}
+        H_prev = None
         for w in sorted(todo):
             Rw = R[w * stride: w * stride + T]
             if kind == "corr":
@@ -687,8 +696,12 @@ def rolling_pipeline(R, T: int, k: int, n_windows: int | None = None, stride: in
             if groups is not None and len(stressed) > 1:
                 cross[w] = cross_sector_mean(S, groups, stressed)
             s_sum, sq, _ = stats(S)
-            H0 = scale_matched_init(s_sum, n, k, seed)
+            if warm_start and H_prev is not None:
+                H0 = H_prev
+            else:
+                H0 = scale_matched_init(s_sum, n, k, seed)
             r = fit_adagrad(S, k, H0, lr=lr, eps=eps, max_iters=iters, rel_tol=0.0, S_sqnorm=sq)
+            H_prev = _f32(r.H)
             lab[w] = labels(_f32(r.H))
             loss[w] = r.loss
             if keep_H:

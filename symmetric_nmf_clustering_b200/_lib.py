@@ -90,6 +90,7 @@ class RollingParams(C.Structure):
         ("calib_end", C.c_int64),
         ("n_stressed", C.c_int),
         ("stressed", C.c_int * 8),
+        ("warm_start", C.c_int),
         ("fit", FitParams),
     ]
 

@@ -363,7 +363,12 @@ static int run_chain(const StudyArgs& A, ChainRun& r) {
         }
         SYMNMF_CUDA_TRY(cudaEventRecord(ev_fit.a, r.s));
         symnmf_fit_stats st;
-        SYMNMF_TRY(symnmf_fit(r.S, n, r.lds, p.k, &p.fit, L.H, &st, L.shared, L.shared_bytes, r.s));
+        // every window from the seeded start, or with a warm start from the
+        // chain's previous window (step 1); the AdaGrad accumulator starts at 0
+        symnmf_fit_params fp = p.fit;
+        fp.init = (p.warm_start && w > r.first) ? SYMNMF_INIT_USER : SYMNMF_INIT_SEEDED;
+        fp.G_inout = nullptr;
+        SYMNMF_TRY(symnmf_fit(r.S, n, r.lds, p.k, &fp, L.H, &st, L.shared, L.shared_bytes, r.s));
         count();
         int32_t* lab = A.out->labels[c] + (size_t)w * (size_t)n;
         SYMNMF_TRY(symnmf_labels(L.H, n, p.k, lab, r.s));
@@ -483,7 +488,8 @@ static int rolling_impl(const float* R, int64_t days, int64_t n, int64_t ldr, co
     {
         const int tries[3][2] = {{2, 2 * nk}, {1, nk}, {1, 1}};
         bool fit = false;
-        for (int t = rolling_serial() ? 2 : 0; t < 3 && !fit; ++t) {
+        // a warm start needs each kind's windows in order on one chain
+        for (int t = rolling_serial() ? 2 : (p.warm_start ? 1 : 0); t < 3 && !fit; ++t) {
             if (tries[t][1] > RL_MAX_CHAINS) continue;
             Arena a;
             a.base = static_cast<char*>(ws);
@@ -666,6 +672,7 @@ void symnmf_rolling_params_default(symnmf_rolling_params* p) {
     p->calib_begin = 0;
     p->calib_end = 0;
     p->n_stressed = 0;
+    p->warm_start = 0;
     symnmf_fit_params_default(&p->fit);
     p->fit.max_iters = 100;
     p->fit.rel_tol = 0.0;
@@ -694,6 +701,10 @@ int symnmf_rolling(const float* R, int64_t days, int64_t n, int64_t ldr, const i
     }
     if (p.n_stressed != 0 && (p.n_stressed < 2 || p.n_stressed > RL_MAX_STRESSED || groups == nullptr)) {
         set_error("n_stressed = %d: 0, or 2..%d with a groups array", p.n_stressed, RL_MAX_STRESSED);
+        return SYMNMF_ERR_INVALID_ARG;
+    }
+    if (p.warm_start != 0 && p.warm_start != 1) {
+        set_error("warm_start = %d must be 0 or 1", p.warm_start);
         return SYMNMF_ERR_INVALID_ARG;
     }
     if (p.k < 1 || p.k > KMAX || p.k > n) {

@@ -222,3 +222,34 @@ def test_rolling_error_in_the_second_chain_is_reported(m):
     # the library is still usable afterwards
     ok = m.rolling(R, window=60, k=6, kinds=3, delta=5, n_windows=3, fit=dict(max_iters=5))
     assert ok["n_windows"] == 3
+
+
+def test_rolling_warm_start_equals_chained_fits(m):
+    # warm_start = 1: window 0 from the seeded start, window w from window
+    # w-1's factor of the same kind, G reset -- the same as chaining the
+    # public fit by hand on the same builders, bit for bit
+    import torch
+    st = _stream_small()
+    R = to_dev(st.R, DEV, pad4=True)
+    T, k, W, iters, seed = 60, 6, 5, 40, 3
+    got = m.rolling(R, window=T, k=k, n_windows=W, delta=2, tail_frac=0.05, tail_sign=-1,
+                    warm_start=1, fit=dict(max_iters=iters, seed=seed))
+    for kind in ("corr", "tpdm"):
+        H = None
+        for w in range(W):
+            Rw = R[w: w + T]
+            S = m.build_corr(Rw) if kind == "corr" else m.build_tpdm(Rw, 0.05, -1)
+            if H is None:
+                H, stt = m.fit(S, k, seed=seed, max_iters=iters, rel_tol=0.0)
+            else:
+                H, stt = m.fit(S, k, H0=H, max_iters=iters, rel_tol=0.0)
+            assert torch.equal(m.labels(H), got[kind]["labels"][w]), (kind, w)
+            assert stt["loss"] == got[kind]["loss"][w], (kind, w)
+    # Parity with the oracle's warm-started pipeline is not compared window by
+    # window: each window starts from its own side's previous result, which
+    # differs at the fit's 1e-3 level, and the difference compounds over the
+    # windows of an unconverged fit.  The oracle's warm start is pinned against
+    # its own chained fits, and each fit's parity is tested on its own.
+    from symmetric_nmf_clustering_b200 import _lib as L
+    with pytest.raises(L.SymNMFError):
+        m.rolling(R, window=T, k=k, n_windows=2, warm_start=2)

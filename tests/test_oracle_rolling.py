@@ -88,6 +88,33 @@ def test_windows_equal_standalone_runs():
         oracle.ari(out["corr"]["labels"][0], out["corr"]["labels"][2]), abs=1e-15)
 
 
+def test_warm_started_windows_equal_chained_fits():
+    # the recipe's warm start: window 0 from the seeded start, window w from
+    # window w-1's factor (float32), G reset; both kinds chain separately
+    st = _small_stream(seed=2)
+    T, k, W = 40, 4, 4
+    out = oracle.rolling_pipeline(st.R, T, k, n_windows=W, stride=3, delta=2, iters=25,
+                                  warm_start=True, keep_H=True)
+    for kind in ("corr", "tpdm"):
+        H = None
+        for w in range(W):
+            Rw = st.R[3 * w: 3 * w + T]
+            S = (oracle.corr_abs(Rw) if kind == "corr" else oracle.tpdm(Rw, 0.05, -1)).astype(np.float32)
+            s_sum, sq, _ = oracle.stats(S)
+            H0 = oracle.scale_matched_init(s_sum, 120, k, 0) if H is None else H
+            r = oracle.fit_adagrad(S, k, H0, max_iters=25)
+            H = r.H.astype(np.float32).astype(np.float64)
+            assert np.array_equal(out[kind]["H"][w], H), (kind, w)
+            assert out[kind]["loss"][w] == r.loss
+    # the first window is the independent fit's; a later one starts elsewhere
+    ind = oracle.rolling_pipeline(st.R, T, k, n_windows=W, stride=3, delta=2, iters=25,
+                                  keep_H=True)
+    assert np.array_equal(ind["corr"]["H"][0], out["corr"]["H"][0])
+    assert not np.array_equal(ind["corr"]["H"][3], out["corr"]["H"][3])
+    with pytest.raises(ValueError):
+        oracle.rolling_pipeline(st.R, T, k, n_windows=W, warm_start=True, only=[1])
+
+
 def test_planted_switch_is_flagged_and_calm_windows_are_not():
     # low noise and no shock: a window's labels are the planted membership of
     # the days it holds, so ARI(t - delta, t) is 1 unless the two windows
