@@ -207,9 +207,11 @@ SYMNMF_API int symnmf_sh(const float* S, int64_t n, int64_t lds, const float* X,
  * and pick k at the clearest gap; "Why this solver": gamma_{k+1}).
  * Writes the n_eig algebraically largest Ritz values, descending, into the
  * host array eigvals_host.  block (1..64) vectors per step, at most max_iter
- * block steps (basis <= block*max_iter <= n); stops when every wanted Ritz
- * residual is <= tol * |lambda_1|.  Start block from the splitmix64 counter
- * stream of `seed`.  Synchronises `stream`.
+ * block steps (basis <= block*max_iter <= n); stops when no wanted Ritz value
+ * moved by more than tol * |theta_1| between two consecutive block steps.
+ * The next block's S pass is issued before the host's Rayleigh-Ritz step (a
+ * converging step leaves one pass unused).  Start block from the splitmix64
+ * counter stream of `seed`.  Synchronises `stream`.
  */
 SYMNMF_API int symnmf_spectral_probe(const float* S, int64_t n, int64_t lds, int n_eig,
                           int block, int max_iter, double tol, uint64_t seed,
