@@ -293,7 +293,8 @@ SYMNMF_API int symnmf_ari(const int32_t* a, const int32_t* b, int64_t n, int k, 
  * [w*stride, w*stride + window) of the returns stream R (days x n fp32,
  * row = day, leading dimension ldr, device).  For every window and every
  * kind of dependence matrix selected in `kinds`, in this order: build S
- * (symnmf_build_corr / symnmf_build_tpdm) into the caller's n x n buffer;
+ * (symnmf_build_corr / symnmf_build_tpdm) into an n x n buffer (the caller's
+ * for the first chain, a chain's own matrix in the workspace otherwise);
  * the cross-sector monitor, when n_stressed >= 2: the mean of S_ij over the
  * pairs of instruments in two different stressed groups (group ids from
  * `groups`, n int32 device); an independent fit from the same seeded start
