@@ -466,19 +466,26 @@ def run_ours(args):
         del ws_corr
 
     # --- the other rows of the path, each timed once on this GPU (CUDA events)
+    # (a failure in a secondary row is reported in the line, not fatal to it)
     rows = None
     if not args.no_rows:
-        rows = measure_rows(m, torch, dev, S, H0, lab, n, k, T, rank, args.workload)
-        rows["roofline"], tf32_peak = row_rooflines(rows, n, k, T, peak)
-        rows["roofline"]["corr_build"] = {
-            "bound": "tensor", "tf32_TFs": 3.0 * n * n * T / (build_ms / 1e3) / 1e12,
-            "peak_TFs": tf32_peak, "frac": 3.0 * n * n * T / (build_ms / 1e3) / 1e12 / tf32_peak,
-            "flops": "3 n^2 T (exact TF32 split, upper triangle of tiles)"}
+        try:
+            rows = measure_rows(m, torch, dev, S, H0, lab, n, k, T, rank, args.workload)
+            rows["roofline"], tf32_peak = row_rooflines(rows, n, k, T, peak)
+            rows["roofline"]["corr_build"] = {
+                "bound": "tensor", "tf32_TFs": 3.0 * n * n * T / (build_ms / 1e3) / 1e12,
+                "peak_TFs": tf32_peak, "frac": 3.0 * n * n * T / (build_ms / 1e3) / 1e12 / tf32_peak,
+                "flops": "3 n^2 T (exact TF32 split, upper triangle of tiles)"}
+        except Exception as exc:
+            rows = {"error": f"{type(exc).__name__}: {exc}"}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        res = oracle_sample(args.workload, 0, 20, 2)
-        cpu = {k2: res[k2] for k2 in ("value", "unit", "cores", "kind", "sample")}
+        try:
+            res = oracle_sample(args.workload, 0, 20, 2)
+            cpu = {k2: res[k2] for k2 in ("value", "unit", "cores", "kind", "sample")}
+        except Exception as exc:
+            cpu = {"error": f"{type(exc).__name__}: {exc}"}
 
     if world > 1:
         dist.barrier()
