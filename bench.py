@@ -44,9 +44,9 @@ UNIT = "iterations/s"
 SAMPLE_ROWS = 8192   # oracle sample: leading principal r x r block of the same window
 # DRAM traffic of one stream_tc_kernel<24> launch from ncu (dram__bytes_read.sum +
 # dram__bytes_write.sum): 1.619 GB + 13.8 MB at n = 20,000 against 1.602 GB of
-# algorithmic bytes (profiles/stream_tc_kernel_n20000_k24.md); the full-size
-# launch (40 GB S, too large to capture) is reported as the same ratio times
-# its algorithmic bytes.  Retake the capture whenever the kernel changes.
+# algorithmic bytes; the full-size launch (40 GB S, too large to capture) is
+# reported as the same ratio times its algorithmic bytes.  Retake the capture
+# whenever the kernel changes.
 STREAM_TRAFFIC_RATIO = (1.618906e9 + 13.768704e6) / (4.0 * 20000 ** 2 + 4.0 * 20000 * 24)
 STREAM_TRAFFIC_SOURCE = ("ncu dram__bytes_read.sum + dram__bytes_write.sum of one launch at "
                          "n = 20,000, k = 24, scaled to this launch by algorithmic bytes")
@@ -173,6 +173,9 @@ def oracle_sample(name: str, seed: int, steps: int, warmup: int):
                    f"block of the n={n} |corr| window (seed {seed}); per-iteration time scaled "
                    f"by (n/r)^2 = {(n / r) ** 2:.1f}"),
         "sample_seconds": dt,
+        "sample_block": r,
+        "sample_iters": steps,
+        "scale_to_full": (n / r) ** 2,
     }
 
 
@@ -344,6 +347,10 @@ def run_reference(args):
         "impl": "reference",
         "cpu_baseline": {k2: res[k2] for k2 in ("value", "unit", "cores", "kind", "sample")},
         "e2e": {"value": res["value"], "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        # what was actually timed: ms_per_step above is this sample extrapolated to the full n
+        "measured_sample": {"seconds": res["sample_seconds"], "iterations": res["sample_iters"],
+                            "block_rows": res["sample_block"], "scale_to_full_n": res["scale_to_full"],
+                            "ms_per_sample_iteration": 1000.0 * res["sample_seconds"] / max(res["sample_iters"], 1)},
     }
     print(json.dumps(line), flush=True)
     return 0

@@ -376,9 +376,11 @@ SYMNMF_API int symnmf_rolling(const float* R, int64_t days, int64_t n, int64_t l
  * TF32 split of X and an error word) lives in a 4 MiB file-scope device array
  * that every GPU loading the library holds until exit.  Limit:
  * 2 * roundup(k, 8) * roundup(n, 32) + 64 <= 1,048,576 floats (for k = 24,
- * n <= 21,824); larger sizes return SYMNMF_ERR_INVALID_ARG.  The first call on
- * a device looks up the array's device address (cudaGetSymbolAddress) with
- * that device current; make that first call before any stream capture.
+ * n <= 21,824); larger sizes return SYMNMF_ERR_INVALID_ARG.  Every call looks
+ * up the array's device address (cudaGetSymbolAddress) with the calling
+ * device current, so the address stays right after cudaDeviceReset or under
+ * another context; the first call on a device also loads the library's
+ * module there, so make that first call before any stream capture.
  * Every call shares the one array and it keeps the last call's contents:
  * calls that overlap on the GPU (on different streams, or from several host
  * threads without ordering) race on it.  S, X, Y as for symnmf_sh.

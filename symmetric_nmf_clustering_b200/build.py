@@ -47,15 +47,26 @@ def _deps_mtime() -> float:
     return max(os.path.getmtime(f) for f in files)
 
 
+def _headers_mtime() -> float:
+    files = [os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith((".h", ".cuh"))]
+    files.append(os.path.join(INCLUDE, "symnmf.h"))
+    return max(os.path.getmtime(f) for f in files)
+
+
 def build(force: bool = False, verbose: bool = False) -> str:
     """Compile every source and link libsymnmf.so; returns the library path."""
     if not force and os.path.exists(LIB) and os.path.getmtime(LIB) >= _deps_mtime():
         return LIB
     nvcc = _nvcc()
     os.makedirs(BUILD, exist_ok=True)
+    hdr = _headers_mtime()
 
     def compile_one(src):
         obj = os.path.join(BUILD, os.path.basename(src) + ".o")
+        # an object newer than its source and every header is up to date
+        if (not force and os.path.exists(obj)
+                and os.path.getmtime(obj) >= max(os.path.getmtime(src), hdr)):
+            return obj
         cmd = [nvcc, *ARCH, *NVCC_FLAGS, "-c", src, "-o", obj]
         if src.endswith(".cpp"):
             cmd = [nvcc, *NVCC_FLAGS, "-x", "c++", "-c", src, "-o", obj]

@@ -7,8 +7,6 @@
 // would fragment it or break its budget), or a latency-critical loop that
 // cannot take cudaMalloc's implicit device-wide synchronisation.  For them
 // this variant keeps its scratch in a fixed file-scope device array instead.
-#include <mutex>
-
 #include "common.cuh"
 
 namespace symnmf {
@@ -20,31 +18,20 @@ constexpr size_t kNoAllocErrFloats = 64;  // error word slot, kept 256-byte alig
 static __device__ __align__(256) float g_noalloc_scratch[kNoAllocScratchFloats];
 
 // Host code cannot use g_noalloc_scratch's name as a device address: it is a
-// host-side stand-in.  The device address is looked up once per device, with
-// that device current, and cached.
-constexpr int kMaxDevices = 128;
-static std::mutex g_noalloc_mu;
-static float* g_noalloc_ptr[kMaxDevices] = {};
-
+// host-side stand-in.  The device address belongs to the context the module
+// was loaded into, so it is looked up on every call, with the calling device
+// current: after cudaDeviceReset, or under another context on the same
+// device, a cached address would point at memory that is no longer the
+// array.  The lookup is a host-side table read once the module is loaded,
+// negligible next to a pass over S.
 static int noalloc_scratch(float** out) {
-    int dev = 0;
-    SYMNMF_CUDA_TRY(cudaGetDevice(&dev));
-    if (dev < 0 || dev >= kMaxDevices) {
-        set_error("device ordinal %d out of range for the static scratch table", dev);
-        return SYMNMF_ERR_NOT_SUPPORTED;
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) {
+        set_error("cudaGetSymbolAddress of the static scratch failed: %s", cudaGetErrorString(e));
+        return SYMNMF_ERR_CUDA;
     }
-    std::lock_guard<std::mutex> lock(g_noalloc_mu);
-    if (g_noalloc_ptr[dev] == nullptr) {
-        void* p = nullptr;
-        const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-        if (e != cudaSuccess) {
-            set_error("cudaGetSymbolAddress of the static scratch failed: %s",
-                      cudaGetErrorString(e));
-            return SYMNMF_ERR_CUDA;
-        }
-        g_noalloc_ptr[dev] = static_cast<float*>(p);
-    }
-    *out = g_noalloc_ptr[dev];
+    *out = static_cast<float*>(p);
     return SYMNMF_OK;
 }
 
@@ -64,6 +51,19 @@ extern "C" int symnmf_sh_noalloc(const float* S, int64_t n, int64_t lds, const f
                   (long long)lds);
         return SYMNMF_ERR_INVALID_ARG;
     }
+    // n alone bounds the scratch (one split row per instrument): reject any n
+    // the array cannot hold before the size product below is formed, so that
+    // product cannot wrap
+    if (n > (int64_t)kNoAllocScratchFloats) {
+        set_error("symnmf_sh_noalloc: n = %lld exceeds the static scratch of %zu floats; "
+                  "use symnmf_sh with a workspace",
+                  (long long)n, kNoAllocScratchFloats);
+        return SYMNMF_ERR_INVALID_ARG;
+    }
+    if (lds > (int64_t(1) << 62) / n) {
+        set_error("n * lds overflows");
+        return SYMNMF_ERR_INVALID_ARG;
+    }
     if (S == nullptr || (reinterpret_cast<uintptr_t>(S) & 15u) != 0) {
         set_error("S must be a non-null 16-byte aligned device pointer");
         return SYMNMF_ERR_INVALID_ARG;
@@ -72,8 +72,9 @@ extern "C" int symnmf_sh_noalloc(const float* S, int64_t n, int64_t lds, const f
         set_error("k = %d must be in [1, %d]", k, KMAX);
         return SYMNMF_ERR_INVALID_ARG;
     }
-    if (X == nullptr || Y == nullptr) {
-        set_error("X and Y must be device pointers");
+    if (X == nullptr || Y == nullptr || (reinterpret_cast<uintptr_t>(X) & 3u) != 0 ||
+        (reinterpret_cast<uintptr_t>(Y) & 3u) != 0) {
+        set_error("X and Y must be non-null 4-byte aligned device pointers");
         return SYMNMF_ERR_INVALID_ARG;
     }
     const size_t need = noalloc_floats_needed(n, k);

@@ -15,7 +15,6 @@ import ctypes as C
 import numpy as np
 import pytest
 
-pytestmark = pytest.mark.gpu
 DEV = "cuda:0"
 
 
@@ -25,6 +24,7 @@ def _rel(a, b):
     return float(np.linalg.norm(a - b) / np.linalg.norm(b))
 
 
+@pytest.mark.gpu
 def test_noalloc_matches_workspace_entry_point_on_two_calls():
     import torch
     from symmetric_nmf_clustering_b200 import build
@@ -56,6 +56,7 @@ def test_noalloc_matches_workspace_entry_point_on_two_calls():
 
 
 def test_noalloc_rejects_sizes_beyond_its_scratch():
+    # argument checks only (no device call): runs without a GPU as well
     from symmetric_nmf_clustering_b200 import build
     build.build()
     from symmetric_nmf_clustering_b200 import _lib
@@ -64,3 +65,11 @@ def test_noalloc_rejects_sizes_beyond_its_scratch():
     # k = 24: 2 * 24 * roundup(n, 32) + 64 <= 1,048,576 allows n <= 21,824
     assert lib.symnmf_sh_noalloc(fake, 21825, 21828, fake, 24, fake, None) == _lib.SYMNMF_ERR_INVALID_ARG
     assert b"static scratch" in lib.symnmf_last_error()
+    # a size whose scratch product would wrap around 2^64 (2 * 8 * 2^60) is
+    # rejected on n alone, before the product is formed
+    big = 1 << 60
+    assert lib.symnmf_sh_noalloc(fake, big, big, fake, 8, fake, None) == _lib.SYMNMF_ERR_INVALID_ARG
+    # n * lds overflow, and misaligned X or Y, as for symnmf_sh
+    assert lib.symnmf_sh_noalloc(fake, 1000, 1 << 62, fake, 8, fake, None) == _lib.SYMNMF_ERR_INVALID_ARG
+    assert lib.symnmf_sh_noalloc(fake, 1000, 1000, fake + 2, 8, fake, None) == _lib.SYMNMF_ERR_INVALID_ARG
+    assert lib.symnmf_sh_noalloc(fake, 1000, 1000, fake, 8, fake + 1, None) == _lib.SYMNMF_ERR_INVALID_ARG
