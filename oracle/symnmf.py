@@ -734,7 +734,12 @@ PINS = {
     "gradient": "central finite differences of the brute-force loss",
     "adagrad_step": "first-step closed form; H >= 0; G non-decreasing",
     "fit_adagrad": "k=1 rank-one recovery; planted blocks ARI = 1; permutation equivariance",
-    "fit_block_svrg": "b = n equals full batch; block unbiasedness identity; H >= 0",
+    "fit_block_svrg": ("b = n equals full batch; block unbiasedness identity; H >= 0; a two-block "
+                       "epoch equals hand-applied steps with the snapshot frozen at the epoch start "
+                       "(ragged block, masked full products); three epochs equal hand-applied epochs "
+                       "in the epoch_permutation order, and differ in the reversed order; the stall "
+                       "rule replayed on consecutive snapshot losses; planted noise-free blocks "
+                       "recovered with ARI = 1 by b < n, growth off, from listed starts"),
     "epoch_permutation": "is a permutation; uniform over orders for small m",
     "top_eigenvalues": "block-of-ones closed form; sum = trace",
     "gap_ratio": "hand values",

@@ -198,3 +198,119 @@ def test_adaptgrow_selects_solver_from_gap():
     flat = np.array([10.0, 9.0, 8.0, 7.0, 6.0, 5.5])
     r2 = oracle.adaptgrow(S.astype(np.float64), 3, max_iters=2, eigvals=flat, block_rows=16)
     assert r2.gamma == pytest.approx(7.0 / 6.0) and r2.solver_used == 1
+
+
+# ------------------------------------------------- Block-SVRG epoch loop, pinned
+# [CaS] "Factorizing with SymNMF": block-sampled gradient corrected with the
+# SVRG control variate, same AdaGrad update; [SMI] AdaptGrow sketch.  The
+# pins below fix the loop around block_svrg_grad: which snapshot the blocks
+# see, which rows a block holds, the visiting order, and the stall rule.
+
+def _blocks_by_hand(n, b):
+    """Row index sets of the contiguous blocks [jb, min((j+1)b, n)), built
+    from index arrays rather than slices."""
+    m = -(-n // b)
+    return [np.arange(j * b, min((j + 1) * b, n)) for j in range(m)]
+
+
+def _epoch_by_hand(S, H, G, b, order, lr=0.1, eps=1e-10):
+    """One Block-SVRG epoch applied step by step: snapshot H~ and P~ = S H~
+    frozen at the epoch start, then one AdaGrad step per block in `order`,
+    each with the corrected block gradient.  The block product is formed as
+    a full product against the difference masked to the block's rows."""
+    n = S.shape[0]
+    blocks = _blocks_by_hand(n, b)
+    m = len(blocks)
+    H_snap = H.copy()
+    P_snap = np.einsum("ij,jc->ic", S, H_snap)
+    for j in order:
+        mask = np.zeros((n, 1))
+        mask[blocks[j]] = 1.0
+        est = P_snap + m * (S @ ((H - H_snap) * mask))
+        g = 4.0 * (H @ (H.T @ H) - est)
+        H, G = oracle.adagrad_step(H, G, g, lr, eps)
+    return H, G
+
+
+def test_svrg_two_block_epoch_equals_hand_applied_steps():
+    # n = 37, b = 20: a full block and a ragged one (m = 2)
+    S, H0 = _small_problem(37, 3, 21)
+    for seed in (0, 1, 2, 5):
+        order = oracle.epoch_permutation(2, seed, 0)
+        r = oracle.fit_block_svrg(S, 3, H0, max_epochs=1, block_rows=20, grow=False,
+                                  seed=seed, mirror=False)
+        H1, G1 = _epoch_by_hand(S, H0.copy(), np.zeros_like(H0), 20, order)
+        np.testing.assert_allclose(r.H, H1, rtol=1e-12, atol=1e-15)
+        np.testing.assert_allclose(r.G, G1, rtol=1e-12, atol=1e-15)
+        assert r.epochs == 1 and r.iters == 0
+        # the two evaluations are the snapshot losses of H0 and of the epoch's result
+        assert len(r.history) == 2
+        assert abs(r.history[0] - _brute_loss(S, H0)) <= 1e-12 * _brute_loss(S, H0)
+        assert abs(r.history[1] - _brute_loss(S, H1)) <= 1e-12 * _brute_loss(S, H0)
+
+
+def test_svrg_visits_blocks_in_the_epoch_permutation_each_once():
+    # n = 50, b = 17: blocks of 17, 17, 16; three epochs, every order distinct
+    S, H0 = _small_problem(50, 4, 22)
+    seed = 7
+    orders = [oracle.epoch_permutation(3, seed, e) for e in range(3)]
+    r = oracle.fit_block_svrg(S, 4, H0, max_epochs=3, block_rows=17, grow=False, seed=seed,
+                              mirror=False)
+    H, G = H0.copy(), np.zeros_like(H0)
+    for o in orders:
+        assert sorted(o) == [0, 1, 2]
+        H, G = _epoch_by_hand(S, H, G, 17, o)
+    np.testing.assert_allclose(r.H, H, rtol=1e-11, atol=1e-14)
+    # the order matters: the same epochs with every order reversed end elsewhere
+    Hx, Gx = H0.copy(), np.zeros_like(H0)
+    for o in orders:
+        Hx, Gx = _epoch_by_hand(S, Hx, Gx, 17, o[::-1])
+    assert np.abs(Hx - r.H).max() > 1e-6
+
+
+def test_svrg_stall_rule_doubles_on_consecutive_snapshots():
+    # the block doubles after the epoch whose snapshot loss fell by less than
+    # stall_tol relative to the previous snapshot (not the first one)
+    S, H0 = _small_problem(96, 4, 23)
+    seed, b0, stall = 3, 12, 0.02
+    E = 8
+    r = oracle.fit_block_svrg(S, 4, H0, max_epochs=E, block_rows=b0, grow=True,
+                              stall_tol=stall, seed=seed, mirror=False)
+    # replay: block schedule from the replay's own snapshot losses
+    H, G, b = H0.copy(), np.zeros_like(H0), b0
+    losses, schedule = [], []
+    for e in range(E + 1):
+        L = _brute_loss(S, H)
+        if losses and (losses[-1] - L) / losses[-1] < stall:
+            b = min(2 * b, 96)
+        losses.append(L)
+        if e == E:
+            break
+        schedule.append(b)
+        if b >= 96:
+            g = oracle.gradient(H, S @ H)
+            H, G = oracle.adagrad_step(H, G, g, 0.1, 1e-10)
+        else:
+            H, G = _epoch_by_hand(S, H, G, b, oracle.epoch_permutation(-(-96 // b), seed, e))
+    np.testing.assert_allclose(r.history, losses, rtol=1e-10)
+    np.testing.assert_allclose(r.H, H, rtol=1e-10, atol=1e-13)
+    assert r.block_final == b
+    # the schedule grew at some epochs and not at others, so the rule was exercised
+    assert b0 < b and len(set(schedule)) >= 3
+
+
+@pytest.mark.parametrize("sizes,b,seed", [([60] * 5, 64, s) for s in range(6)]
+                         + [([40] * 6, 48, s) for s in (0, 3, 7)]
+                         + [([50] * 8, 64, s) for s in (1, 2, 4)])
+def test_svrg_recovers_planted_blocks_with_growth_off(sizes, b, seed):
+    # noise-free planted blocks, b < n and growth off: the sampled solver alone
+    # reaches the planted factorisation (ARI = 1, loss ~ 0) from these starts
+    S, planted = synth.planted_block_matrix(sizes, order_seed=seed)
+    n, k = S.shape[0], len(sizes)
+    s_sum, sq, _ = oracle.stats(S)
+    H0 = oracle.scale_matched_init(s_sum, n, k, 1000 + seed)
+    r = oracle.fit_block_svrg(S, k, H0, max_epochs=300, block_rows=b, grow=False, seed=seed,
+                              S_sqnorm=sq)
+    assert r.block_final == b and r.epochs == 300
+    assert oracle.ari(oracle.labels(r.H), planted) == 1.0
+    assert r.loss < 1e-9 * sq
