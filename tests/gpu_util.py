@@ -33,3 +33,27 @@ def to_dev(x, device, pad4=False):
         buf[:, :x.shape[1]] = torch.from_numpy(x).to(device)
         return buf[:, :x.shape[1]]
     return torch.from_numpy(x).to(device)
+
+
+def assert_labels_differ_only_on_near_ties(lab_gpu, lab_oracle, H_gpu, H_oracle, tol=1e-3):
+    """Labels of two factors that agree to the fit's H tolerance.
+
+    Every row whose labels differ must be a near-tie that the H difference
+    explains: the oracle's top-two margin there is at most twice that row's
+    largest deviation |H_gpu - H_oracle| (a smaller margin cannot flip the
+    argmax), and at most tol * max|H| (the H tolerance).  Returns and prints
+    the number of differing rows, so a run shows how many there were.
+    """
+    lab_gpu = np.asarray(lab_gpu)
+    lab_oracle = np.asarray(lab_oracle)
+    H_gpu = np.asarray(H_gpu, dtype=np.float64)
+    H_oracle = np.asarray(H_oracle, dtype=np.float64)
+    diff = lab_gpu != lab_oracle
+    srt = np.sort(H_oracle, axis=1)
+    margin = srt[:, -1] - srt[:, -2] if H_oracle.shape[1] > 1 else np.full(len(srt), np.inf)
+    dev = np.abs(H_gpu - H_oracle).max(axis=1)
+    bad = diff & ((margin > 2.0 * dev) | (margin > tol * np.abs(H_oracle).max()))
+    print(f"labels: {int(diff.sum())} of {diff.size} rows differ, all on near-ties"
+          if not bad.any() else f"labels: {int(bad.sum())} rows differ on clear margins")
+    assert not bad.any(), np.flatnonzero(bad)[:10]
+    return int(diff.sum())

@@ -11,7 +11,10 @@ top-two margin of H exceeds 1e-3 max|H| (the fit's H tolerance); loss within
 perturbation of e_S moves f = ||S - H H^T||^2 to first order; cross-sector
 mean within e_S plus 1e-6 relative; an ARI bit-equal whenever both of its
 windows' label vectors are equal; the 3-sigma limit and flags equal when
-every calibration ARI is.
+every calibration ARI is.  Those cross-side checks run only where labels
+agree, so each test also asserts how many of them ran, and checks in every
+window that the library's ARI series, limit and flags are the oracle's
+functions of the library's own labels.
 """
 import numpy as np
 import pytest
@@ -89,6 +92,27 @@ def _compare_windows(got, ref, k, windows, H, kind):
     return equal
 
 
+def _check_series_from_own_labels(g, k, delta, calib, kind):
+    """The library's ARI(t-1, t), ARI(t-delta, t), 3-sigma limit and flags are
+    the oracle's ARI and control limit applied to the library's own labels,
+    in every window (no window is skipped, whatever the labels are)."""
+    lab = g["labels"].cpu().numpy()
+    W = lab.shape[0]
+    for w in range(1, W):
+        want = oracle.ari_from_table(oracle.contingency(lab[w - 1], lab[w], k, k))
+        assert g["ari_prev"][w] == want, (kind, w)
+        if w >= delta:
+            want = oracle.ari_from_table(oracle.contingency(lab[w - delta], lab[w], k, k))
+            assert g["ari_delta"][w] == want, (kind, w)
+    cw = range(max(calib[0], delta), min(calib[1], W))
+    mu, sd, lim = oracle.control_limit(np.asarray(g["ari_delta"], dtype=np.float64), cw)
+    assert g["mean"] == pytest.approx(mu, rel=1e-12, abs=1e-15), kind
+    assert g["std"] == pytest.approx(sd, rel=1e-12, abs=1e-15), kind
+    assert g["limit"] == pytest.approx(lim, rel=1e-12, abs=1e-15), kind
+    flags = np.array([np.isfinite(x) and x < g["limit"] for x in g["ari_delta"]], dtype=bool)
+    assert np.array_equal(np.asarray(g["flags"], dtype=bool), flags), kind
+
+
 def _stream_small():
     return synth.rolling_stream(seed=5, n=360, g=6, days=90, sigma=1.0, boundary=0.1,
                                 switch_day=45, switch_frac=0.1, shock_days=(5, 9),
@@ -111,15 +135,27 @@ def test_rolling_parity_small(m):
     for kind in ("corr", "tpdm"):
         g, r = got[kind], ref[kind]
         equal = _compare_windows(g, r, k, range(W), r["H"], kind)
+        _check_series_from_own_labels(g, k, delta, (10, 20), kind)
+        n_prev = n_delta = 0
         for w in range(1, W):
             if w in equal and w - 1 in equal:
                 assert g["ari_prev"][w] == r["ari_prev"][w], (kind, w)
+                n_prev += 1
             if w >= delta and w in equal and w - delta in equal:
                 assert g["ari_delta"][w] == r["ari_delta"][w], (kind, w)
+                n_delta += 1
         assert np.isnan(g["ari_prev"][0]) and np.all(np.isnan(g["ari_delta"][:delta]))
-        if all(w in equal and w - delta in equal for w in range(10, 20)):
+        calib_equal = all(w in equal and w - delta in equal for w in range(10, 20))
+        if calib_equal:
             assert g["mean"] == r["mean"] and g["std"] == r["std"] and g["limit"] == r["limit"]
             assert np.array_equal(g["flags"], r["flags"])
+        print(f"{kind}: {len(equal)} of {W} windows with equal labels; {n_prev} ARI(t-1,t) and "
+              f"{n_delta} ARI(t-delta,t) compared with the oracle; calibration equal: {calib_equal}")
+        # the cross-side comparisons above must have run on (nearly) every window:
+        # on B200 all 31 windows of both kinds agree, calibration included
+        assert len(equal) >= W - 2, (kind, len(equal))
+        assert n_prev >= W - 5 and n_delta >= W - delta - 4, (kind, n_prev, n_delta)
+        assert calib_equal, kind
         assert g["build_ms"] > 0 and g["fit_ms"] > 0
     assert got["launches"] > 0
 
@@ -161,11 +197,18 @@ def test_rolling_full_size_sampled_windows(m):
                                   only=sample, keep_H=True)
     for kind in ("corr", "tpdm"):
         equal = _compare_windows(got[kind], ref[kind], 24, sample, ref[kind]["H"], kind)
+        _check_series_from_own_labels(got[kind], 24, 50, (50, 125), kind)
+        compared = 0
         for w in (1, 125):
             if w in equal and w - 1 in equal:
                 assert got[kind]["ari_prev"][w] == ref[kind]["ari_prev"][w]
+                compared += 1
         if 174 in equal and 124 in equal:
             assert got[kind]["ari_delta"][174] == ref[kind]["ari_delta"][174]
+            compared += 1
+        print(f"{kind}: sampled windows with equal labels {sorted(equal)}; "
+              f"{compared} of 3 ARIs compared with the oracle")
+        assert len(equal) >= 4 and compared >= 2, (kind, sorted(equal), compared)
         a = got[kind]["ari_delta"]
         assert np.all(np.isnan(a[:50])) and np.all((a[50:] >= -1.0) & (a[50:] <= 1.0))
 
