@@ -201,7 +201,26 @@ def _timed(torch, fn):
     return a.elapsed_time(b), out
 
 
-def measure_rows(m, torch, dev, S, H0, lab, n, k, T, rank, workload):
+def converge_row(m, torch, S, k, planted_dev, solver, **kw):
+    """One fit to the relative-loss-change stop (rel < 1e-5), timed with CUDA
+    events: passes or epochs, seconds, loss, ARI of its labels against the
+    planted groups, and a sampled loss curve."""
+    ms, (H, st) = _timed(torch, lambda: m.fit(S, k, seed=1000, solver=solver, rel_tol=1e-5,
+                                              history=True, **kw))
+    lab = m.labels(H)
+    h = st["history"]
+    pts = sorted({0, 1, 2, 5, 10, 20, 50, 100, 200, 500, 1000, 2000, 5000, 10000, len(h) - 1}
+                 & set(range(len(h))))
+    return lab, {
+        "solver": solver, "seconds": ms / 1e3, "converged": bool(st["converged"]),
+        "full_batch_passes": st["iters"], "epochs": st["epochs"], "evaluations": st["evaluations"],
+        "block_final": st["block_final"], "loss": st["loss"], "rel_change": st["rel_change"],
+        "s_sqnorm": st["s_sqnorm"], "explained": 1.0 - st["loss"] / st["s_sqnorm"],
+        "ARI_vs_planted": m.ari(lab, planted_dev, max(k, int(planted_dev.max().item()) + 1))[0],
+        "loss_curve": {str(i): float(h[i]) for i in pts}}
+
+
+def measure_rows(m, torch, dev, S, H0, lab, n, k, T, rank, workload, planted=None):
     """One timing per remaining row of the path on the resident |corr| matrix
     (probe, labels, statistics, spherical k-means), on a TPDM of the
     heavy-tailed window of the same size (builder, one Block-SVRG epoch), and
@@ -219,7 +238,11 @@ def measure_rows(m, torch, dev, S, H0, lab, n, k, T, rank, workload):
     p = m.fit_params(probe_block=16, probe_max_iter=12)
     wsp = m.workspace(m._lib.OP_SPECTRAL_PROBE, n, k + 2, params=p, device=dev)
     ms, ev = _timed(torch, lambda: m.spectral_probe(S, k + 2, block=16, max_iter=12, tol=1e-7, ws=wsp))
+    info = m.probe_last_info()
     out["probe_ms"] = ms
+    out["probe_s_passes"] = info["s_passes"]
+    out["probe_block_steps"] = info["block_steps"]
+    out["probe_GBs"] = info["s_passes"] * 4.0 * n * n / (ms / 1e3) / 1e9
     out["probe_top"] = [float(x) for x in ev[:3]]
     out["probe_gamma_k1"] = float(ev[k] / abs(ev[k + 1]))
     del wsp
@@ -252,7 +275,16 @@ def measure_rows(m, torch, dev, S, H0, lab, n, k, T, rank, workload):
         out["svrg_fit_1epoch_ms"] = svrg[1][0]
         out["svrg_block_rows"] = b
         out["svrg_epochs"] = svrg[3][1][1]["epochs"]
-        del S2, wsf, Hs
+        del wsf, Hs
+        # the heavy-tailed workload to convergence: Block-SVRG at b = 8,192 with
+        # growth until the snapshot loss changes by less than 1e-5 (cap 2,000 epochs)
+        _, tplanted, _ = synth.workload(tname, seed=rank)
+        tpl = torch.from_numpy(np.asarray(tplanted, dtype=np.int32)).to(dev)
+        tlab, conv = converge_row(m, torch, S2, k, tpl, "block_svrg", block_rows=b, max_iters=2000)
+        kl, _, _, _ = m.spherical_kmeans(S2, k, seed=rank, max_iters=30)
+        conv["kmeans_vs_symnmf_ARI"] = m.ari(kl, tlab, k)[0]
+        out["converge_tpdm_block_svrg"] = conv
+        del S2, tpl
         torch.cuda.empty_cache()
     # spherical k-means on the resident |corr| matrix (two S passes per step),
     # and its agreement with the SymNMF labels (the pages quote about 0.83 on
@@ -267,6 +299,14 @@ def measure_rows(m, torch, dev, S, H0, lab, n, k, T, rank, workload):
     out["kmeans_S_GBs"] = (2 * ksteps - (1 if kconv else 0)) * 4.0 * n * n / (ms / 1e3) / 1e9
     out["kmeans_vs_symnmf_ARI"] = m.ari(klab, lab, k)[0]
     del wsk
+    # the |corr| workload to convergence: full-batch AdaGrad until the loss
+    # changes by less than 1e-5 (cap 20,000 passes)
+    if planted is not None:
+        pl = torch.from_numpy(np.asarray(planted, dtype=np.int32)).to(dev)
+        clab, conv = converge_row(m, torch, S, k, pl, "adagrad", max_iters=20000)
+        conv["kmeans_vs_symnmf_ARI"] = m.ari(klab, clab, k)[0]
+        out["converge_corr_adagrad"] = conv
+        del pl
     # the rolling study: 250 windows of 250 days, |corr| and TPDM, 100-iteration
     # fits, ARI series, 3-sigma limit, cross-sector monitor
     st = synth.rolling_stream(seed=rank)
@@ -297,6 +337,60 @@ def measure_rows(m, torch, dev, S, H0, lab, n, k, T, rank, workload):
     return out
 
 
+def measure_n20000(m, torch, dev, rank):
+    """The two n = 20,000 workloads at their stated sizes: the rank-24 |corr|
+    window (T = 500) with 500 full-batch AdaGrad iterations and a 64-eigenvalue
+    probe, and the heavy-tailed TPDM window (T = 1,000) with 50 Block-SVRG
+    epochs at b = 2,048 (growth on)."""
+    out = {}
+    R, planted, spec = synth.workload("corr_n20000_k24", seed=rank)
+    n, k = spec["n"], spec["k"]
+    Rd = torch.from_numpy(R).to(dev)
+    S = m.alloc_S(n, dev)
+    m.build_corr(Rd, out=S)
+    pl = torch.from_numpy(np.asarray(planted, dtype=np.int32)).to(dev)
+    p = m.fit_params(max_iters=500, rel_tol=0.0)
+    ws = m.workspace(m._lib.OP_FIT, n, k, params=p, device=dev)
+    H = torch.empty((n, k), dtype=torch.float32, device=dev)
+    m.fit(S, k, seed=1000 + rank, max_iters=5, rel_tol=0.0, out=H, ws=ws)   # warm-up
+    ms, (H, st) = _timed(torch, lambda: m.fit(S, k, seed=1000 + rank, max_iters=500, rel_tol=0.0,
+                                              out=H, ws=ws, timing=True))
+    c2 = {"workload": "corr_n20000_k24", "iterations": 500, "ms": ms,
+          "iterations_per_s": 501 / (ms / 1e3),
+          "stream_ms_per_pass": st["stream_ms"] / max(st["stream_launches"], 1),
+          "ARI_vs_planted": m.ari(m.labels(H), pl, k)[0], "loss": st["loss"]}
+    c2["stream_GBs"] = (4.0 * n * n + 4.0 * n * k) / (c2["stream_ms_per_pass"] / 1e3) / 1e9
+    pp = m.fit_params(probe_block=16, probe_max_iter=40)
+    wsp = m.workspace(m._lib.OP_SPECTRAL_PROBE, n, 64, params=pp, device=dev)
+    m.spectral_probe(S, 64, block=16, max_iter=40, tol=1e-7, ws=wsp)   # warm-up
+    pms, ev = _timed(torch, lambda: m.spectral_probe(S, 64, block=16, max_iter=40, tol=1e-7, ws=wsp))
+    info = m.probe_last_info()
+    c2.update({"probe64_ms": pms, "probe64_s_passes": info["s_passes"],
+               "probe64_GBs": info["s_passes"] * 4.0 * n * n / (pms / 1e3) / 1e9,
+               "probe64_gamma_k25": float(ev[24] / abs(ev[25])), "probe64_top": [float(x) for x in ev[:2]]})
+    out["corr_n20000_k24"] = c2
+    del ws, wsp, Rd
+    # heavy-tailed TPDM, Block-SVRG b = 2,048, 50 epochs
+    R, planted, spec = synth.workload("tpdm_n20000_k24", seed=rank)
+    Rd = torch.from_numpy(R).to(dev)
+    m.build_tpdm(Rd, 0.05, 1, out=S)
+    pl = torch.from_numpy(np.asarray(planted, dtype=np.int32)).to(dev)
+    pf = m.fit_params(solver="block_svrg", block_rows=2048, max_iters=50, rel_tol=0.0)
+    wsf = m.workspace(m._lib.OP_FIT, n, k, params=pf, device=dev)
+    m.fit(S, k, seed=1000 + rank, solver="block_svrg", block_rows=2048, max_iters=2, rel_tol=0.0,
+          out=H, ws=wsf)   # warm-up
+    ms, (H, st) = _timed(torch, lambda: m.fit(S, k, seed=1000 + rank, solver="block_svrg",
+                                              block_rows=2048, max_iters=50, rel_tol=0.0,
+                                              out=H, ws=wsf))
+    out["tpdm_n20000_k24"] = {"workload": "tpdm_n20000_k24", "epochs": st["epochs"],
+                              "full_batch_passes": st["iters"], "block_final": st["block_final"],
+                              "ms": ms, "epochs_per_s": 50 / (ms / 1e3),
+                              "ARI_vs_planted": m.ari(m.labels(H), pl, k)[0], "loss": st["loss"]}
+    del S, Rd, wsf
+    torch.cuda.empty_cache()
+    return out
+
+
 def row_rooflines(rows, n, k, T, hbm_peak):
     """Algorithmic traffic (or flops) of each timed row over its time, as a fraction of
     the measured peaks: HBM copy bandwidth for streams, and for the |corr| Gram the
@@ -308,6 +402,8 @@ def row_rooflines(rows, n, k, T, hbm_peak):
             gbs = bytes_ / (ms / 1e3) / 1e9
             out[name] = {"bound": "hbm", "GBs": gbs, "frac": gbs / hbm_peak}
     hbm("stats", sbytes, rows.get("stats_ms"))
+    if "probe_s_passes" in rows:
+        hbm("probe", rows["probe_s_passes"] * sbytes, rows.get("probe_ms"))
     if "kmeans_steps" in rows:
         # two S passes per assignment step; the last step stops after its assignment
         hbm("kmeans_step", 2 * sbytes, rows.get("kmeans_ms_per_step"))
@@ -477,7 +573,9 @@ def run_ours(args):
     rows = None
     if not args.no_rows:
         try:
-            rows = measure_rows(m, torch, dev, S, H0, lab, n, k, T, rank, args.workload)
+            rows = measure_rows(m, torch, dev, S, H0, lab, n, k, T, rank, args.workload, planted)
+            if n == 100000:
+                rows["n20000"] = measure_n20000(m, torch, dev, rank)
             rows["roofline"], tf32_peak = row_rooflines(rows, n, k, T, peak)
             rows["roofline"]["corr_build"] = {
                 "bound": "tensor", "tf32_TFs": 3.0 * n * n * T / (build_ms / 1e3) / 1e12,
@@ -517,7 +615,9 @@ def run_ours(args):
             "e2e": e2e,
             "cpu_baseline": cpu,
             "rows": rows,
-            "context": {"corr_build_ms": build_ms,
+            "context": {"pages_time_to_converge_s": {"corr": 13.0, "tpdm": 12.4,
+                                                     "hardware": "4x GB200 (the pages' own data)"},
+                        "corr_build_ms": build_ms,
                         "corr_build_tf32_TFs": 3.0 * n * n * T / (build_ms / 1e3) / 1e12, "torch_mm_S_H_ms": mm_ms,
                         "ARI_vs_planted": ari_planted,
                         "final_loss": st["loss"], "loop_ms": st["loop_ms"]},

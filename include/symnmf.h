@@ -219,6 +219,21 @@ SYMNMF_API int symnmf_spectral_probe(const float* S, int64_t n, int64_t lds, int
                           symnmf_stream_t stream);
 
 /*
+ * What the last symnmf_spectral_probe call on this host thread did: the
+ * number of passes over S it launched (each reads the n x n matrix once,
+ * with a block-wide operand) and the kernels it launched in all.  Lets a
+ * caller put the probe's time on the HBM roofline (bytes = s_passes * 4 n^2).
+ * Zeros before the first call.  Returns SYMNMF_OK, or SYMNMF_ERR_INVALID_ARG
+ * for a NULL out.
+ */
+typedef struct {
+    int s_passes;           /* S-stream passes (one per Krylov block, plus the start) */
+    int block_steps;        /* Lanczos block steps taken */
+    int kernel_launches;    /* kernels launched by the call */
+} symnmf_probe_info;
+SYMNMF_API int symnmf_probe_last_info(symnmf_probe_info* out);
+
+/*
  * Factorise S ~ H H^T, H >= 0 ([SMI] AdaptGrow sketch; [CaS] "Factorizing
  * with SymNMF": G <- G + g*g, H <- max(H - lr g/(sqrt(G)+eps), 0)).
  *   ADAGRAD:    g = 4 (H (H^T H) - S H), one S pass per iteration; the pass

@@ -278,6 +278,17 @@ def _f32(a):
     return a.astype(np.float32).astype(np.float64)
 
 
+def _operand(S):
+    """S as the solvers use it.  Normally the matrix widened to float64.  An
+    object that declares ``exact_float64_products = True`` is passed through
+    unchanged: it supplies the two products the solvers form, ``S @ X`` and
+    ``S[:, rows] @ D``, exactly in float64 (a matrix too large to widen at
+    once, read in row chunks).  The solvers then need ``S_sqnorm`` given."""
+    if getattr(S, "exact_float64_products", False):
+        return S
+    return np.asarray(S, dtype=np.float64)
+
+
 def fit_adagrad(S, k, H0, lr=0.1, eps=1e-10, max_iters=200, rel_tol=0.0,
                 G0=None, mirror=True, S_sqnorm=None, hook=None) -> FitResult:
     """Full-batch projected AdaGrad ([SMI] AdaptGrow sketch, phi >= 1 branch).
@@ -287,7 +298,7 @@ def fit_adagrad(S, k, H0, lr=0.1, eps=1e-10, max_iters=200, rel_tol=0.0,
     t = max_iters, and returns H_t; otherwise it takes the update of H_t.
     ``hook(t, H, P)`` (tests only) sees every evaluated iterate.
     """
-    S = np.asarray(S, dtype=np.float64)
+    S = _operand(S)
     n = S.shape[0]
     H = np.asarray(H0, dtype=np.float64).reshape(n, k).copy()
     G = np.zeros_like(H) if G0 is None else np.asarray(G0, dtype=np.float64).copy()
@@ -386,7 +397,7 @@ def fit_block_svrg(S, k, H0, lr=0.1, eps=1e-10, max_epochs=50, rel_tol=0.0,
     ("same diagonal AdaGrad update either way"); each such iteration counts
     as one epoch of the budget.
     """
-    S = np.asarray(S, dtype=np.float64)
+    S = _operand(S)
     n = S.shape[0]
     H = np.asarray(H0, dtype=np.float64).reshape(n, k).copy()
     G = np.zeros_like(H) if G0 is None else np.asarray(G0, dtype=np.float64).copy()

@@ -117,6 +117,10 @@ class RollingOut(C.Structure):
     ]
 
 
+class ProbeInfo(C.Structure):
+    _fields_ = [("s_passes", C.c_int), ("block_steps", C.c_int), ("kernel_launches", C.c_int)]
+
+
 _vp, _i64, _int, _sz = C.c_void_p, C.c_int64, C.c_int, C.c_size_t
 
 # name -> (restype, argtypes); every symbol include/symnmf.h declares
@@ -132,6 +136,7 @@ SIGNATURES = {
     "symnmf_sh": (_int, [_vp, _i64, _i64, _vp, _int, _vp, _vp, _sz, _vp]),
     "symnmf_spectral_probe": (_int, [_vp, _i64, _i64, _int, _int, _int, C.c_double, C.c_uint64,
                                      C.POINTER(C.c_double), _vp, _sz, _vp]),
+    "symnmf_probe_last_info": (_int, [C.POINTER(ProbeInfo)]),
     "symnmf_fit": (_int, [_vp, _i64, _i64, _int, C.POINTER(FitParams), _vp, C.POINTER(FitStats),
                           _vp, _sz, _vp]),
     "symnmf_labels": (_int, [_vp, _i64, _int, _vp, _vp]),

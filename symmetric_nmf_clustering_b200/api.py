@@ -128,6 +128,15 @@ def spectral_probe(S: torch.Tensor, n_eig: int, block: int = 16, max_iter: int =
     return np.array(out[:], dtype=np.float64)
 
 
+def probe_last_info() -> dict:
+    """S passes, block steps and kernel launches of the last spectral_probe
+    call on this thread (the probe's bytes are s_passes * 4 n^2)."""
+    info = L.ProbeInfo()
+    L.check("symnmf_probe_last_info", _lib().symnmf_probe_last_info(C.byref(info)))
+    return {"s_passes": info.s_passes, "block_steps": info.block_steps,
+            "kernel_launches": info.kernel_launches}
+
+
 def fit_params(**kw) -> FitParams:
     p = FitParams()
     _lib().symnmf_fit_params_default(C.byref(p))

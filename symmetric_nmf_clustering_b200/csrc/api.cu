@@ -926,9 +926,14 @@ static int orthonormalize(const ProbeLayout& L, float* V, int64_t n, int64_t ldv
     return SYMNMF_OK;
 }
 
+// what the last probe on this host thread did (symnmf_probe_last_info)
+static thread_local symnmf_probe_info g_probe_info = {0, 0, 0};
+
 static int probe_impl(const Dev& d, const float* S, int64_t n, int64_t lds, int n_eig, int b,
                       int max_iter, double tol, uint64_t seed, double* eig_out, void* ws,
                       size_t ws_bytes, cudaStream_t s) {
+    g_probe_info = symnmf_probe_info{0, 0, 0};
+    const int launches0 = launches();
     Arena a;
     a.base = static_cast<char*>(ws);
     a.cap = ws_bytes;
@@ -965,7 +970,9 @@ static int probe_impl(const Dev& d, const float* S, int64_t n, int64_t lds, int 
     bool converged = false;
     // W = S Q_0 (one S pass)
     SYMNMF_TRY(stream_pass(d, sa, L.Q, nullptr, ldq, 0, n, false, epi_product(n, b, L.W), s, nullptr));
+    g_probe_info.s_passes = 1;
     for (int j = 0; j < steps; ++j) {
+        g_probe_info.block_steps = j + 1;
         // W holds S Q_j: full reorthogonalisation against Q_0..Q_j, twice; the
         // Q_j coefficients are A_j
         const int nq = (j + 1) * b;
@@ -996,6 +1003,7 @@ static int probe_impl(const Dev& d, const float* S, int64_t n, int64_t lds, int 
                 }
             SYMNMF_TRY(stream_pass(d, sa, Qn, nullptr, ldq, 0, n, false, epi_product(n, b, L.W), s,
                                    nullptr));
+            g_probe_info.s_passes += 1;
         }
         // Rayleigh-Ritz on the leading nq x nq block of the block tridiagonal T
         if (nq >= n_eig) {
@@ -1026,6 +1034,7 @@ static int probe_impl(const Dev& d, const float* S, int64_t n, int64_t lds, int 
         return SYMNMF_ERR_INVALID_ARG;
     }
     for (int i = 0; i < n_eig; ++i) eig_out[i] = theta[i];
+    g_probe_info.kernel_launches = launches() - launches0;
     return SYMNMF_OK;
 }
 
@@ -1404,6 +1413,13 @@ int symnmf_sh(const float* S, int64_t n, int64_t lds, const float* X, int k, flo
         set_error("an S-stream pipeline wait timed out on the device (code %d)", h);
         return SYMNMF_ERR_TIMEOUT;
     }
+    return SYMNMF_OK;
+}
+
+int symnmf_probe_last_info(symnmf_probe_info* out) {
+    clear_error();
+    SYMNMF_CHECK_ARG(out != nullptr, "out must not be NULL");
+    *out = g_probe_info;
     return SYMNMF_OK;
 }
 

@@ -57,3 +57,75 @@ def assert_labels_differ_only_on_near_ties(lab_gpu, lab_oracle, H_gpu, H_oracle,
           if not bad.any() else f"labels: {int(bad.sum())} rows differ on clear margins")
     assert not bad.any(), np.flatnonzero(bad)[:10]
     return int(diff.sum())
+
+
+class DeviceRowChunks:
+    """A device n x n float32 matrix as the oracle's solvers see it when it is
+    too large to widen at once: it supplies S @ X and S[:, cols] @ D in
+    float64, copying row chunks (or their column slabs) from the device into
+    pinned host memory, widening them exactly to float64 in a reused buffer
+    and multiplying on the host.  Test plumbing only: copies and a library
+    matrix product, none of the method's arithmetic."""
+
+    exact_float64_products = True
+
+    def __init__(self, S_dev, rows_per_chunk=2048):
+        import torch
+        self.S = S_dev
+        self.n = S_dev.shape[0]
+        self.shape = (self.n, S_dev.shape[1])
+        self.c = rows_per_chunk
+        self.cuda = S_dev.is_cuda
+        pin = torch.empty(self.c * self.shape[1], dtype=torch.float32)
+        self.pin = pin.pin_memory() if self.cuda else pin
+        self.f64 = torch.empty(self.c * self.shape[1], dtype=torch.float64)
+
+    def _chunks(self, c0=0, c1=None):
+        import torch
+        c1 = self.shape[1] if c1 is None else c1
+        w = c1 - c0
+        for r0 in range(0, self.n, self.c):
+            r1 = min(self.n, r0 + self.c)
+            hb = self.pin[: (r1 - r0) * w].view(r1 - r0, w)     # contiguous
+            hb.copy_(self.S[r0:r1, c0:c1])
+            if self.cuda:
+                torch.cuda.synchronize()
+            db = self.f64[: (r1 - r0) * w].view(r1 - r0, w)
+            db.copy_(hb)
+            yield r0, r1, db
+
+    def __matmul__(self, X):
+        import torch
+        X = torch.from_numpy(np.ascontiguousarray(X, dtype=np.float64))
+        out = np.empty((self.n, X.shape[1]))
+        for r0, r1, db in self._chunks():
+            out[r0:r1] = torch.mm(db, X).numpy()
+        return out
+
+    def __getitem__(self, key):
+        rows, cols = key
+        assert rows == slice(None, None, None) and isinstance(cols, slice) and cols.step is None
+        return _ColumnSlab(self, cols.start, min(cols.stop, self.shape[1]))
+
+    def stats(self):
+        """(sum, squared norm, non-finite count) from the oracle's stats on each chunk."""
+        t = [0.0, 0.0, 0]
+        for _, _, db in self._chunks():
+            a, b, c = oracle.stats(db.numpy())
+            t[0] += a
+            t[1] += b
+            t[2] += c
+        return tuple(t)
+
+
+class _ColumnSlab:
+    def __init__(self, parent, c0, c1):
+        self.p, self.c0, self.c1 = parent, c0, c1
+
+    def __matmul__(self, D):
+        import torch
+        D = torch.from_numpy(np.ascontiguousarray(D, dtype=np.float64))
+        out = np.empty((self.p.n, D.shape[1]))
+        for r0, r1, db in self.p._chunks(self.c0, self.c1):
+            out[r0:r1] = torch.mm(db, D).numpy()
+        return out

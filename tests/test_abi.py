@@ -40,7 +40,9 @@ def test_every_declared_symbol_is_exported(lib):
 def test_struct_layout_matches_c(lib):
     from symmetric_nmf_clustering_b200 import _lib
     probes = []
-    for cname, py in (("symnmf_fit_params", _lib.FitParams), ("symnmf_fit_stats", _lib.FitStats)):
+    structs = (("symnmf_fit_params", _lib.FitParams), ("symnmf_fit_stats", _lib.FitStats),
+               ("symnmf_probe_info", _lib.ProbeInfo))
+    for cname, py in structs:
         probes.append(f'printf("{cname} %zu\\n", sizeof({cname}));')
         for f, _ in py._fields_:
             probes.append(f'printf("{cname}.{f} %zu\\n", offsetof({cname}, {f}));')
@@ -53,7 +55,7 @@ def test_struct_layout_matches_c(lib):
         subprocess.run(["gcc", "-std=c11", "-I", os.path.dirname(HEADER), c, "-o", exe], check=True)
         lines = subprocess.run([exe], capture_output=True, text=True, check=True).stdout.split("\n")
     want = dict(l.split() for l in lines if l.strip())
-    for cname, py in (("symnmf_fit_params", _lib.FitParams), ("symnmf_fit_stats", _lib.FitStats)):
+    for cname, py in structs:
         assert int(want[cname]) == C.sizeof(py)
         for f, _ in py._fields_:
             assert int(want[f"{cname}.{f}"]) == getattr(py, f).offset, f
