@@ -84,7 +84,8 @@ enum {
     SYMNMF_OP_STATS = 5,
     SYMNMF_OP_SPHERICAL_KMEANS = 6,
     SYMNMF_OP_ARI = 7,
-    SYMNMF_OP_ROLLING = 8
+    SYMNMF_OP_ROLLING = 8,
+    SYMNMF_OP_SH_UPPER = 9
 };
 enum { SYMNMF_KIND_CORR = 1, SYMNMF_KIND_TPDM = 2 };
 
@@ -104,7 +105,9 @@ typedef struct {
     int grow;                /* AdaptGrow: double b when an epoch stalls; default 1 */
     double stall_tol;        /* stall = relative snapshot-loss decrease below this; default 1e-4 */
     double gap_threshold;    /* AUTO: gamma_{k+1} >= this selects full batch; default 5.0 */
-    int upper_only;          /* reserved; must be 0 */
+    int upper_only;          /* 1: full-batch passes and Block-SVRG snapshots read only the tiles on or
+                                above the diagonal of S (symnmf_sh_upper; k <= 24, S rounded to TF32 in
+                                the product); Block-SVRG block steps read their slab as usual. Default 0 */
     float* G_inout;          /* optional device n*k: AdaGrad accumulator in (resume) and out; NULL = start at 0 */
     double* loss_history;    /* optional host array: f(H_t) of every evaluation (snapshots for Block-SVRG) */
     int loss_history_len;    /* capacity of loss_history */
@@ -200,6 +203,27 @@ SYMNMF_API int symnmf_stats(const float* S, int64_t n, int64_t lds, double* out_
  */
 SYMNMF_API int symnmf_sh(const float* S, int64_t n, int64_t lds, const float* X, int k,
               float* Y, void* ws, size_t ws_bytes, symnmf_stream_t stream);
+
+/*
+ * Y = S X like symnmf_sh, reading only the 128 x 128 tiles of S on or above
+ * the diagonal and using symmetry for the rest: half of the n^2 entries.  The
+ * scope of this hot path allows the S-stream to read only the upper triangle
+ * and exploit symmetry; the pages stream the full matrix ([CaS]
+ * "Factorization at scale").  Each tile S[p, q], p <= q, feeds Y_p += S[p, q] X_q
+ * and, for p < q, Y_q += S[p, q]^T X_p; partial sums are reduced in a fixed
+ * order (bitwise reproducible).  The entries below the diagonal tiles are
+ * never read, so S must be symmetric there.
+ *
+ * Precision: X enters as its exact TF32 split (as in symnmf_sh); S enters
+ * rounded to the nearest TF32 value, an unbiased per-entry error of at most
+ * 2^-12 relative that averages out along a row (a few 1e-6 relative in Y on
+ * the |corr| and TPDM workloads); a matrix whose entries all round in the same
+ * direction sees up to 2^-12.  1 <= k <= 24.  Workspace: SYMNMF_OP_SH_UPPER
+ * (partial slabs, about (n^2 / 256 + n * items) * 4 k bytes: 1.2 GB at
+ * n = 100,000, k = 24).  Synchronises `stream` (reads the device error word).
+ */
+SYMNMF_API int symnmf_sh_upper(const float* S, int64_t n, int64_t lds, const float* X, int k,
+                               float* Y, void* ws, size_t ws_bytes, symnmf_stream_t stream);
 
 /*
  * Leading eigenvalues of S by block Lanczos with full reorthogonalisation on

@@ -22,7 +22,7 @@ SYMNMF_ERR_NOT_SUPPORTED = 6
 SOLVER_ADAGRAD, SOLVER_BLOCK_SVRG, SOLVER_AUTO = 0, 1, 2
 INIT_SEEDED, INIT_USER = 0, 1
 (OP_BUILD_CORR, OP_BUILD_TPDM, OP_SPECTRAL_PROBE, OP_FIT, OP_SH, OP_STATS,
- OP_SPHERICAL_KMEANS, OP_ARI, OP_ROLLING) = range(9)
+ OP_SPHERICAL_KMEANS, OP_ARI, OP_ROLLING, OP_SH_UPPER) = range(10)
 KIND_CORR, KIND_TPDM = 1, 2
 
 
@@ -134,6 +134,7 @@ SIGNATURES = {
     "symnmf_build_tpdm": (_int, [_vp, _i64, _i64, _i64, C.c_double, _int, _vp, _i64, _vp, _sz, _vp]),
     "symnmf_stats": (_int, [_vp, _i64, _i64, _vp, _vp, _sz, _vp]),
     "symnmf_sh": (_int, [_vp, _i64, _i64, _vp, _int, _vp, _vp, _sz, _vp]),
+    "symnmf_sh_upper": (_int, [_vp, _i64, _i64, _vp, _int, _vp, _vp, _sz, _vp]),
     "symnmf_spectral_probe": (_int, [_vp, _i64, _i64, _int, _int, _int, C.c_double, C.c_uint64,
                                      C.POINTER(C.c_double), _vp, _sz, _vp]),
     "symnmf_probe_last_info": (_int, [C.POINTER(ProbeInfo)]),

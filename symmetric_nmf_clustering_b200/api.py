@@ -115,6 +115,19 @@ def sh(S: torch.Tensor, X: torch.Tensor, ws: torch.Tensor | None = None) -> torc
     return Y
 
 
+def sh_upper(S: torch.Tensor, X: torch.Tensor, ws: torch.Tensor | None = None) -> torch.Tensor:
+    """Y = S X reading only the tiles of S on or above the diagonal (k <= 24)."""
+    n, _, lds = _matrix(S, "S")
+    _dense(X, "X")
+    k = X.shape[1]
+    Y = torch.empty_like(X)
+    ws = workspace(L.OP_SH_UPPER, n, k, device=S.device) if ws is None else ws
+    L.check("symnmf_sh_upper", _lib().symnmf_sh_upper(S.data_ptr(), n, lds, X.data_ptr(), k,
+                                                      Y.data_ptr(), ws.data_ptr(), ws.numel(),
+                                                      _stream(S.device)))
+    return Y
+
+
 def spectral_probe(S: torch.Tensor, n_eig: int, block: int = 16, max_iter: int = 40,
                    tol: float = 1e-6, seed: int = 0, ws: torch.Tensor | None = None) -> np.ndarray:
     """The n_eig leading eigenvalues of S (descending) by block Lanczos."""
@@ -152,7 +165,7 @@ def fit(S: torch.Tensor, k: int, *, H0: torch.Tensor | None = None, G: torch.Ten
         max_iters: int = 2000, rel_tol: float = 1e-5, block_rows: int = 0, grow: bool = True,
         stall_tol: float = 1e-4, gap_threshold: float = 5.0, eigvals=None,
         probe_block: int = 16, probe_max_iter: int = 40, probe_tol: float = 1e-6,
-        check_every: int = 16, timing: bool = False, history: bool = False,
+        check_every: int = 16, timing: bool = False, history: bool = False, upper_only: bool = False,
         out: torch.Tensor | None = None, ws: torch.Tensor | None = None):
     """Factorise S ~ H H^T with H >= 0.  Returns (H, stats dict).
 
@@ -175,7 +188,7 @@ def fit(S: torch.Tensor, k: int, *, H0: torch.Tensor | None = None, G: torch.Ten
                    rel_tol=rel_tol, block_rows=block_rows, grow=int(grow), stall_tol=stall_tol,
                    gap_threshold=gap_threshold, probe_block=probe_block,
                    probe_max_iter=probe_max_iter, probe_tol=probe_tol, check_every=check_every,
-                   timing=int(timing))
+                   timing=int(timing), upper_only=int(upper_only))
     if G is not None:
         _dense(G, "G")
         p.G_inout = G.data_ptr()

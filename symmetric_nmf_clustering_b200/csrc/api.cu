@@ -100,6 +100,9 @@ struct StreamArgs {
     int* err;
     int* counters; // one per 128-row tile, zero between passes (tensor-core path)
     const FitState* st;
+    bool upper = false;       // full passes read only the tiles on or above the diagonal
+    float* tpart = nullptr;   // their partial slabs
+    float* fpart = nullptr;
 };
 
 // One pass over S: part[s] = S[:, r0:r1] X[r0:r1, :] with X = Xa - Xb (Xb may be
@@ -128,6 +131,8 @@ struct FitLayout {
     float* XT[2] = {nullptr, nullptr};   // split operand of Hb[0] / Hb[1]
     int64_t ldxt = 0;
     int* counters = nullptr;
+    float* tpart = nullptr;              // upper-triangle partial slabs (upper_only = 1)
+    float* fpart = nullptr;
 };
 
 static int64_t default_block_rows(int64_t n) {
@@ -199,6 +204,12 @@ static int plan_fit(const Dev& d, Arena& a, int64_t n, int k, const symnmf_fit_p
             }
         }
     }
+    if (P.upper_only) {
+        const TriPlan tp = plan_stream_tri(d, n, k);
+        pf = std::max(pf, (size_t)n * k);   // the reduced product goes to part
+        L->tpart = a.take<float>(tri_tpart_floats(tp));
+        L->fpart = a.take<float>(tri_fpart_floats(tp));
+    }
     L->part = a.take<float>(pf);
     L->ldxt = xt_ld(n);
     L->XT[0] = a.take<float>((size_t)xt_rows(k) * L->ldxt);
@@ -234,7 +245,8 @@ static int check_params(const symnmf_fit_params& P, int64_t n, int k) {
     SYMNMF_CHECK_ARG(P.max_iters >= 0 && P.max_iters < (1 << 30), "max_iters must be >= 0");
     SYMNMF_CHECK_ARG(P.rel_tol >= 0.0, "rel_tol must be >= 0");
     SYMNMF_CHECK_ARG(P.block_rows >= 0, "block_rows must be >= 0");
-    SYMNMF_CHECK_ARG(P.upper_only == 0, "upper_only is reserved and must be 0");
+    SYMNMF_CHECK_ARG(P.upper_only == 0 || P.upper_only == 1, "upper_only must be 0 or 1");
+    SYMNMF_CHECK_ARG(!P.upper_only || tri_supported(k), "upper_only = 1 supports k <= 24 (k = %d)", k);
     SYMNMF_CHECK_ARG(P.check_every >= 1, "check_every must be >= 1");
     if (P.solver == SYMNMF_SOLVER_AUTO) {
         SYMNMF_CHECK_ARG(k + 2 <= n, "AUTO needs n >= k + 2 eigenvalues");
@@ -329,6 +341,21 @@ static int stream_pass(const Dev& d, const StreamArgs& a, const float* Xa, const
                        int64_t ldx, int64_t r0, int64_t r1, bool xt_ready, EpiArgs epi,
                        cudaStream_t s, Timing* tm) {
     epi.part = a.part;
+    if (a.upper && r0 == 0 && r1 == a.n) {
+        // upper-triangle stream: S X into part (or straight into Y for a product),
+        // then the standalone epilogue over that one partial
+        const TriPlan p = plan_stream_tri(d, a.n, a.k);
+        if (!xt_ready) SYMNMF_TRY(launch_split(Xa, Xb, ldx, a.k, 0, a.n, 0, a.n, a.XT, a.ldxt, s));
+        if (tm) SYMNMF_TRY(tm->begin(s));
+        SYMNMF_TRY(launch_stream_tri(p, a.S, a.lds, a.XT, a.ldxt, a.tpart, a.fpart, a.err, a.st, s));
+        if (tm) SYMNMF_TRY(tm->end(s));
+        const bool product = epi.mode == MODE_PRODUCT;
+        SYMNMF_TRY(launch_tri_reduce(p, a.tpart, a.fpart, product ? epi.Y : a.part, a.st, s));
+        if (product) return SYMNMF_OK;
+        return launch_epilogue(epi.mode, epi.n, epi.k, a.part, 1, epi.H, epi.G, epi.Hn, epi.Gn,
+                               epi.Psnap, epi.m_scale, epi.lr, epi.eps, epi.tr_part, epi.gram_part,
+                               epi.Y, epi.st, s, epi.XT, epi.ldxt);
+    }
     if (use_tc()) {
         const TcPlan p = plan_stream_tc(d, a.n, a.k, r0, r1);
         if (!xt_ready)
@@ -385,6 +412,9 @@ struct FitCtx {
         a.err = &L.st->kerr;
         a.counters = L.counters;
         a.st = L.st;
+        a.upper = P->upper_only != 0;
+        a.tpart = L.tpart;
+        a.fpart = L.fpart;
         return a;
     }
     // epilogue arguments of a pass that reads Hb[cur] and writes Hb[cur ^ 1]
@@ -1267,6 +1297,15 @@ int symnmf_workspace_size(int op, int64_t n, int k, int64_t T, const symnmf_fit_
             a.take<int>((size_t)epilogue_blocks(n));
             break;
         }
+        case SYMNMF_OP_SH_UPPER: {
+            SYMNMF_CHECK_ARG(tri_supported(k), "SYMNMF_OP_SH_UPPER supports 1 <= k <= 24");
+            const TriPlan tp = plan_stream_tri(d, n, k);
+            a.take<float>(tri_tpart_floats(tp));
+            a.take<float>(tri_fpart_floats(tp));
+            a.take<float>((size_t)xt_rows(k) * xt_ld(n));
+            a.take<int>(64);
+            break;
+        }
         case SYMNMF_OP_STATS:
             a.take<double>((size_t)stats_blocks() * 3);
             break;
@@ -1406,6 +1445,50 @@ int symnmf_sh(const float* S, int64_t n, int64_t lds, const float* X, int k, flo
     SYMNMF_CUDA_TRY(cudaMemsetAsync(sa.counters, 0, (size_t)epilogue_blocks(n) * sizeof(int), s));
     SYMNMF_TRY(stream_pass(d, sa, X, nullptr, k, 0, n, false, epi_product(n, k, Y), s, nullptr));
     // a bounded device-side wait that gave up is reported in the error word
+    int h = 0;
+    SYMNMF_CUDA_TRY(cudaMemcpyAsync(&h, sa.err, sizeof(int), cudaMemcpyDeviceToHost, s));
+    SYMNMF_CUDA_TRY(cudaStreamSynchronize(s));
+    if (h != 0) {
+        set_error("an S-stream pipeline wait timed out on the device (code %d)", h);
+        return SYMNMF_ERR_TIMEOUT;
+    }
+    return SYMNMF_OK;
+}
+
+int symnmf_sh_upper(const float* S, int64_t n, int64_t lds, const float* X, int k, float* Y,
+                    void* ws, size_t ws_bytes, symnmf_stream_t stream) {
+    clear_error();
+    SYMNMF_TRY(check_S(S, n, lds));
+    SYMNMF_CHECK_ARG(tri_supported(k), "k = %d must be in [1, 24]", k);
+    SYMNMF_CHECK_ARG(X != nullptr && Y != nullptr && aligned4(X) && aligned4(Y), "X and Y must be device pointers");
+    SYMNMF_TRY(check_ws(ws, ws_bytes));
+    Dev d;
+    SYMNMF_TRY(device_info(&d));
+    Arena a;
+    a.base = static_cast<char*>(ws);
+    a.cap = ws_bytes;
+    const TriPlan tp = plan_stream_tri(d, n, k);
+    StreamArgs sa;
+    sa.S = S;
+    sa.n = n;
+    sa.lds = lds;
+    sa.k = k;
+    sa.part = nullptr;
+    sa.tpart = a.take<float>(tri_tpart_floats(tp));
+    sa.fpart = a.take<float>(tri_fpart_floats(tp));
+    sa.ldxt = xt_ld(n);
+    sa.XT = a.take<float>((size_t)xt_rows(k) * sa.ldxt);
+    sa.err = a.take<int>(64);
+    sa.counters = nullptr;
+    sa.st = nullptr;
+    sa.upper = true;
+    if (!a.ok()) {
+        set_error("workspace too small: %zu given, %zu needed", ws_bytes, a.used);
+        return SYMNMF_ERR_WORKSPACE;
+    }
+    cudaStream_t s = (cudaStream_t)stream;
+    SYMNMF_CUDA_TRY(cudaMemsetAsync(sa.err, 0, sizeof(int), s));
+    SYMNMF_TRY(stream_pass(d, sa, X, nullptr, k, 0, n, false, epi_product(n, k, Y), s, nullptr));
     int h = 0;
     SYMNMF_CUDA_TRY(cudaMemcpyAsync(&h, sa.err, sizeof(int), cudaMemcpyDeviceToHost, s));
     SYMNMF_CUDA_TRY(cudaStreamSynchronize(s));

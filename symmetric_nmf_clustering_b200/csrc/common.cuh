@@ -141,6 +141,26 @@ struct EpiArgs;
 int launch_stream_tc(const TcPlan& p, const float* S, int64_t lds, const float* XT, int64_t ldxt,
                      float* part, int* err, const FitState* st, cudaStream_t s,
                      const EpiArgs* epi = nullptr, int* counters = nullptr);
+// Upper-triangle S-stream (stream_tri.cu): Y = S X from the tiles S[p, q], p <= q,
+// S rounded to TF32; partial slabs in the workspace, reduced by a second kernel.
+struct TriPlan {
+    int64_t n;
+    int k, KP;
+    int T;            // 128-row tiles
+    int items;        // work items (panel x run of column tiles)
+    int grid;         // persistent CTAs
+    int64_t tslabs;   // transposed partial slabs
+};
+TriPlan plan_stream_tri(const Dev& d, int64_t n, int k);
+size_t tri_tpart_floats(const TriPlan& p);
+size_t tri_fpart_floats(const TriPlan& p);
+bool tri_supported(int k);
+int launch_stream_tri(const TriPlan& p, const float* S, int64_t lds, const float* XT, int64_t ldxt,
+                      float* tpart, float* fpart, int* err, const FitState* st, cudaStream_t s);
+int launch_tri_reduce(const TriPlan& p, const float* tpart, const float* fpart, float* Y,
+                      const FitState* st, cudaStream_t s);
+int tri_set_stall(int on);
+
 int launch_split(const float* Xa, const float* Xb, int64_t ldx, int k, int64_t r0, int64_t r1,
                  int64_t jlo, int64_t jhi, float* XT, int64_t ldxt, cudaStream_t s);
 inline int64_t xt_ld(int64_t n) { return (n + 31) / 32 * 32; }

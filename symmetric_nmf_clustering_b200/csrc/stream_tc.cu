@@ -444,8 +444,8 @@ static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 
 // Row-major fp32 matrix (rows x cols, row pitch `ld` elements) as a 2-D TMA
 // map with boxes of 32 columns x box_rows rows and 128-byte swizzle.
-static int make_map(CUtensorMap* m, const float* base, int64_t cols, int64_t rows, int64_t ld,
-                    uint32_t box_rows) {
+int make_map(CUtensorMap* m, const float* base, int64_t cols, int64_t rows, int64_t ld,
+             uint32_t box_rows) {
     auto fn = encode_fn();
     if (fn == nullptr) {
         set_error("cuTensorMapEncodeTiled is not available from the driver");
@@ -543,5 +543,5 @@ extern "C" int symnmf_test_stall_pipeline(int on) {
         symnmf::set_error("cudaMemcpyToSymbol failed: %s", cudaGetErrorString(e));
         return SYMNMF_ERR_CUDA;
     }
-    return SYMNMF_OK;
+    return symnmf::tri_set_stall(v);
 }

@@ -107,10 +107,15 @@ def test_argument_validation_before_any_device_work(lib):
     assert lib.symnmf_build_tpdm(fake, 20, 8, 8, 0.05, 2, fake, 8, fake, 0, None) == 1
     # T < 2 for correlation
     assert lib.symnmf_build_corr(fake, 1, 8, 8, fake, 8, fake, 0, None) == 1
-    # reserved option
-    p.upper_only = 1
+    # upper_only: 0 or 1, and k <= 24 with the upper-triangle stream
+    p.upper_only = 2
     assert lib.symnmf_fit(fake, 12, 12, 3, C.byref(p), fake, None, fake, 0, None) == 1
     assert b"upper_only" in lib.symnmf_last_error()
+    p.upper_only = 1
+    assert lib.symnmf_fit(fake, 40, 40, 25, C.byref(p), fake, None, fake, 0, None) == 1
+    assert b"upper_only" in lib.symnmf_last_error()
+    assert lib.symnmf_sh_upper(fake, 40, 40, fake, 25, fake, fake, 0, None) == 1
+    assert lib.symnmf_sh_upper(fake + 4, 40, 40, fake, 8, fake, fake, 0, None) == 1
 
 
 def test_python_binding_fails_loudly_without_library(tmp_path):

@@ -68,3 +68,17 @@ def test_fit_reports_the_timeout_and_the_context_recovers(m):
     torch.cuda.synchronize()
     assert st1["iters"] == 20 and np.isfinite(st1["loss"])
     assert torch.equal(H1, H2) and st1["loss"] == st2["loss"]
+
+
+def test_sh_upper_reports_the_timeout_and_the_context_recovers(m):
+    # the upper-triangle stream's waits are bounded the same way
+    import torch
+    from symmetric_nmf_clustering_b200 import _lib as L
+    lib = L.load()
+    S_host, S, X = _problem(1000, 8, 2)
+    _stalled(lib, lambda: m.sh_upper(S, X))
+    Y = m.sh_upper(S, X)
+    torch.cuda.synchronize()
+    ref = S_host.astype(np.float64) @ X.cpu().numpy().astype(np.float64)
+    got = Y.cpu().numpy().astype(np.float64)
+    assert np.linalg.norm(got - ref) <= 1e-4 * np.linalg.norm(ref)
