@@ -243,6 +243,51 @@ SYMNMF_API int symnmf_spectral_probe(const float* S, int64_t n, int64_t lds, int
                           symnmf_stream_t stream);
 
 /*
+ * Row-sharded fit, per-rank pieces ([CaS] "Factorization at scale" and
+ * "Scale-out": S sharded by rows across GPUs, H replicated, the S H products
+ * local, O(n k) exchanged per iteration).  Rank p holds rows [row0, row0 + rows)
+ * of S (rows x n, row pitch lds, a multiple of 4, 16-byte aligned) and the
+ * whole current iterate H (n x k).  The caller runs the loop and the
+ * collectives (symmetric_nmf_clustering_b200.sharded does it over
+ * torch.distributed); these calls never wait on another rank.
+ *
+ * symnmf_stats_rows: out_dev[0..2] = (sum, squared norm, non-finite count) of
+ *   the block, fp64, as symnmf_stats; summed over the ranks they are those of
+ *   S.  Workspace: symnmf_workspace_size(SYMNMF_OP_STATS, ...).
+ *   Asynchronous.
+ * symnmf_seeded_init: H (n x k) = the scale-matched seeded start of
+ *   symnmf_fit (INIT_SEEDED) for a matrix whose entries sum to s_sum.
+ *   Every rank draws the same H.  Asynchronous.
+ * symnmf_gram: A_dev (k x k, device, fp64) = H^T H over `rows` rows of H, a
+ *   fixed-order sum (bitwise reproducible).  Workspace: (rows/128 + 1) *
+ *   (k^2 + 1) doubles, rounded up.  Asynchronous.
+ * symnmf_shard_step: one full-batch iteration restricted to the block, with
+ *   A_dev = H^T H of the current iterate (the sum of every rank's Gram):
+ *   P = S[rows, :] H; the rows of the projected AdaGrad step of symnmf_fit
+ *   ([CaS] "Factorizing with SymNMF") go to H_rows_next and G_rows_next
+ *   (rows x k each; G_rows is the accumulator of those rows before the step);
+ *   partial_dev (k^2 + 1 doubles, device) = (Gram of the new rows, then
+ *   sum_{i in rows} H_i . P_i).  Summed over the ranks, partial_dev gives the
+ *   next Gram and tr(H^T S H), and f(H) = ||S||^2 - 2 tr + ||A||_F^2.  Reads
+ *   the whole of H (its split operand); H_rows_next must not alias H.
+ *   Workspace: symnmf_shard_workspace_size(rows, n, k).  Synchronises `stream`
+ *   (reads the device error word: SYMNMF_ERR_TIMEOUT when a bounded wait gave up).
+ */
+SYMNMF_API int symnmf_stats_rows(const float* S, int64_t rows, int64_t n, int64_t lds,
+                                 double* out_dev, void* ws, size_t ws_bytes,
+                                 symnmf_stream_t stream);
+SYMNMF_API int symnmf_seeded_init(float* H, int64_t n, int k, uint64_t seed, double s_sum,
+                                  symnmf_stream_t stream);
+SYMNMF_API int symnmf_gram(const float* H, int64_t rows, int k, double* A_dev, void* ws,
+                           size_t ws_bytes, symnmf_stream_t stream);
+SYMNMF_API int symnmf_shard_workspace_size(int64_t rows, int64_t n, int k, size_t* bytes);
+SYMNMF_API int symnmf_shard_step(const float* S_rows, int64_t rows, int64_t n, int64_t lds,
+                                 int64_t row0, int k, const float* H, const double* A_dev,
+                                 const float* G_rows, float lr, float eps, float* H_rows_next,
+                                 float* G_rows_next, double* partial_dev, void* ws,
+                                 size_t ws_bytes, symnmf_stream_t stream);
+
+/*
  * What the last symnmf_spectral_probe call on this host thread did: the
  * number of passes over S it launched (each reads the n x n matrix once,
  * with a block-wide operand) and the kernels it launched in all.  Lets a

@@ -138,6 +138,12 @@ SIGNATURES = {
     "symnmf_spectral_probe": (_int, [_vp, _i64, _i64, _int, _int, _int, C.c_double, C.c_uint64,
                                      C.POINTER(C.c_double), _vp, _sz, _vp]),
     "symnmf_probe_last_info": (_int, [C.POINTER(ProbeInfo)]),
+    "symnmf_stats_rows": (_int, [_vp, _i64, _i64, _i64, _vp, _vp, _sz, _vp]),
+    "symnmf_seeded_init": (_int, [_vp, _i64, _int, C.c_uint64, C.c_double, _vp]),
+    "symnmf_gram": (_int, [_vp, _i64, _int, _vp, _vp, _sz, _vp]),
+    "symnmf_shard_workspace_size": (_int, [_i64, _i64, _int, C.POINTER(_sz)]),
+    "symnmf_shard_step": (_int, [_vp, _i64, _i64, _i64, _i64, _int, _vp, _vp, _vp, C.c_float,
+                                 C.c_float, _vp, _vp, _vp, _vp, _sz, _vp]),
     "symnmf_fit": (_int, [_vp, _i64, _i64, _int, C.POINTER(FitParams), _vp, C.POINTER(FitStats),
                           _vp, _sz, _vp]),
     "symnmf_labels": (_int, [_vp, _i64, _int, _vp, _vp]),

@@ -688,7 +688,7 @@ static int fit_impl(const float* S, int64_t n, int64_t lds, int k, const symnmf_
 
     // statistics pre-pass into the state head
     SYMNMF_CUDA_TRY(cudaMemsetAsync(c.L.st, 0, fit_state_bytes(), s));
-    SYMNMF_TRY(launch_stats(S, n, lds, c.L.stats_part, stats_blocks(), &c.L.st->s_sum, s));
+    SYMNMF_TRY(launch_stats(S, n, n, lds, c.L.stats_part, stats_blocks(), &c.L.st->s_sum, s));
     HostState hs;
     SYMNMF_TRY(read_state(c.L.st, &hs, s));
     if (hs.s_bad > 0.0) {
@@ -1410,7 +1410,7 @@ int symnmf_stats(const float* S, int64_t n, int64_t lds, double* out_dev, void* 
         set_error("workspace too small: %zu given, %zu needed", ws_bytes, a.used);
         return SYMNMF_ERR_WORKSPACE;
     }
-    return launch_stats(S, n, lds, part, stats_blocks(), out_dev, (cudaStream_t)stream);
+    return launch_stats(S, n, n, lds, part, stats_blocks(), out_dev, (cudaStream_t)stream);
 }
 
 int symnmf_sh(const float* S, int64_t n, int64_t lds, const float* X, int k, float* Y, void* ws,

@@ -126,7 +126,8 @@ size_t fit_state_bytes();
 // Tensor-core S-stream (stream_tc.cu): X enters as its exact TF32 split
 // XT = [X_hi; X_lo] stored K-major (2*KP rows of length ldxt, KP = k rounded up to 8).
 struct TcPlan {
-    int64_t n;
+    int64_t n;        // rows of the output (rows of S read)
+    int64_t ncols;    // columns of S (the contraction's extent)
     int k, KP;
     int64_t j0, j1;   // contraction range, j0 a multiple of 32
     int64_t tiles;    // 128-row tiles of the output
@@ -134,6 +135,8 @@ struct TcPlan {
     int64_t jspan;    // columns per split (multiple of 32)
 };
 TcPlan plan_stream_tc(const Dev& d, int64_t n, int k, int64_t j0, int64_t j1);
+// a block of `rows` rows of S (all ncols columns): S[r0 + i, :] X for i < rows
+TcPlan plan_stream_tc_rows(const Dev& d, int64_t rows, int64_t ncols, int k);
 size_t tc_partial_floats(const TcPlan& p);
 struct EpiArgs;
 // epi != NULL: the last split CTA of each row tile runs the epilogue in place
@@ -179,9 +182,10 @@ int launch_finalize(int mode, int nblk, int k, const double* tr_part,
                     int max_evals, double* history, int history_cap,
                     cudaStream_t s);
 
-int launch_stats(const float* S, int64_t n, int64_t lds, double* part, int nblk,
+int launch_stats(const float* S, int64_t rows, int64_t n, int64_t lds, double* part, int nblk,
                  double* out3, cudaStream_t s);
 int stats_blocks();
+int launch_init_sum(float* H, int64_t n, int k, uint64_t seed, double s_sum, cudaStream_t s);
 int launch_init(float* H, int64_t n, int k, uint64_t seed, const FitState* st,
                 cudaStream_t s);
 int launch_labels(const float* H, int64_t n, int k, int32_t* labels, cudaStream_t s);

@@ -31,11 +31,11 @@ constexpr int STATS_THREADS = 256;
 int stats_blocks() { return STATS_BLOCKS; }
 
 __global__ void __launch_bounds__(STATS_THREADS)
-stats_partial_kernel(const float* __restrict__ S, int64_t n, int64_t lds,
+stats_partial_kernel(const float* __restrict__ S, int64_t rows, int64_t n, int64_t lds,
                      double* __restrict__ part) {
     double sum = 0.0, sq = 0.0, bad = 0.0;
     const int64_t n4 = n >> 2;
-    for (int64_t r = blockIdx.x; r < n; r += gridDim.x) {
+    for (int64_t r = blockIdx.x; r < rows; r += gridDim.x) {
         const float4* row = reinterpret_cast<const float4*>(S + r * lds);
         constexpr int U = 4;  // loads in flight per thread
         for (int64_t q0 = threadIdx.x; q0 < n4; q0 += (int64_t)U * blockDim.x) {
@@ -126,9 +126,9 @@ __global__ void stats_final_kernel(const double* __restrict__ part, int nblk,
     if (threadIdx.x < 3) out3[threadIdx.x] = red[threadIdx.x][0];
 }
 
-int launch_stats(const float* S, int64_t n, int64_t lds, double* part, int nblk,
+int launch_stats(const float* S, int64_t rows, int64_t n, int64_t lds, double* part, int nblk,
                  double* out3, cudaStream_t s) {
-    stats_partial_kernel<<<nblk, STATS_THREADS, 0, s>>>(S, n, lds, part);
+    stats_partial_kernel<<<nblk, STATS_THREADS, 0, s>>>(S, rows, n, lds, part);
     SYMNMF_LAUNCH_CHECK();
     stats_final_kernel<<<1, STATS_THREADS, 0, s>>>(part, nblk, out3);
     SYMNMF_LAUNCH_CHECK();
@@ -147,6 +147,26 @@ __global__ void init_kernel(float* __restrict__ H, int64_t count, int k, int64_t
     for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < count;
          e += (int64_t)gridDim.x * blockDim.x)
         H[e] = sm64_uniform(seed, (uint64_t)e) * c;
+}
+
+// Same draw with the sum of S given by the caller (a row-sharded fit gets it
+// from an all-reduce of every shard's statistics).
+__global__ void init_sum_kernel(float* __restrict__ H, int64_t count, int k, int64_t n,
+                                uint64_t seed, double s_sum) {
+    const double mean = s_sum / ((double)n * (double)n);
+    const float c = (float)sqrt(fmax(mean, 0.0) / (double)k);
+    for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < count;
+         e += (int64_t)gridDim.x * blockDim.x)
+        H[e] = sm64_uniform(seed, (uint64_t)e) * c;
+}
+
+int launch_init_sum(float* H, int64_t n, int k, uint64_t seed, double s_sum, cudaStream_t s) {
+    const int64_t count = n * k;
+    const int threads = 256;
+    const int64_t blocks = min64((count + threads - 1) / threads, 4096);
+    init_sum_kernel<<<(unsigned)blocks, threads, 0, s>>>(H, count, k, n, seed, s_sum);
+    SYMNMF_LAUNCH_CHECK();
+    return SYMNMF_OK;
 }
 
 int launch_init(float* H, int64_t n, int k, uint64_t seed, const FitState* st,

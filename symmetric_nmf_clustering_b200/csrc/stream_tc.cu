@@ -468,6 +468,7 @@ int make_map(CUtensorMap* m, const float* base, int64_t cols, int64_t rows, int6
 TcPlan plan_stream_tc(const Dev& d, int64_t n, int k, int64_t j0, int64_t j1) {
     TcPlan p;
     p.n = n;
+    p.ncols = n;
     p.k = k;
     p.KP = (k + 7) / 8 * 8;
     p.j0 = j0 / TC_BK * TC_BK;                                 // 128-byte aligned TMA x
@@ -494,6 +495,31 @@ TcPlan plan_stream_tc(const Dev& d, int64_t n, int k, int64_t j0, int64_t j1) {
     return p;
 }
 
+TcPlan plan_stream_tc_rows(const Dev& d, int64_t rows, int64_t ncols, int k) {
+    // the split choice depends on the row tiles and the contraction length only
+    TcPlan p = plan_stream_tc(d, ncols, k, 0, ncols);
+    p.n = rows;
+    p.ncols = ncols;
+    p.tiles = (rows + TC_BM - 1) / TC_BM;
+    const int64_t steps = std::max<int64_t>(1, (p.j1 - p.j0 + TC_BK - 1) / TC_BK);
+    const int64_t slots = (int64_t)d.sms * 2;
+    int best = 1;
+    double best_waste = 1e30;
+    for (int sp = 1; sp <= 32; ++sp) {
+        if (sp > 1 && steps / sp < 8) break;
+        const int64_t ctas = p.tiles * sp;
+        const int64_t waves = (ctas + slots - 1) / slots;
+        const double waste = (double)(waves * slots) / (double)ctas - 1.0 + 0.002 * sp;
+        if (waste < best_waste - 1e-12) {
+            best_waste = waste;
+            best = sp;
+        }
+    }
+    p.splits = best;
+    p.jspan = (steps + best - 1) / best * TC_BK;
+    return p;
+}
+
 size_t tc_partial_floats(const TcPlan& p) { return (size_t)p.splits * p.n * p.k; }
 
 int launch_stream_tc(const TcPlan& p, const float* S, int64_t lds, const float* XT, int64_t ldxt,
@@ -505,8 +531,8 @@ int launch_stream_tc(const TcPlan& p, const float* S, int64_t lds, const float* 
     const EpiArgs ea = epi != nullptr ? *epi : none;
     int* cnt = epi != nullptr ? counters : nullptr;
     CUtensorMap mapS, mapX;
-    SYMNMF_TRY(make_map(&mapS, S, p.n, p.n, lds, TC_BM));
-    SYMNMF_TRY(make_map(&mapX, XT, p.n, 2 * p.KP, ldxt, (uint32_t)(2 * p.KP)));
+    SYMNMF_TRY(make_map(&mapS, S, p.ncols, p.n, lds, TC_BM));
+    SYMNMF_TRY(make_map(&mapX, XT, p.ncols, 2 * p.KP, ldxt, (uint32_t)(2 * p.KP)));
     dim3 grid((unsigned)p.tiles, (unsigned)p.splits);
 #define SYMNMF_TC(KP)                                                                         \
     do {                                                                                      \
