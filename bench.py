@@ -303,6 +303,25 @@ def measure_rows(m, torch, dev, S, H0, lab, n, k, T, rank, workload, planted=Non
     out["kmeans_S_GBs"] = (2 * ksteps - (1 if kconv else 0)) * 4.0 * n * n / (ms / 1e3) / 1e9
     out["kmeans_vs_symnmf_ARI"] = m.ari(klab, lab, k)[0]
     del wsk
+    # the upper-triangle S-stream (upper_only = 1): the same fit reading only the
+    # 128 x 128 tiles on or above the diagonal (S rounded to TF32 in the product)
+    if k <= 24:
+        pu = m.fit_params(max_iters=19, rel_tol=0.0, upper_only=1, timing=1)
+        wsu = m.workspace(m._lib.OP_FIT, n, k, params=pu, device=dev)
+        Hu = H0.clone()
+        m.fit(S, k, H0=Hu, out=Hu, max_iters=2, rel_tol=0.0, upper_only=True, ws=wsu)   # warm-up
+        Hu.copy_(H0)
+        ms, (_, stu) = _timed(torch, lambda: m.fit(S, k, H0=Hu, out=Hu, max_iters=19, rel_tol=0.0,
+                                                  upper_only=True, timing=True, ws=wsu))
+        T = (n + 127) // 128
+        tile_bytes = 4.0 * 128 * 128 * T * (T + 1) / 2      # the tiles read per pass
+        kms = stu["stream_ms"] / max(stu["stream_launches"], 1)
+        out["upper_triangle"] = {
+            "iterations_per_s": 20 / (ms / 1e3), "ms_per_iteration": ms / 20,
+            "tri_kernel_ms": kms, "tile_bytes_read": tile_bytes,
+            "tri_kernel_GBs_over_bytes_read": (tile_bytes + 4.0 * n * k) / (kms / 1e3) / 1e9,
+            "loss_after_19": stu["loss"]}
+        del wsu, Hu
     # the |corr| workload to convergence: full-batch AdaGrad until the loss
     # changes by less than 1e-5 (cap 20,000 passes)
     if planted is not None:
@@ -406,6 +425,11 @@ def row_rooflines(rows, n, k, T, hbm_peak):
             gbs = bytes_ / (ms / 1e3) / 1e9
             out[name] = {"bound": "hbm", "GBs": gbs, "frac": gbs / hbm_peak}
     hbm("stats", sbytes, rows.get("stats_ms"))
+    if "upper_triangle" in rows:
+        u = rows["upper_triangle"]
+        out["upper_triangle_stream"] = {"bound": "hbm", "GBs": u["tri_kernel_GBs_over_bytes_read"],
+                                        "frac": u["tri_kernel_GBs_over_bytes_read"] / hbm_peak,
+                                        "bytes": "tiles on or above the diagonal (about 2 n^2) + X"}
     if "probe_s_passes" in rows:
         hbm("probe", rows["probe_s_passes"] * sbytes, rows.get("probe_ms"))
     if "kmeans_steps" in rows:
