@@ -2,6 +2,7 @@
 // full-batch loop, Block-SVRG with AdaptGrow growth, AUTO solver selection
 // and the block-Lanczos spectral probe.  Every arithmetic step on n-sized
 // data runs in the kernels of stream.cu, misc.cu and builders.cu.
+#include <chrono>
 #include <cmath>
 #include <cstdarg>
 #include <cstdlib>
@@ -998,6 +999,15 @@ static int probe_impl(const Dev& d, const float* S, int64_t n, int64_t lds, int 
                                       cudaMemcpyDeviceToDevice, s));
     SYMNMF_TRY(orthonormalize(L, L.Q, n, ldq, b, L.Q, ldq, 0, seed + 1, B, s));
     bool converged = false;
+    // The Rayleigh-Ritz step costs O(nq^3) on the host and overlaps the next
+    // block's S pass.  While it is shorter than a block step it runs every
+    // step; when it grows longer (large bases on small matrices), the check
+    // is spaced out so that the host work stays within half of the block
+    // steps' time.  The last step always computes it (it is the result).
+    using clk = std::chrono::steady_clock;
+    double rr_ms = 0.0, step_ms = 0.0;
+    int next_check = 0;
+    auto step_t0 = clk::now();
     // W = S Q_0 (one S pass)
     SYMNMF_TRY(stream_pass(d, sa, L.Q, nullptr, ldq, 0, n, false, epi_product(n, b, L.W), s, nullptr));
     g_probe_info.s_passes = 1;
@@ -1036,7 +1046,10 @@ static int probe_impl(const Dev& d, const float* S, int64_t n, int64_t lds, int 
             g_probe_info.s_passes += 1;
         }
         // Rayleigh-Ritz on the leading nq x nq block of the block tridiagonal T
-        if (nq >= n_eig) {
+        const auto now = clk::now();
+        step_ms = std::chrono::duration<double, std::milli>(now - step_t0).count();
+        if (nq >= n_eig && (!more || j >= next_check)) {
+            const auto r0 = clk::now();
             std::vector<double> sub((size_t)nq * nq);
             for (int r = 0; r < nq; ++r)
                 for (int c2 = 0; c2 < nq; ++c2) sub[(size_t)r * nq + c2] = T[(size_t)r * mtot + c2];
@@ -1047,7 +1060,11 @@ static int probe_impl(const Dev& d, const float* S, int64_t n, int64_t lds, int 
                 if (dmax <= tol * std::fabs(theta[0])) converged = true;
             }
             prev = theta;
+            rr_ms = std::chrono::duration<double, std::milli>(clk::now() - r0).count();
+            const int gap = step_ms > 0.0 ? (int)std::ceil(rr_ms / (0.5 * step_ms)) : 1;
+            next_check = j + std::max(1, gap);
         }
+        step_t0 = clk::now();
         if (converged || !more) break;
     }
     {
