@@ -150,6 +150,7 @@ struct TriPlan {
     int64_t n;
     int k, KP;
     int T;            // 128-row tiles
+    int C;            // column tiles per work item
     int items;        // work items (panel x run of column tiles)
     int grid;         // persistent CTAs
     int64_t tslabs;   // transposed partial slabs

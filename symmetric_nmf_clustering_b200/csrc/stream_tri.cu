@@ -28,7 +28,7 @@
 // forward MMA.
 //
 // Work decomposition.  Row tiles are grouped in panels of TR_PANEL; a work
-// item is one panel times a run of TR_CHUNK column tiles q >= the panel's
+// item is one panel times a run of C column tiles q >= the panel's
 // first row tile, visited q-outer, p-inner (p <= q).  Per tile pair both
 // accumulators are drained into registers: forward rows accumulate over the
 // item in registers (one partial slab per item and panel row), transposed
@@ -67,7 +67,7 @@ __device__ int g_tri_stall = 0;
 constexpr int TR_BM = 128;         // tile edge
 constexpr int TR_BK = 32;          // columns per TMA box (128 bytes of fp32)
 constexpr int TR_PANEL = 4;        // row tiles per panel
-constexpr int TR_CHUNK = 16;       // column tiles per work item
+constexpr int TR_CHUNK_MAX = 16;   // column tiles per work item (fewer when the items would be too few)
 constexpr int TR_THREADS = 256;
 #ifndef SYMNMF_TRI_PREFETCH
 #define SYMNMF_TRI_PREFETCH 4
@@ -95,8 +95,8 @@ struct TrCfg {
 };
 
 // ---------------------------------------------------------------- schedule
-__host__ __device__ __forceinline__ int tr_chunks(int T, int P) {
-    return (T - TR_PANEL * P + TR_CHUNK - 1) / TR_CHUNK;
+__host__ __device__ __forceinline__ int tr_chunks(int T, int C, int P) {
+    return (T - TR_PANEL * P + C - 1) / C;
 }
 // index of the transposed slab of panel P and column tile q (q >= TR_PANEL P):
 // panels' slabs are stored one after another, panel P holding T - 4P of them
@@ -107,14 +107,14 @@ __host__ __device__ __forceinline__ int tr_panels(int T) { return (T + TR_PANEL 
 
 // geometry of work item `item`; (P, pbase) advance monotonically over calls
 // with increasing items
-__device__ __forceinline__ void tr_item(int T, int item, int& P, int& pbase, int& qa, int& qb,
-                                        int& pr0, int& pr1) {
-    while (item >= pbase + tr_chunks(T, P)) {
-        pbase += tr_chunks(T, P);
+__device__ __forceinline__ void tr_item(int T, int C, int item, int& P, int& pbase, int& qa,
+                                        int& qb, int& pr0, int& pr1) {
+    while (item >= pbase + tr_chunks(T, C, P)) {
+        pbase += tr_chunks(T, C, P);
         ++P;
     }
-    qa = TR_PANEL * P + (item - pbase) * TR_CHUNK;
-    qb = min(T, qa + TR_CHUNK);
+    qa = TR_PANEL * P + (item - pbase) * C;
+    qb = min(T, qa + C);
     pr0 = TR_PANEL * P;
     pr1 = min(T, pr0 + TR_PANEL);
 }
@@ -122,10 +122,11 @@ __device__ __forceinline__ void tr_item(int T, int item, int& P, int& pbase, int
 // A position in a CTA's sequence of tile pairs (items b, b + G, ...; q-outer,
 // p-inner), advanced one tile pair at a time.
 struct TrCursor {
-    int T, items, stride, item, P, pbase, qa, qb, pr0, pr1, q, p;
+    int T, C, items, stride, item, P, pbase, qa, qb, pr0, pr1, q, p;
     bool valid;
-    __device__ __forceinline__ void start(int T_, int items_, int first, int stride_) {
+    __device__ __forceinline__ void start(int T_, int C_, int items_, int first, int stride_) {
         T = T_;
+        C = C_;
         items = items_;
         stride = stride_;
         item = first;
@@ -133,7 +134,7 @@ struct TrCursor {
         pbase = 0;
         valid = item < items;
         if (valid) {
-            tr_item(T, item, P, pbase, qa, qb, pr0, pr1);
+            tr_item(T, C, item, P, pbase, qa, qb, pr0, pr1);
             q = qa;
             p = pr0;
         }
@@ -147,7 +148,7 @@ struct TrCursor {
         item += stride;
         valid = item < items;
         if (!valid) return;
-        tr_item(T, item, P, pbase, qa, qb, pr0, pr1);
+        tr_item(T, C, item, P, pbase, qa, qb, pr0, pr1);
         q = qa;
         p = pr0;
     }
@@ -164,8 +165,8 @@ __device__ __forceinline__ uint64_t tr_desc(uint32_t saddr) { return sm100::umma
 template <int KP>
 __global__ void __launch_bounds__(TR_THREADS, 1)
 stream_tri_kernel(const __grid_constant__ CUtensorMap mapS, const __grid_constant__ CUtensorMap mapX,
-                  int T, int items, int k, float* __restrict__ tpart, float* __restrict__ fpart,
-                  int* __restrict__ err, const FitState* st) {
+                  int T, int C, int items, int k, float* __restrict__ tpart,
+                  float* __restrict__ fpart, int* __restrict__ err, const FitState* st) {
     using Cfg = TrCfg<KP>;
     using namespace sm100;
     pdl_wait();
@@ -215,14 +216,14 @@ stream_tri_kernel(const __grid_constant__ CUtensorMap mapS, const __grid_constan
         // loads into the two shared-memory slots find them there: the HBM
         // latency is covered without more shared memory
         TrCursor ahead;
-        ahead.start(T, items, blockIdx.x, gridDim.x);
+        ahead.start(T, C, items, blockIdx.x, gridDim.x);
         for (int d = 0; d < TR_PREFETCH && ahead.valid; ++d, ahead.next())
             for (int s = 0; s < 4; ++s) tma_prefetch_2d(&mapS, ahead.q * TR_BM + s * TR_BK, ahead.p * TR_BM);
         uint32_t u = 0, g = 0;   // tile pairs and column groups issued so far
         int P = 0, pbase = 0;
         for (int item = blockIdx.x; item < items && !abort_sh; item += gridDim.x) {
             int qa, qb, pr0, pr1;
-            tr_item(T, item, P, pbase, qa, qb, pr0, pr1);
+            tr_item(T, C, item, P, pbase, qa, qb, pr0, pr1);
             for (int q = qa; q < qb && !abort_sh; ++q) {
                 const uint32_t xs = g & 1u;
                 if (g >= 2 && !mbar_wait(&b_xqfree[xs], ((g - 2) >> 1) & 1u)) {
@@ -276,7 +277,7 @@ stream_tri_kernel(const __grid_constant__ CUtensorMap mapS, const __grid_constan
         bool ok = true;
         for (int item = blockIdx.x; item < items && ok; item += gridDim.x) {
             int qa, qb, pr0, pr1;
-            tr_item(T, item, P, pbase, qa, qb, pr0, pr1);
+            tr_item(T, C, item, P, pbase, qa, qb, pr0, pr1);
             for (int q = qa; q < qb && ok; ++q, ++g) {
                 const uint32_t xs = g & 1u;
                 const int pe = min(pr1, q + 1);
@@ -317,7 +318,7 @@ stream_tri_kernel(const __grid_constant__ CUtensorMap mapS, const __grid_constan
         bool ok = true;
         for (int item = blockIdx.x; item < items && ok; item += gridDim.x) {
             int qa, qb, pr0, pr1;
-            tr_item(T, item, P, pbase, qa, qb, pr0, pr1);
+            tr_item(T, C, item, P, pbase, qa, qb, pr0, pr1);
             for (int q = qa; q < qb && ok; ++q) {
                 const int pe = min(pr1, q + 1);
                 for (int p = pr0; p < pe; ++p, ++u) {
@@ -429,7 +430,7 @@ stream_tri_kernel(const __grid_constant__ CUtensorMap mapS, const __grid_constan
         int P = 0, pbase = 0;
         for (int item = blockIdx.x; item < items && alive; item += gridDim.x) {
             int qa, qb, pr0, pr1;
-            tr_item(T, item, P, pbase, qa, qb, pr0, pr1);
+            tr_item(T, C, item, P, pbase, qa, qb, pr0, pr1);
             for (int q = qa; q < qb && alive; ++q) {
                 const int pe = min(pr1, q + 1);
                 for (int p = pr0; p < pe; ++p, ++u) {
@@ -514,7 +515,7 @@ constexpr int TR_RED_THREADS = 256;
 constexpr int TR_RED_BATCH = 8;
 
 __global__ void __launch_bounds__(TR_RED_THREADS)
-tri_reduce_kernel(int T, int64_t n, int k, const float* __restrict__ tpart,
+tri_reduce_kernel(int T, int C, int64_t n, int k, const float* __restrict__ tpart,
                   const float* __restrict__ fpart, float* __restrict__ Y, const FitState* st) {
     pdl_wait();
     pdl_trigger();
@@ -525,8 +526,8 @@ tri_reduce_kernel(int T, int64_t n, int k, const float* __restrict__ tpart,
     if (e >= rows * k) return;
     const int P = t / TR_PANEL, pp = t % TR_PANEL;
     int ib = 0;
-    for (int Q = 0; Q < P; ++Q) ib += tr_chunks(T, Q);
-    const int nf = tr_chunks(T, P), nt = P + 1, ns = nf + nt;
+    for (int Q = 0; Q < P; ++Q) ib += tr_chunks(T, C, Q);
+    const int nf = tr_chunks(T, C, P), nt = P + 1, ns = nf + nt;
     const int64_t slab = (int64_t)TR_BM * k;
     // source of the s-th term: forward slabs first, then transposed slabs
     auto src = [&](int s2) -> const float* {
@@ -556,14 +557,19 @@ TriPlan plan_stream_tri(const Dev& d, int64_t n, int k) {
     p.KP = (k + 7) / 8 * 8;
     p.T = (int)((n + TR_BM - 1) / TR_BM);
     const int TP = tr_panels(p.T);
-    int64_t items = 0, slabs = 0;
-    for (int P = 0; P < TP; ++P) {
-        items += tr_chunks(p.T, P);
-        slabs += p.T - TR_PANEL * P;
-    }
-    p.items = (int)items;
+    // the widest items that still give every SM at least four of them
+    auto count = [&](int C) {
+        int64_t c = 0;
+        for (int P = 0; P < TP; ++P) c += tr_chunks(p.T, C, P);
+        return c;
+    };
+    p.C = TR_CHUNK_MAX;
+    while (p.C > 1 && count(p.C) < 4 * (int64_t)d.sms) p.C /= 2;
+    int64_t slabs = 0;
+    for (int P = 0; P < TP; ++P) slabs += p.T - TR_PANEL * P;
+    p.items = (int)count(p.C);
     p.tslabs = slabs;
-    p.grid = (int)std::min<int64_t>(items, d.sms);
+    p.grid = (int)std::min<int64_t>(p.items, d.sms);
     return p;
 }
 
@@ -588,7 +594,7 @@ int launch_stream_tri(const TriPlan& p, const float* S, int64_t lds, const float
             kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)TrCfg<KP>::SMEM);         \
         SYMNMF_CUDA_TRY(attr_rc);                                                             \
         SYMNMF_CUDA_TRY(launch_pdl(kern, dim3(p.grid), dim3(TR_THREADS), TrCfg<KP>::SMEM, s,  \
-                                   mapS, mapX, p.T, p.items, p.k, tpart, fpart, err, st));    \
+                                   mapS, mapX, p.T, p.C, p.items, p.k, tpart, fpart, err, st)); \
     } while (0)
     switch (p.KP) {
         case 8: SYMNMF_TRI(8); break;
@@ -603,8 +609,8 @@ int launch_stream_tri(const TriPlan& p, const float* S, int64_t lds, const float
 int launch_tri_reduce(const TriPlan& p, const float* tpart, const float* fpart, float* Y,
                       const FitState* st, cudaStream_t s) {
     const dim3 grid((unsigned)p.T, (unsigned)((TR_BM * p.k + TR_RED_THREADS - 1) / TR_RED_THREADS));
-    SYMNMF_CUDA_TRY(launch_pdl(tri_reduce_kernel, grid, dim3(TR_RED_THREADS), 0, s, p.T, p.n, p.k,
-                               tpart, fpart, Y, st));
+    SYMNMF_CUDA_TRY(launch_pdl(tri_reduce_kernel, grid, dim3(TR_RED_THREADS), 0, s, p.T, p.C, p.n,
+                               p.k, tpart, fpart, Y, st));
     SYMNMF_LAUNCH_CHECK();
     return SYMNMF_OK;
 }
