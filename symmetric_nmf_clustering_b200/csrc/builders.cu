@@ -5,15 +5,14 @@
 // Both end in a symmetric Gram S = c * op(Z^T Z) over the day index, computed
 // by one tiled kernel with the builder's epilogue (abs + unit diagonal for
 // correlation, the n/N scale for TPDM).
+#include <cuda_fp16.h>
+
 #include <cstdlib>
 #include <cstring>
 
 #include "common.cuh"
 
 namespace symnmf {
-
-int launch_gram_tc(const float* ZF, const float* ZL, int64_t n, int64_t n_pad, int64_t Kp,
-                   bool corr, float scale, float* S, int64_t lds, int* err, cudaStream_t s);
 
 // Tensor-core Gram by default; SYMNMF_STREAM=cuda_core selects the CUDA-core one.
 static bool builders_tc() {
@@ -24,7 +23,8 @@ static bool builders_tc() {
     return v;
 }
 constexpr int TCB_ROWS = 128;   // row padding of the transposed operands
-constexpr int TCB_K = 32;       // contraction padding of the transposed operands
+constexpr int TCB_K = 32;       // contraction padding of the transposed fp32 operands (TPDM)
+constexpr int TCB_K16 = 64;     // contraction padding of the transposed fp16 operands (|corr|)
 
 constexpr int GB = 128;   // Gram output tile (GB x GB)
 constexpr int GK = 16;    // day-slab per stage
@@ -152,9 +152,10 @@ int corr_plan(Arena& a, int64_t T, int64_t n, double** mu, double** inv, float**
     const int64_t Kp = round_up(T, GK);
     *mu = a.take<double>(n);
     *inv = a.take<double>(n);
-    // CUDA-core layout: Z (Kp x ldz); tensor-core layout: Z^T planes (n_pad x Kt) x 2 + err
+    // CUDA-core layout: Z (Kp x ldz) floats; tensor-core layout: two fp16 Z^T
+    // planes (n_pad x Kt) + err, counted in floats
     const size_t cc = (size_t)Kp * *ldz;
-    const size_t tc = 2 * (size_t)round_up(n, TCB_ROWS) * round_up(T, TCB_K) + 64;
+    const size_t tc = (size_t)round_up(n, TCB_ROWS) * round_up(T, TCB_K16) + 64;
     *Z = a.take<float>(std::max(cc, tc));
     return SYMNMF_OK;
 }
@@ -192,13 +193,16 @@ __global__ void normalize_kernel(const float* __restrict__ R, int64_t T, int64_t
     }
 }
 
-// Z^T planes for the tensor-core Gram: ZF[i][t] = z_ti (fp32) and
-// ZL[i][t] = z_ti - trunc_tf32(z_ti), zero in the padding (i >= n, t >= T).
+// Z^T planes for the tensor-core Gram, in fp16 and scaled by c = CORR_F16_SCALE:
+// ZH[i][t] = rn16(c z_ti) and ZL[i][t] = rn16(c z_ti - ZH[i][t]), zero in the
+// padding (i >= n, t >= T).  |c z| <= 2^14, so neither part overflows; the pair
+// carries c z to within 2^-22 of its magnitude (each rounding to nearest loses
+// at most 2^-11 of what it rounds, and the remainder is at most 2^-11 c |z|).
 // 32 x 32 tiles through shared memory: coalesced reads of R rows, writes of ZT rows.
 __global__ void normalize_t_kernel(const float* __restrict__ R, int64_t T, int64_t n,
                                    int64_t ldr, const double* __restrict__ mu,
-                                   const double* __restrict__ inv, float* __restrict__ ZF,
-                                   float* __restrict__ ZL, int64_t Kt) {
+                                   const double* __restrict__ inv, __half* __restrict__ ZH,
+                                   __half* __restrict__ ZL, int64_t Kt) {
     __shared__ float tile[32][33];
     const int64_t t0 = (int64_t)blockIdx.y * 32, i0 = (int64_t)blockIdx.x * 32;
     const int tx = threadIdx.x, ty = threadIdx.y;     // 32 x 8
@@ -211,10 +215,10 @@ __global__ void normalize_t_kernel(const float* __restrict__ R, int64_t T, int64
     __syncthreads();
     for (int r = ty; r < 32; r += 8) {
         const int64_t i = i0 + r, t = t0 + tx;
-        const float z = tile[tx][r];
-        const float hi = __uint_as_float(__float_as_uint(z) & 0xFFFFE000u);
-        ZF[i * Kt + t] = z;
-        ZL[i * Kt + t] = z - hi;
+        const float zs = tile[tx][r] * CORR_F16_SCALE;     // exact: a power of two
+        const __half hi = __float2half_rn(zs);
+        ZH[i * Kt + t] = hi;
+        ZL[i * Kt + t] = __float2half_rn(zs - __half2float(hi));   // the difference is exact in fp32
     }
 }
 
@@ -237,15 +241,15 @@ int launch_corr(const float* R, int64_t T, int64_t n, int64_t ldr, float* S,
     colstats_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(R, T, n, ldr, mu, inv);
     SYMNMF_LAUNCH_CHECK();
     if (builders_tc()) {
-        const int64_t n_pad = round_up(n, TCB_ROWS), Kt = round_up(T, TCB_K);
-        float* ZF = Z;
-        float* ZL = Z + (size_t)n_pad * Kt;
+        const int64_t n_pad = round_up(n, TCB_ROWS), Kt = round_up(T, TCB_K16);
+        __half* ZH = reinterpret_cast<__half*>(Z);
+        __half* ZL = ZH + (size_t)n_pad * Kt;
         int* err = reinterpret_cast<int*>(ZL + (size_t)n_pad * Kt);
         SYMNMF_CUDA_TRY(cudaMemsetAsync(err, 0, sizeof(int), s));
         dim3 grid((unsigned)(n_pad / 32), (unsigned)(Kt / 32));
-        normalize_t_kernel<<<grid, dim3(32, 8), 0, s>>>(R, T, n, ldr, mu, inv, ZF, ZL, Kt);
+        normalize_t_kernel<<<grid, dim3(32, 8), 0, s>>>(R, T, n, ldr, mu, inv, ZH, ZL, Kt);
         SYMNMF_LAUNCH_CHECK();
-        SYMNMF_TRY(launch_gram_tc(ZF, ZL, n, n_pad, Kt, true, 1.f, S, lds, err, s));
+        SYMNMF_TRY(launch_gram_tc(ZH, ZL, n, n_pad, Kt, true, 1.f, S, lds, err, s));
         return gram_status(err, s);
     }
     const int64_t Kp = round_up(T, GK);

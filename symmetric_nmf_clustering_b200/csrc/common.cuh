@@ -206,6 +206,13 @@ int launch_normalize_centroids(const float* Z, int64_t n, int k, double* part, f
 int launch_label_change(const int32_t* lab, int32_t* old, int64_t n, int* count, cudaStream_t s);
 
 // builders
+// Tensor-core Gram (gram_tc.cu) of the K-major operand planes F (hi parts) and
+// L (remainders), n_pad x Kp each.  |corr| (corr = true): fp16 planes holding
+// z * CORR_F16_SCALE, Kp a multiple of 64; TPDM: fp32 planes (TF32 split), Kp a
+// multiple of 32.  err: one device int, zero on entry.
+constexpr float CORR_F16_SCALE = 16384.f;   // 2^14: |z| <= 1 stays far below the fp16 maximum
+int launch_gram_tc(const void* F, const void* L, int64_t n, int64_t n_pad, int64_t Kp,
+                   bool corr, float scale, float* S, int64_t lds, int* err, cudaStream_t s);
 int corr_plan(Arena& a, int64_t T, int64_t n, double** mu, double** inv, float** Z,
               int64_t* ldz);
 int launch_corr(const float* R, int64_t T, int64_t n, int64_t ldr, float* S,

@@ -5,21 +5,28 @@
 // stability through time with the Rand index"; the one dense contraction of
 // the pipeline (2 n^2 T flop).
 //
-// Z enters transposed and K-major as two planes of n_pad x Kp: ZF (the fp32
-// values, which the tensor core truncates to their TF32 part) and ZL (the
-// exact remainder z - trunc(z)), so
-//     Z^T Z = ZF.ZF + (ZF.ZL + ZL.ZF) + O(2^-22)
-// accumulated in two TMEM accumulators (main and correction).
+// Z enters transposed and K-major as two planes of n_pad x Kp, a hi part F and
+// a remainder L with Z = F + L to about 2^-22, so that
+//     Z^T Z = F.F + (F.L + L.F) + (L.L, dropped)
+// accumulated in two TMEM accumulators (main and correction):
+//   |corr|  fp16 planes of c z (c = 2^14, both parts rounded to nearest),
+//           kind::f16 MMAs (K = 16) at twice the TF32 rate, the sum scaled
+//           back by c^-2 (exact) in the epilogue
+//   TPDM    fp32 planes: F the values (the tensor core reads their TF32 part),
+//           L = w - trunc_tf32(w) exact; kind::tf32 MMAs (K = 8)
+// A stage holds 128 bytes of each row in either case (64 fp16 or 32 fp32
+// contraction columns), so the shared-memory layout and the descriptors'
+// 32-byte steps are the same for both.
 //
 // Persistent: one CTA per SM walks its share of the 128 x 128 output tiles
 // (I <= J, the upper triangle of tiles; each tile is also written
 // transposed), 256 threads:
-//   warp 0      TMA producer: per 32-column stage the rows I of ZF and ZL and,
-//               off the diagonal, the rows J of ZF and ZL (16 KB each), one
-//               stage ring across the CTA's tiles
-//   warp 1      MMA issuer (M = N = 128, K = 8, both operands in shared
-//               memory) into one of two TMEM accumulator sets, so that a
-//               tile's epilogue overlaps the next tile's loads and MMAs
+//   warp 0      TMA producer: per stage the rows I of F and L and, off the
+//               diagonal, the rows J of F and L (16 KB each), one stage ring
+//               across the CTA's tiles
+//   warp 1      MMA issuer (M = N = 128, both operands in shared memory) into
+//               one of two TMEM accumulator sets, so that a tile's epilogue
+//               overlaps the next tile's loads and MMAs
 //   warp 2      TMEM allocator
 //   warps 4-7   epilogue: thread r owns row I0 + r, reads the accumulators in
 //               32-column chunks, stages S[I-tile][chunk] (128-byte swizzle)
@@ -35,10 +42,10 @@
 namespace symnmf {
 
 constexpr int GT_BM = 128;                    // tile rows and columns
-constexpr int GT_BK = 32;                     // contraction columns per stage
+constexpr int GT_ROW_BYTES = 128;             // bytes of each operand row per stage
 constexpr int GT_NS_MAX = 3;                  // pipeline stages (|corr|; TPDM uses 2)
 constexpr int GT_THREADS = 256;
-constexpr uint32_t GT_PLANE = GT_BM * GT_BK * 4;   // 16 KB: 128 rows x 128 B
+constexpr uint32_t GT_PLANE = GT_BM * GT_ROW_BYTES; // 16 KB: 128 rows x 128 B
 constexpr uint32_t GT_STAGE = 4 * GT_PLANE;        // AF, AL, BF, BL
 constexpr uint32_t GT_OUT = GT_BM * 32 * 4;        // 16 KB: one 32-column output chunk
 // |corr| (long contraction): a 3-stage ring, one staging pair for the output;
@@ -49,8 +56,9 @@ constexpr uint32_t GT_ACC = 256;                   // one accumulator set: main 
 constexpr uint32_t GT_TMEM_COLS = 2 * GT_ACC;      // two sets: a tile drains while the next accumulates
 
 enum GramTcMode { GT_CORR = 0, GT_TPDM = 1 };
-template <> struct GtShape<GT_CORR> { static constexpr int NS = 3, NOUT = 1; };
-template <> struct GtShape<GT_TPDM> { static constexpr int NS = 2, NOUT = 2; };
+// BK: contraction columns per stage (128 bytes of fp16 or fp32)
+template <> struct GtShape<GT_CORR> { static constexpr int NS = 3, NOUT = 1, BK = 64; };
+template <> struct GtShape<GT_TPDM> { static constexpr int NS = 2, NOUT = 2, BK = 32; };
 template <int MODE>
 constexpr uint32_t gt_smem() {
     return GtShape<MODE>::NS * GT_STAGE + GtShape<MODE>::NOUT * 2 * GT_OUT + 1024;
@@ -116,6 +124,7 @@ gram_tc_kernel(const __grid_constant__ CUtensorMap mapF, const __grid_constant__
     // staging pair p: outD(p) [128 rows][32] with 128-byte swizzle, then outT(p) [32 rows][128]
     float* outBase = reinterpret_cast<float*>(smem + GT_NS * GT_STAGE);
 
+    constexpr int GT_BK = GtShape<MODE>::BK;
     const int ksteps = Kp / GT_BK;
     const int64_t nt = (n + GT_BM - 1) / GT_BM;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -181,7 +190,7 @@ gram_tc_kernel(const __grid_constant__ CUtensorMap mapF, const __grid_constant__
         }
     } else if (warp == 1 && lane == 0) {
         // ---------------- MMA issuer: tile u accumulates into set u % 2
-        constexpr uint32_t id = idesc_tf32(GT_BM, GT_BM);
+        constexpr uint32_t id = MODE == GT_CORR ? idesc_f16(GT_BM, GT_BM) : idesc_tf32(GT_BM, GT_BM);
         int64_t g = 0;
         int u = 0;
         for (int64_t x = blockIdx.x; x < vtiles && !abort_sh; x += gridDim.x) {
@@ -209,12 +218,18 @@ gram_tc_kernel(const __grid_constant__ CUtensorMap mapF, const __grid_constant__
                 const uint32_t bf = diag ? af : smem_u32(plane(slot, 2));
                 const uint32_t bl = diag ? al : smem_u32(plane(slot, 3));
 #pragma unroll
-                for (int kk = 0; kk < GT_BK / 8; ++kk) {
+                for (int kk = 0; kk < 4; ++kk) {   // four MMAs of 32 bytes of K each
                     const uint32_t o = (uint32_t)kk * 32u;
                     const uint32_t acc = (s | kk) ? 1u : 0u;
-                    umma_tf32_ss(dm, umma_desc_sw128(af + o), umma_desc_sw128(bf + o), id, acc);
-                    umma_tf32_ss(dc, umma_desc_sw128(af + o), umma_desc_sw128(bl + o), id, acc);
-                    umma_tf32_ss(dc, umma_desc_sw128(al + o), umma_desc_sw128(bf + o), id, 1u);
+                    if constexpr (MODE == GT_CORR) {
+                        umma_f16_ss(dm, umma_desc_sw128(af + o), umma_desc_sw128(bf + o), id, acc);
+                        umma_f16_ss(dc, umma_desc_sw128(af + o), umma_desc_sw128(bl + o), id, acc);
+                        umma_f16_ss(dc, umma_desc_sw128(al + o), umma_desc_sw128(bf + o), id, 1u);
+                    } else {
+                        umma_tf32_ss(dm, umma_desc_sw128(af + o), umma_desc_sw128(bf + o), id, acc);
+                        umma_tf32_ss(dc, umma_desc_sw128(af + o), umma_desc_sw128(bl + o), id, acc);
+                        umma_tf32_ss(dc, umma_desc_sw128(al + o), umma_desc_sw128(bf + o), id, 1u);
+                    }
                 }
                 umma_commit(&bar_empty[slot]);
             }
@@ -259,7 +274,7 @@ gram_tc_kernel(const __grid_constant__ CUtensorMap mapF, const __grid_constant__
                 for (int e = 0; e < 32; ++e) {
                     float z = __uint_as_float(vm[e]) + __uint_as_float(vc[e]);
                     if (MODE == GT_CORR) {
-                        z = fabsf(z);
+                        z = fabsf(z) * (1.f / (CORR_F16_SCALE * CORR_F16_SCALE));   // exact: 2^-28
                         if (i == J0 + q * 32 + e) z = 1.f;
                     } else {
                         z *= scale;
@@ -327,20 +342,23 @@ static PFN_cuTensorMapEncodeTiled_v12000 gt_encode_fn() {
     return fn;
 }
 
-static int gt_map(CUtensorMap* m, const float* base, int64_t Kp, int64_t rows) {
+// Load map over an operand plane: rows x Kp elements of `esize` bytes, a box of
+// 128 bytes x GT_BM rows.
+static int gt_map(CUtensorMap* m, const void* base, int64_t Kp, int64_t rows, bool f16) {
     auto fn = gt_encode_fn();
     if (fn == nullptr) {
         set_error("cuTensorMapEncodeTiled is not available from the driver");
         return SYMNMF_ERR_NOT_SUPPORTED;
     }
+    const int esize = f16 ? 2 : 4;
     cuuint64_t dims[2] = {(cuuint64_t)Kp, (cuuint64_t)rows};
-    cuuint64_t strides[1] = {(cuuint64_t)Kp * sizeof(float)};
-    cuuint32_t box[2] = {(cuuint32_t)GT_BK, (cuuint32_t)GT_BM};
+    cuuint64_t strides[1] = {(cuuint64_t)Kp * esize};
+    cuuint32_t box[2] = {(cuuint32_t)(GT_ROW_BYTES / esize), (cuuint32_t)GT_BM};
     cuuint32_t estr[2] = {1, 1};
-    const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(base), dims,
-                          strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    const CUresult r = fn(m, f16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2,
+                          const_cast<void*>(base), dims, strides, box, estr,
+                          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) {
         set_error("cuTensorMapEncodeTiled failed (%d)", (int)r);
         return SYMNMF_ERR_CUDA;
@@ -370,12 +388,17 @@ static int gt_store_map(CUtensorMap* m, float* S, int64_t n, int64_t lds, uint32
     return SYMNMF_OK;
 }
 
-// ZF, ZL: n_pad x Kp (n_pad multiple of 128, Kp multiple of 32, zero padding).
-int launch_gram_tc(const float* ZF, const float* ZL, int64_t n, int64_t n_pad, int64_t Kp,
+// F, L: n_pad x Kp (n_pad multiple of 128, zero padding); fp16 with Kp a
+// multiple of 64 for |corr|, fp32 with Kp a multiple of 32 for TPDM.
+int launch_gram_tc(const void* F, const void* L, int64_t n, int64_t n_pad, int64_t Kp,
                    bool corr, float scale, float* S, int64_t lds, int* err, cudaStream_t s) {
+    if (n_pad % GT_BM != 0 || Kp % (corr ? GtShape<GT_CORR>::BK : GtShape<GT_TPDM>::BK) != 0) {
+        set_error("tensor-core Gram: operand planes not padded to whole stages");
+        return SYMNMF_ERR_INVALID_ARG;
+    }
     CUtensorMap mapF, mapL, mapD, mapT;
-    SYMNMF_TRY(gt_map(&mapF, ZF, Kp, n_pad));
-    SYMNMF_TRY(gt_map(&mapL, ZL, Kp, n_pad));
+    SYMNMF_TRY(gt_map(&mapF, F, Kp, n_pad, corr));
+    SYMNMF_TRY(gt_map(&mapL, L, Kp, n_pad, corr));
     SYMNMF_TRY(gt_store_map(&mapD, S, n, lds, 32, GT_BM, CU_TENSOR_MAP_SWIZZLE_128B));
     SYMNMF_TRY(gt_store_map(&mapT, S, n, lds, GT_BM, 32, CU_TENSOR_MAP_SWIZZLE_NONE));
     const int64_t nt = n_pad / GT_BM;

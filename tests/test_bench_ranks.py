@@ -92,14 +92,14 @@ def test_row_rooflines_and_config_on_the_cpu():
     sbytes = 4.0 * n * n
     rows = {"stats_ms": 8.0, "kmeans_steps": 10, "kmeans_ms_per_step": 16.0,
             "svrg_epoch_ms": 16.0, "tpdm_build_ms": 10.0}
-    out, tf32 = bench.row_rooflines(rows, n, k, T, peak)
+    out, f16 = bench.row_rooflines(rows, n, k, T, peak)
     assert out["stats"]["GBs"] == pytest.approx(sbytes / 8e-3 / 1e9)
     assert out["stats"]["frac"] == pytest.approx(sbytes / 8e-3 / 1e9 / peak)
     assert out["kmeans_step"]["GBs"] == pytest.approx(2 * sbytes / 16e-3 / 1e9)
     assert out["svrg_epoch"]["GBs"] == pytest.approx(2 * sbytes / 16e-3 / 1e9)
     assert out["tpdm_build_writes"]["GBs"] == pytest.approx(sbytes / 10e-3 / 1e9)
     assert all(v["bound"] == "hbm" for v in out.values())
-    assert tf32 > 0
+    assert f16 > 0
     cfg = bench.bench_config("corr_n100000_k24", 1)
     assert (cfg["workload"], cfg["n"], cfg["k"], cfg["T"]) == ("corr_n100000_k24", n, k, T)
     assert cfg["parallelism"] == "single"
