@@ -207,6 +207,90 @@ def _timed(torch, fn):
     return a.elapsed_time(b), out
 
 
+def stream_clock_bins(m, torch, dev, S, H0, n, k, peak):
+    """The S-stream's launch time against the SM clock: 60 back-to-back
+    products Y = S H (the sustained regime, where the power cap lowers the SM
+    clock) after a second idle, then 12 launches spaced by 40 ms idle, with
+    nvidia-smi clock samples every 50 ms.  Each back-to-back launch takes the
+    clock sampled nearest its midpoint; launches are grouped by that clock."""
+    import datetime
+    gpu = int(os.environ.get("LOCAL_RANK", "0"))
+    ws = m.workspace(m._lib.OP_SH, n, k, device=dev)
+    X = H0.contiguous()
+    m.sh(S, X, ws=ws)
+    out_f = tempfile.TemporaryFile(mode="w+")
+    proc = subprocess.Popen(["nvidia-smi", "-i", str(gpu), "--query-gpu=timestamp,clocks.sm",
+                             "--format=csv,noheader,nounits", "-lms", "50"],
+                            stdout=out_f, stderr=subprocess.DEVNULL)
+    try:
+        torch.cuda.synchronize()
+        time.sleep(1.0)
+        es = [torch.cuda.Event(enable_timing=True) for _ in range(61)]
+        es[0].record()
+        t_start = time.time()
+        for i in range(60):
+            m.sh(S, X, ws=ws)
+            es[i + 1].record()
+        torch.cuda.synchronize()
+        b2b = [es[i].elapsed_time(es[i + 1]) for i in range(60)]
+        spaced = []
+        for _ in range(12):
+            time.sleep(0.04)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            m.sh(S, X, ws=ws)
+            b.record()
+            torch.cuda.synchronize()
+            spaced.append(a.elapsed_time(b))
+        time.sleep(0.1)
+    finally:
+        proc.terminate()
+        try:
+            proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            proc.kill()
+    out_f.seek(0)
+    samples = []
+    for line in out_f.read().strip().splitlines():
+        try:
+            ts, mhz = line.split(",")[:2]
+            t = datetime.datetime.strptime(ts.strip(), "%Y/%m/%d %H:%M:%S.%f").timestamp()
+            samples.append((t, float(mhz)))
+        except (ValueError, IndexError):
+            continue
+    gb = (4.0 * n * n + 4.0 * n * k) / 1e9
+    del ws
+    return {"spaced": _launch_row(spaced, [], gb, peak),
+            "back_to_back": bin_by_clock(b2b, t_start, samples, gb, peak)}
+
+
+def _launch_row(ms_list, mhz_list, gb, peak):
+    ms = statistics.median(ms_list)
+    return {"launches": len(ms_list), "ms": ms, "GBs": gb / ms * 1e3, "frac": gb / ms * 1e3 / peak,
+            "sm_mhz": statistics.median(mhz_list) if mhz_list else None}
+
+
+def bin_by_clock(ms_list, t_start, samples, gb, peak,
+                 edges=((1800.0, None), (1500.0, 1800.0), (0.0, 1500.0))):
+    """Back-to-back launch times (ms, in order from host time t_start) grouped
+    by the clock sample (time, MHz) nearest each launch's midpoint."""
+    if not samples:
+        return [_launch_row(ms_list, [], gb, peak)]
+    clk, t = [], t_start
+    for ms in ms_list:
+        mid = t + ms / 2e3
+        clk.append(min(samples, key=lambda sm: abs(sm[0] - mid))[1])
+        t += ms / 1e3
+    out = []
+    for lo, hi in edges:
+        sel = [i for i in range(len(ms_list)) if clk[i] >= lo and (hi is None or clk[i] < hi)]
+        if sel:
+            r = _launch_row([ms_list[i] for i in sel], [clk[i] for i in sel], gb, peak)
+            r["sm_mhz_range"] = [lo, hi]
+            out.append(r)
+    return out
+
+
 def converge_row(m, torch, S, k, planted_dev, solver, **kw):
     """One fit to the relative-loss-change stop (rel < 1e-5), timed with CUDA
     events: passes or epochs, seconds, loss, ARI of its labels against the
@@ -232,6 +316,12 @@ def measure_rows(m, torch, dev, S, H0, lab, n, k, T, rank, workload, planted=Non
     heavy-tailed window of the same size (builder, one Block-SVRG epoch), and
     the rolling-window study at its own size (n = 5,000, 250 windows)."""
     out = {}
+    # the S-stream against the SM clock (sustained back-to-back vs spaced launches)
+    if n >= 50000:
+        try:
+            out["stream_clock_bins"] = stream_clock_bins(m, torch, dev, S, H0, n, k, peaks()[0])
+        except Exception as exc:
+            out["stream_clock_bins"] = {"error": f"{type(exc).__name__}: {exc}"}
     # statistics pre-pass: one read of S
     ws = m.workspace(m._lib.OP_STATS, n, device=dev)
     ms, _ = _timed(torch, lambda: m.stats(S, ws=ws))

@@ -104,3 +104,21 @@ def test_row_rooflines_and_config_on_the_cpu():
     assert (cfg["workload"], cfg["n"], cfg["k"], cfg["T"]) == ("corr_n100000_k24", n, k, T)
     assert cfg["parallelism"] == "single"
     assert bench.bench_config("corr_n100000_k24", 8)["parallelism"].endswith("x8")
+
+
+def test_bin_by_clock_groups_launches_by_the_nearest_sample():
+    # launches of 10, 10, 12 and 14 ms from t = 100 s; samples at 100.000 s
+    # (1965 MHz), 100.025 s (1600 MHz) and 100.035 s (1400 MHz): the launch
+    # midpoints 100.005, 100.015, 100.026 and 100.039 take 1965, 1600, 1600
+    # and 1400
+    sys.path.insert(0, ROOT)
+    import bench
+    samples = [(100.0, 1965.0), (100.025, 1600.0), (100.035, 1400.0)]
+    rows = bench.bin_by_clock([10.0, 10.0, 12.0, 14.0], 100.0, samples, 40.0, 6500.0)
+    by = {tuple(r["sm_mhz_range"]): r for r in rows}
+    assert by[(1800.0, None)]["launches"] == 1
+    assert by[(1500.0, 1800.0)]["launches"] == 2 and by[(1500.0, 1800.0)]["ms"] == 11.0
+    assert by[(0.0, 1500.0)]["launches"] == 1 and by[(0.0, 1500.0)]["ms"] == 14.0
+    assert by[(0.0, 1500.0)]["GBs"] == pytest.approx(40.0 / 14.0 * 1e3)
+    # no samples: one row over every launch
+    assert bench.bin_by_clock([1.0, 3.0], 0.0, [], 1.0, 1.0)[0]["ms"] == 2.0
