@@ -465,6 +465,59 @@ int make_map(CUtensorMap* m, const float* base, int64_t cols, int64_t rows, int6
     return SYMNMF_OK;
 }
 
+// CTAs of stream_tc_kernel<KP> resident on one SM: two while both the tensor
+// memory (256 columns each) and the shared memory (228 KB an SM, 1 KB of it
+// reserved per CTA) allow, else one.
+template <int KP>
+static int tc_resident_per_sm() {
+    using Cfg = TcCfg<KP>;
+    if (Cfg::TMEM_COLS != 256u) return 1;
+    return 2 * (Cfg::SMEM + 1024) <= 228u * 1024u ? 2 : 1;
+}
+static int tc_resident(int KP) {
+    switch (KP) {
+        case 8: return tc_resident_per_sm<8>();
+        case 16: return tc_resident_per_sm<16>();
+        case 24: return tc_resident_per_sm<24>();
+        case 32: return tc_resident_per_sm<32>();
+        case 40: return tc_resident_per_sm<40>();
+        case 48: return tc_resident_per_sm<48>();
+        case 56: return tc_resident_per_sm<56>();
+        default: return tc_resident_per_sm<64>();
+    }
+}
+
+// Contraction splits of a pass over `tiles` row tiles and `steps` stages of
+// 32 columns: the count that minimises a model of the pass time fitted to
+// timings of Y = S X on B200 (k = 24; n = 10,000, 20,000 and 50,000 with
+// every split count from 1 to 15, where it picks the fastest count of each).
+// The CTAs run in waves of `resident`; a wave takes the longer of its HBM
+// time (16 KB of S a stage at 6.5 TB/s) and one CTA's stage cadence (0.55 us
+// a stage), plus 5 us of setup and tail; each split adds 1 us to the
+// epilogue's partial sums.  Every split keeps at least 8 stages.
+static int choose_splits(int64_t tiles, int64_t steps, int64_t resident) {
+    constexpr double kBW = 6.5e12, kStageBytes = 16384.0, kCadence = 0.55e-6, kWave = 5e-6,
+                     kSplit = 1e-6;
+    int best = 1;
+    double best_t = 1e30;
+    for (int s = 1; s <= 32; ++s) {
+        if (s > 1 && steps / s < 8) break;
+        const int64_t per = (steps + s - 1) / s;
+        int64_t left = tiles * s;
+        double t = kSplit * s;
+        while (left > 0) {
+            const int64_t w = std::min(left, resident);
+            left -= w;
+            t += std::max((double)w * (double)per * kStageBytes / kBW, (double)per * kCadence) + kWave;
+        }
+        if (t < best_t - 1e-12) {
+            best_t = t;
+            best = s;
+        }
+    }
+    return best;
+}
+
 TcPlan plan_stream_tc(const Dev& d, int64_t n, int k, int64_t j0, int64_t j1) {
     TcPlan p;
     p.n = n;
@@ -475,23 +528,8 @@ TcPlan plan_stream_tc(const Dev& d, int64_t n, int k, int64_t j0, int64_t j1) {
     p.j1 = std::min<int64_t>(n, (j1 + TC_BK - 1) / TC_BK * TC_BK);
     p.tiles = (n + TC_BM - 1) / TC_BM;
     const int64_t steps = std::max<int64_t>(1, (p.j1 - p.j0 + TC_BK - 1) / TC_BK);
-    const int64_t slots = (int64_t)d.sms * 2;                  // two CTAs per SM
-    // contraction splits: fill whole waves of resident CTAs, >= 8 stages each
-    int best = 1;
-    double best_waste = 1e30;
-    for (int s = 1; s <= 32; ++s) {
-        if (s > 1 && steps / s < 8) break;
-        const int64_t ctas = p.tiles * s;
-        const int64_t waves = (ctas + slots - 1) / slots;
-        const double waste = (double)(waves * slots) / (double)ctas - 1.0 + 0.002 * s;
-        if (waste < best_waste - 1e-12) {
-            best_waste = waste;
-            best = s;
-        }
-    }
-    p.splits = best;
-    const int64_t per = (steps + best - 1) / best;
-    p.jspan = per * TC_BK;
+    p.splits = choose_splits(p.tiles, steps, (int64_t)d.sms * tc_resident(p.KP));
+    p.jspan = (steps + p.splits - 1) / p.splits * TC_BK;
     return p;
 }
 
@@ -502,21 +540,8 @@ TcPlan plan_stream_tc_rows(const Dev& d, int64_t rows, int64_t ncols, int k) {
     p.ncols = ncols;
     p.tiles = (rows + TC_BM - 1) / TC_BM;
     const int64_t steps = std::max<int64_t>(1, (p.j1 - p.j0 + TC_BK - 1) / TC_BK);
-    const int64_t slots = (int64_t)d.sms * 2;
-    int best = 1;
-    double best_waste = 1e30;
-    for (int sp = 1; sp <= 32; ++sp) {
-        if (sp > 1 && steps / sp < 8) break;
-        const int64_t ctas = p.tiles * sp;
-        const int64_t waves = (ctas + slots - 1) / slots;
-        const double waste = (double)(waves * slots) / (double)ctas - 1.0 + 0.002 * sp;
-        if (waste < best_waste - 1e-12) {
-            best_waste = waste;
-            best = sp;
-        }
-    }
-    p.splits = best;
-    p.jspan = (steps + best - 1) / best * TC_BK;
+    p.splits = choose_splits(p.tiles, steps, (int64_t)d.sms * tc_resident(p.KP));
+    p.jspan = (steps + p.splits - 1) / p.splits * TC_BK;
     return p;
 }
 

@@ -88,13 +88,13 @@ def test_sh_matches_oracle(m, n, k):
 
 
 def test_sh_partials_staged_in_several_batches(m):
-    # k = 64 at n = 4,000: 9 contraction splits, while the epilogue's shared
-    # memory holds 5 partial tiles, so each tile's partials arrive in two
-    # batches (summed in split order either way)
+    # k = 64 at n = 2,000: 7 contraction splits (one CTA per SM at this k),
+    # while the epilogue's shared memory holds 5 partial tiles, so each
+    # tile's partials arrive in two batches (summed in split order either way)
     rng = np.random.default_rng(5)
-    A = rng.random((4000, 4000), dtype=np.float32)
+    A = rng.random((2000, 2000), dtype=np.float32)
     S = ((A + A.T) * np.float32(0.5)).astype(np.float32)
-    X = synth.uniform_h0(4000, 64, 0.5, seed=3)
+    X = synth.uniform_h0(2000, 64, 0.5, seed=3)
     Y = m.sh(to_dev(S, DEV), to_dev(X, DEV)).cpu().numpy()
     ref = S.astype(np.float64) @ X.astype(np.float64)
     assert rel_fro(Y, ref) <= 2e-6
