@@ -42,12 +42,15 @@ import synth  # noqa: E402
 METRIC = "SymNMF iterations/sec and S-stream HBM GB/s (% of peak) at n=1e5, k=24 fp32"
 UNIT = "iterations/s"
 SAMPLE_ROWS = 8192   # oracle sample: leading principal r x r block of the same window
-# DRAM traffic of one stream_tc_kernel<24> launch from ncu (dram__bytes_read.sum +
-# dram__bytes_write.sum): 1.619 GB + 13.8 MB at n = 20,000 against 1.602 GB of
-# algorithmic bytes; the full-size launch (40 GB S, too large to capture) is
-# reported as the same ratio times its algorithmic bytes.  Retake the capture
-# whenever the kernel changes.
-STREAM_TRAFFIC_RATIO = (1.618906e9 + 13.768704e6) / (4.0 * 20000 ** 2 + 4.0 * 20000 * 24)
+# DRAM traffic of one launch of each S-stream kernel from ncu (dram__bytes_read.sum
+# + dram__bytes_write.sum) at n = 20,000, k = 24, over its algorithmic bytes
+# (4n^2 + 4nk = 1.602 GB); the full-size launch (40 GB S, too large to capture)
+# is reported as the same ratio times its algorithmic bytes.  A kernel without
+# an entry (changed since its capture) reports null.  Retake a capture whenever
+# its kernel changes.
+STREAM_TRAFFIC_RATIO = {
+    "stream_tc_kernel": (1.618906e9 + 13.768704e6) / (4.0 * 20000 ** 2 + 4.0 * 20000 * 24),
+}
 STREAM_TRAFFIC_SOURCE = ("ncu dram__bytes_read.sum + dram__bytes_write.sum of one launch at "
                          "n = 20,000, k = 24, scaled to this launch by algorithmic bytes")
 
@@ -68,7 +71,13 @@ def parse():
                     help="with more than one GPU: independent windows, one per GPU")
     ap.add_argument("--upper", action="store_true",
                     help="time the upper-triangle S-stream (upper_only = 1) in the main loop")
-    return ap.parse_args()
+    ap.add_argument("--h16-min-n", type=int, default=None,
+                    help="size from which full-batch fits run the fp16 S-stream "
+                         "(sets SYMNMF_H16_MIN_N; the library's default is 32768, 0 = never)")
+    args = ap.parse_args()
+    if args.h16_min_n is not None:
+        os.environ["SYMNMF_H16_MIN_N"] = str(args.h16_min_n)
+    return args
 
 
 # ----------------------------------------------------------------------------- plumbing
@@ -725,8 +734,10 @@ def run_ours(args):
     if rank == 0:
         planted_dev = torch.from_numpy(np.asarray(planted, dtype=np.int32)).to(dev)
         ari_planted = m.ari(lab, planted_dev, max(k, int(planted.max()) + 1))[0]
-        traffic = (STREAM_TRAFFIC_RATIO * alg_bytes
-                   if args.workload == "corr_n100000_k24" and k == 24 and not up else None)
+        kname = m._lib.STREAM_KERNEL_NAMES.get(st.get("stream_kernel", 0), "stream_tc_kernel")
+        ratio = STREAM_TRAFFIC_RATIO.get(kname)
+        traffic = (ratio * alg_bytes
+                   if ratio is not None and args.workload == "corr_n100000_k24" and k == 24 else None)
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
             "warmup": W, "ms_per_step": t_max / K, "higher_is_better": True,
@@ -735,7 +746,7 @@ def run_ours(args):
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak, "traffic": traffic,
                          "traffic_source": STREAM_TRAFFIC_SOURCE if traffic is not None else None,
-                         "kernel": "stream_tri_kernel" if up else "stream_tc_kernel",
+                         "kernel": kname,
                          "peak_source": peak_src,
                          "alg_bytes_per_launch": alg_bytes, "launch_ms": stream_ms,
                          "frac_of_8000": achieved / 8000.0},

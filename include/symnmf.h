@@ -136,7 +136,23 @@ typedef struct {
     double stream_ms;        /* with timing = 1: their summed CUDA-event time, ms */
     double loop_ms;          /* with timing = 1: CUDA-event time of the iteration loop, ms */
     int kernel_launches;     /* kernels this call launched */
+    int stream_kernel;       /* S-stream of the full-batch passes: SYMNMF_STREAM_* */
 } symnmf_fit_stats;
+
+/* Which S-stream ran the full-batch passes of a fit (symnmf_fit_stats.stream_kernel):
+ * TF32: the tensor-core stream with S and X as exact TF32 splits (the default
+ *       below n = 32,768, for k > 24, and for Block-SVRG);
+ * FP16: the tensor-core stream with S and X as power-of-two scaled fp16 hi/lo
+ *       pairs (the AdaGrad solver from n = 32,768 up, k <= 24; the environment
+ *       variable SYMNMF_H16_MIN_N moves the threshold, 0 turns it off);
+ * UPPER: the upper-triangle stream (upper_only = 1);
+ * CUDA_CORE: the CUDA-core stream (SYMNMF_STREAM=cuda_core). */
+enum {
+    SYMNMF_STREAM_TF32 = 0,
+    SYMNMF_STREAM_FP16 = 1,
+    SYMNMF_STREAM_UPPER = 2,
+    SYMNMF_STREAM_CUDA_CORE = 3
+};
 
 /* Defaults listed in symnmf_fit_params. */
 SYMNMF_API void symnmf_fit_params_default(symnmf_fit_params* params);

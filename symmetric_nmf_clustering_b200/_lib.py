@@ -53,6 +53,12 @@ class FitParams(C.Structure):
     ]
 
 
+# symnmf_fit_stats.stream_kernel
+STREAM_TF32, STREAM_FP16, STREAM_UPPER, STREAM_CUDA_CORE = range(4)
+STREAM_KERNEL_NAMES = {STREAM_TF32: "stream_tc_kernel", STREAM_FP16: "stream_h16_kernel",
+                       STREAM_UPPER: "stream_tri_kernel", STREAM_CUDA_CORE: "stream_partial_kernel"}
+
+
 class FitStats(C.Structure):
     _fields_ = [
         ("iters", C.c_int),
@@ -70,6 +76,7 @@ class FitStats(C.Structure):
         ("stream_ms", C.c_double),
         ("loop_ms", C.c_double),
         ("kernel_launches", C.c_int),
+        ("stream_kernel", C.c_int),
     ]
 
     def as_dict(self):

@@ -134,6 +134,9 @@ struct FitLayout {
     int* counters = nullptr;
     float* tpart = nullptr;              // upper-triangle partial slabs (upper_only = 1)
     float* fpart = nullptr;
+    uint16_t* XT16 = nullptr;            // fp16 operand of the fp16 S-stream (k <= 24)
+    float* hmax_part = nullptr;          // per-tile max |H_{t+1}| (fp16 S-stream)
+    float* amax_part = nullptr;          // per-block max |S| of the statistics pass
 };
 
 static int64_t default_block_rows(int64_t n) {
@@ -205,6 +208,7 @@ static int plan_fit(const Dev& d, Arena& a, int64_t n, int k, const symnmf_fit_p
             }
         }
     }
+    if (h16_supported(k)) pf = std::max(pf, tc_partial_floats(plan_stream_h16(d, n, k)));
     if (P.upper_only) {
         const TriPlan tp = plan_stream_tri(d, n, k);
         pf = std::max(pf, (size_t)n * k);   // the reduced product goes to part
@@ -220,6 +224,11 @@ static int plan_fit(const Dev& d, Arena& a, int64_t n, int k, const symnmf_fit_p
     L->tr_part = a.take<double>((size_t)nb);
     L->gram_part = a.take<double>((size_t)nb * k * k);
     L->stats_part = a.take<double>((size_t)stats_blocks() * 3);
+    L->amax_part = a.take<float>((size_t)stats_blocks());
+    if (h16_supported(k)) {
+        L->XT16 = a.take<uint16_t>(h16_xt_halves(n, k));
+        L->hmax_part = a.take<float>((size_t)nb);
+    }
     L->hist_cap = std::max(1, P.max_iters + 1);
     L->hist = a.take<double>((size_t)L->hist_cap);
     if (svrg) {
@@ -235,6 +244,20 @@ static int plan_fit(const Dev& d, Arena& a, int64_t n, int k, const symnmf_fit_p
         L->probe_bytes = pb + 256;
     }
     return SYMNMF_OK;
+}
+
+// The full-batch loop of the AdaGrad solver streams S through the fp16
+// tensor-core kernel (stream_h16.cu) from n = 32,768 up (k <= 24, tensor-core
+// path, full matrix); below that the TF32 kernel, whose passes need no extra
+// launch for the operand split.  SYMNMF_H16_MIN_N overrides the size (0: never).
+static int64_t h16_min_n() {
+    const char* e = getenv("SYMNMF_H16_MIN_N");   // read per call: tests switch it
+    if (e != nullptr && *e != 0) return std::strtoll(e, nullptr, 10);
+    return 32768;
+}
+static bool h16_path(int64_t n, int k, const symnmf_fit_params& P) {
+    const int64_t m = h16_min_n();
+    return use_tc() && h16_supported(k) && P.upper_only == 0 && m > 0 && n >= m;
 }
 
 static int check_params(const symnmf_fit_params& P, int64_t n, int k) {
@@ -401,6 +424,7 @@ struct FitCtx {
     int epochs = 0;
     cudaStream_t s;
     Timing tm;
+    bool h16 = false;  // full-batch passes on the fp16 S-stream
     StreamArgs args() const {
         StreamArgs a;
         a.S = S;
@@ -445,6 +469,25 @@ struct FitCtx {
 // One S pass + epilogue + finalise in `mode`, reading Hb[cur], writing Hb[cur^1].
 // xt_ready: the split operand of Hb[cur] is already in XT (full-batch loop).
 static int full_pass(FitCtx& c, int mode, int max_evals, bool xt_ready) {
+    if (c.h16 && mode == MODE_FULL) {
+        // fp16 S-stream with the fused epilogue (which reports max |H_{t+1}| per
+        // tile instead of writing the TF32 split), the finalise step (which
+        // turns those maxima into the next operand's scale), then the fp16
+        // operand of H_{t+1}
+        const TcPlan p = plan_stream_h16(c.d, c.n, c.k);
+        EpiArgs e = c.epi(mode, 0.f, false);
+        e.part = c.L.part;
+        e.splits = p.splits;
+        e.hmax_part = c.L.hmax_part;
+        SYMNMF_TRY(c.tm.begin(c.s));
+        SYMNMF_TRY(launch_stream_h16(p, c.S, c.lds, c.L.XT16, c.L.part, &c.L.st->kerr, c.L.st, c.s,
+                                     &e, c.L.counters));
+        SYMNMF_TRY(c.tm.end(c.s));
+        SYMNMF_TRY(launch_finalize(mode, epilogue_blocks(c.n), c.k, c.L.tr_part, c.L.gram_part,
+                                   c.L.st, c.P->rel_tol, max_evals, c.L.hist, c.L.hist_cap, c.s,
+                                   c.L.hmax_part));
+        return launch_split16(c.Hb[c.cur ^ 1], c.n, c.k, c.L.st, c.L.XT16, c.s);
+    }
     SYMNMF_TRY(stream_pass(c.d, c.args(), c.Hb[c.cur], nullptr, c.k, 0, c.n, xt_ready,
                            c.epi(mode, 0.f, mode == MODE_FULL), c.s, &c.tm));
     return launch_finalize(mode, epilogue_blocks(c.n), c.k, c.L.tr_part, c.L.gram_part, c.L.st,
@@ -689,7 +732,8 @@ static int fit_impl(const float* S, int64_t n, int64_t lds, int k, const symnmf_
 
     // statistics pre-pass into the state head
     SYMNMF_CUDA_TRY(cudaMemsetAsync(c.L.st, 0, fit_state_bytes(), s));
-    SYMNMF_TRY(launch_stats(S, n, n, lds, c.L.stats_part, stats_blocks(), &c.L.st->s_sum, s));
+    SYMNMF_TRY(launch_stats(S, n, n, lds, c.L.stats_part, stats_blocks(), &c.L.st->s_sum, s,
+                            c.L.amax_part, c.L.st));
     HostState hs;
     SYMNMF_TRY(read_state(c.L.st, &hs, s));
     if (hs.s_bad > 0.0) {
@@ -722,11 +766,14 @@ static int fit_impl(const float* S, int64_t n, int64_t lds, int k, const symnmf_
     for (int b = 0; b < 2; ++b)
         SYMNMF_CUDA_TRY(cudaMemsetAsync(c.L.XT[b], 0, (size_t)xt_rows(k) * c.L.ldxt * sizeof(float), s));
     SYMNMF_CUDA_TRY(cudaMemsetAsync(c.L.counters, 0, (size_t)epilogue_blocks(n) * sizeof(int), s));
+    c.h16 = solver == SYMNMF_SOLVER_ADAGRAD && h16_path(n, k, P);
+    float* hmax = c.h16 ? c.L.hmax_part : nullptr;
     SYMNMF_TRY(launch_epilogue(MODE_GRAM, n, k, nullptr, 0, H, nullptr, nullptr, nullptr, nullptr,
                                0.f, 0.f, 0.f, c.L.tr_part, c.L.gram_part, nullptr, c.L.st, s,
-                               c.L.XT[0], c.L.ldxt));
+                               c.L.XT[0], c.L.ldxt, hmax));
     SYMNMF_TRY(launch_finalize(MODE_GRAM, epilogue_blocks(n), k, c.L.tr_part, c.L.gram_part,
-                               c.L.st, P.rel_tol, P.max_iters + 1, c.L.hist, c.L.hist_cap, s));
+                               c.L.st, P.rel_tol, P.max_iters + 1, c.L.hist, c.L.hist_cap, s, hmax));
+    if (c.h16) SYMNMF_TRY(launch_split16(H, n, k, c.L.st, c.L.XT16, s));   // the fp16 operand of H0
 
     cudaEvent_t e0 = nullptr, e1 = nullptr;
     if (c.tm.on) {
@@ -792,6 +839,9 @@ static int fit_impl(const float* S, int64_t n, int64_t lds, int k, const symnmf_
         out->stream_ms = c.tm.ms;
         out->loop_ms = loop_ms;
         out->kernel_launches = launches();
+        out->stream_kernel = c.h16 ? SYMNMF_STREAM_FP16
+                             : P.upper_only ? SYMNMF_STREAM_UPPER
+                             : use_tc() ? SYMNMF_STREAM_TF32 : SYMNMF_STREAM_CUDA_CORE;
     }
     return SYMNMF_OK;
 }

@@ -5,6 +5,7 @@
 #include <stdint.h>
 
 #include <algorithm>
+#include <cmath>
 #include <cstdio>
 #include <string>
 #include <utility>
@@ -88,6 +89,11 @@ struct FitState {
     int converged;
     int nonfinite;
     int kerr;                          // device-side error code (bounded wait gave up)
+    // fp16 S-stream of the full-batch loop (stream_h16.cu): max|S| over the
+    // finite entries, and the power-of-two scales of S and of the current
+    // iterate's operand (c |.| < 2^14 for every entry)
+    double s_absmax;
+    float sscale, xscale;
 };
 
 // Epilogue / finalise modes.
@@ -122,6 +128,12 @@ int launch_stream_partial(const StreamPlan& p, const float* S, int64_t lds,
                           const float* Xa, const float* Xb, int64_t ldx, float* part,
                           const FitState* st, cudaStream_t s);
 size_t fit_state_bytes();
+
+// Contraction splits of an S-stream pass (stream_tc.cu): the count that
+// minimises the pass-time model for `tiles` row tiles of `steps` stages of
+// `stage_bytes` of S, `resident` CTAs at a time, `cadence` seconds a stage.
+int choose_splits(int64_t tiles, int64_t steps, int64_t resident, double stage_bytes,
+                  double cadence);
 
 // Tensor-core S-stream (stream_tc.cu): X enters as its exact TF32 split
 // XT = [X_hi; X_lo] stored K-major (2*KP rows of length ldxt, KP = k rounded up to 8).
@@ -163,6 +175,20 @@ int launch_stream_tri(const TriPlan& p, const float* S, int64_t lds, const float
                       float* tpart, float* fpart, int* err, const FitState* st, cudaStream_t s);
 int launch_tri_reduce(const TriPlan& p, const float* tpart, const float* fpart, float* Y,
                       const FitState* st, cudaStream_t s);
+
+// fp16 S-stream of the full-batch loop (stream_h16.cu): S and X as scaled fp16
+// hi/lo pairs (scales st->sscale, st->xscale); its operand XT16 = [X_hi; X_lo]
+// is 2 KP rows of h16_ld(n) halves, written by launch_split16 from H and
+// st->xscale.  k <= 24, fused epilogue only.
+bool h16_supported(int k);
+int64_t h16_ld(int64_t n);
+size_t h16_xt_halves(int64_t n, int k);
+int launch_split16(const float* H, int64_t n, int k, const FitState* st, uint16_t* XT16,
+                   cudaStream_t s);
+TcPlan plan_stream_h16(const Dev& d, int64_t n, int k);
+int launch_stream_h16(const TcPlan& p, const float* S, int64_t lds, const uint16_t* XT16,
+                      float* part, int* err, const FitState* st, cudaStream_t s,
+                      const EpiArgs* epi, int* counters);
 int tri_set_stall(int on);
 
 int launch_split(const float* Xa, const float* Xb, int64_t ldx, int k, int64_t r0, int64_t r1,
@@ -177,14 +203,26 @@ int launch_epilogue(int mode, int64_t n, int k, const float* part, int splits,
                     float* Psnap, float m_scale, float lr, float eps,
                     double* tr_part, double* gram_part, float* Y,
                     const FitState* st, cudaStream_t s, float* XT = nullptr,
-                    int64_t ldxt = 0);
+                    int64_t ldxt = 0, float* hmax_part = nullptr);
+// hmax_part (FULL / GRAM passes of the fp16 stream): per-tile max |H_{t+1}|,
+// reduced into st->xscale
 int launch_finalize(int mode, int nblk, int k, const double* tr_part,
                     const double* gram_part, FitState* st, double rel_tol,
                     int max_evals, double* history, int history_cap,
-                    cudaStream_t s);
+                    cudaStream_t s, const float* hmax_part = nullptr);
 
+// amax_part (stats_blocks() floats) and st: optional; with both, max|S| over
+// the finite entries goes to st->s_absmax and its power-of-two scale to st->sscale
 int launch_stats(const float* S, int64_t rows, int64_t n, int64_t lds, double* part, int nblk,
-                 double* out3, cudaStream_t s);
+                 double* out3, cudaStream_t s, float* amax_part = nullptr, FitState* st = nullptr);
+// 2^(14 - e) for m < 2^e (m > 0 finite), at most 2^127; 1 otherwise: c m < 2^14
+__host__ __device__ inline float pow2_scale_below_2_14(double m) {
+    if (!(m > 0.0) || !(m <= 1.7976931348623157e308)) return 1.f;
+    int e = 0;
+    (void)frexp(m, &e);                 // m = f 2^e, f in [0.5, 1)
+    const int sh = 14 - e > 127 ? 127 : 14 - e;
+    return ldexpf(1.f, sh);
+}
 int stats_blocks();
 int launch_init_sum(float* H, int64_t n, int k, uint64_t seed, double s_sum, cudaStream_t s);
 int launch_init(float* H, int64_t n, int k, uint64_t seed, const FitState* st,

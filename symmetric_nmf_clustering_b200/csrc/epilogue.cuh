@@ -50,7 +50,22 @@ struct EpiArgs {
     const FitState* st;
     float* XT;             // split operand of the rows left in h (may be null)
     int64_t ldxt;
+    float* hmax_part;      // FULL / GRAM: max |h| over the tile's rows left in h (may be null)
 };
+
+// Max over the threads of a block of `nt` threads (a multiple of 32); the
+// result is valid in every thread.  wred: nt / 32 floats of shared memory.
+__device__ __forceinline__ float ep_block_max(float v, int tid, int nt, float* wred) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+    __syncthreads();
+    if ((tid & 31) == 0) wred[tid >> 5] = v;
+    __syncthreads();
+    float m = 0.f;
+    for (int w = 0; w < nt / 32; ++w) m = fmaxf(m, wred[w]);
+    __syncthreads();
+    return m;
+}
 
 // The evaluation's scalar step (one thread): f_t = ||S||^2 - 2 tr + ||A||^2,
 // history, relative change, stopping test ([CaS] "Factorizing with SymNMF";
@@ -212,6 +227,16 @@ __device__ void epilogue_tile(const EpiArgs& a, int tile, int tid, float* smem, 
                 a.XT[(int64_t)(KP + c) * a.ldxt + i] = h[c] - hb;
             }
         }
+    }
+
+    if (a.hmax_part != nullptr && (mode == MODE_FULL || mode == MODE_GRAM)) {
+        __shared__ float wred[EP_ROWS / 32];
+        float m = 0.f;
+#pragma unroll
+        for (int c = 0; c < KE; ++c)
+            if (valid && c < k) m = fmaxf(m, fabsf(h[c]));
+        m = ep_block_max(m, tid, EP_ROWS, wred);
+        if (tid == 0) a.hmax_part[tile] = m;
     }
 
     // Gram partial of the rows now in h (new iterate, or the given H for GRAM)
@@ -531,6 +556,14 @@ __device__ void epilogue_tile_cta(const EpiArgs& a, int tile, int tid, float* sm
     for (int q = 0; q < EPT; ++q) {
         const int e = tid + q * NT, r = e / KE, c = e % KE;
         hreg[q] = (r < rows && c < k) ? T1[r * k + c] : 0.f;
+    }
+    if (a.hmax_part != nullptr && (mode == MODE_FULL || mode == MODE_GRAM)) {
+        __shared__ float wred[NT / 32];
+        float m = 0.f;
+#pragma unroll
+        for (int q = 0; q < EPT; ++q) m = fmaxf(m, fabsf(hreg[q]));
+        m = ep_block_max(m, tid, NT, wred);
+        if (tid == 0) a.hmax_part[tile] = m;
     }
     __syncthreads();
 #pragma unroll

@@ -32,8 +32,9 @@ int stats_blocks() { return STATS_BLOCKS; }
 
 __global__ void __launch_bounds__(STATS_THREADS)
 stats_partial_kernel(const float* __restrict__ S, int64_t rows, int64_t n, int64_t lds,
-                     double* __restrict__ part) {
+                     double* __restrict__ part, float* __restrict__ amax_part) {
     double sum = 0.0, sq = 0.0, bad = 0.0;
+    float amax = 0.f;   // max |S| over the finite entries
     const int64_t n4 = n >> 2;
     for (int64_t r = blockIdx.x; r < rows; r += gridDim.x) {
         const float4* row = reinterpret_cast<const float4*>(S + r * lds);
@@ -66,6 +67,8 @@ stats_partial_kernel(const float* __restrict__ S, int64_t rows, int64_t n, int64
                     // (no carry reaches bit 31); the conversion instruction's
                     // throughput, not HBM, limited this pass
 #pragma unroll
+                    for (int w = 0; w < 4; ++w) amax = fmaxf(amax, fabsf(e[w]));
+#pragma unroll
                     for (int w = 0; w < 4; ++w) {
                         const uint32_t b = __float_as_uint(e[w]);
                         const uint32_t hi = ((uint32_t)((int32_t)b >> 3) & 0x8FFFFFFFu) + 0x38000000u;
@@ -80,6 +83,7 @@ stats_partial_kernel(const float* __restrict__ S, int64_t rows, int64_t n, int64
                             const double d = e[w];
                             sum += d;
                             sq = fma(d, d, sq);
+                            amax = fmaxf(amax, fabsf(e[w]));
                         } else {
                             bad += 1.0;
                         }
@@ -92,6 +96,7 @@ stats_partial_kernel(const float* __restrict__ S, int64_t rows, int64_t n, int64
             if (isfinite(e)) {
                 sum += (double)e;
                 sq = fma((double)e, (double)e, sq);
+                amax = fmaxf(amax, fabsf(e));
             } else {
                 bad += 1.0;
             }
@@ -108,10 +113,24 @@ stats_partial_kernel(const float* __restrict__ S, int64_t rows, int64_t n, int64
         __syncthreads();
     }
     if (threadIdx.x < 3) part[blockIdx.x * 3 + threadIdx.x] = red[threadIdx.x][0];
+    if (amax_part != nullptr) {
+        // max is exact in any order
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+        __shared__ float wmax[STATS_THREADS / 32];
+        if ((threadIdx.x & 31) == 0) wmax[threadIdx.x >> 5] = amax;
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            float m = 0.f;
+            for (int w = 0; w < STATS_THREADS / 32; ++w) m = fmaxf(m, wmax[w]);
+            amax_part[blockIdx.x] = m;
+        }
+    }
 }
 
 __global__ void stats_final_kernel(const double* __restrict__ part, int nblk,
-                                   double* __restrict__ out3) {
+                                   double* __restrict__ out3, const float* __restrict__ amax_part,
+                                   FitState* st) {
     __shared__ double red[3][STATS_THREADS];
     double a[3] = {0.0, 0.0, 0.0};
     for (int b = threadIdx.x; b < nblk; b += blockDim.x)
@@ -124,13 +143,19 @@ __global__ void stats_final_kernel(const double* __restrict__ part, int nblk,
         __syncthreads();
     }
     if (threadIdx.x < 3) out3[threadIdx.x] = red[threadIdx.x][0];
+    if (amax_part != nullptr && st != nullptr && threadIdx.x == 0) {
+        float m = 0.f;
+        for (int b = 0; b < nblk; ++b) m = fmaxf(m, amax_part[b]);
+        st->s_absmax = m;
+        st->sscale = pow2_scale_below_2_14((double)m);
+    }
 }
 
 int launch_stats(const float* S, int64_t rows, int64_t n, int64_t lds, double* part, int nblk,
-                 double* out3, cudaStream_t s) {
-    stats_partial_kernel<<<nblk, STATS_THREADS, 0, s>>>(S, rows, n, lds, part);
+                 double* out3, cudaStream_t s, float* amax_part, FitState* st) {
+    stats_partial_kernel<<<nblk, STATS_THREADS, 0, s>>>(S, rows, n, lds, part, amax_part);
     SYMNMF_LAUNCH_CHECK();
-    stats_final_kernel<<<1, STATS_THREADS, 0, s>>>(part, nblk, out3);
+    stats_final_kernel<<<1, STATS_THREADS, 0, s>>>(part, nblk, out3, amax_part, st);
     SYMNMF_LAUNCH_CHECK();
     return SYMNMF_OK;
 }

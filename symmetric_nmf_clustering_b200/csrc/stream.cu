@@ -16,6 +16,8 @@
 // contraction over j reads rows of S, each a contiguous, coalesced run of
 // the output index i.  Every reduction has a fixed order, so results are
 // bitwise reproducible run to run on a given device.
+#include <cstring>
+
 #include "common.cuh"
 #include "epilogue.cuh"
 
@@ -184,9 +186,11 @@ int launch_epilogue(int mode, int64_t n, int k, const float* part, int splits,
                     const float* H, const float* G, float* Hn, float* Gn,
                     float* Psnap, float m_scale, float lr, float eps,
                     double* tr_part, double* gram_part, float* Y,
-                    const FitState* st, cudaStream_t s, float* XT, int64_t ldxt) {
+                    const FitState* st, cudaStream_t s, float* XT, int64_t ldxt,
+                    float* hmax_part) {
     const int nb = epilogue_blocks(n);
     EpiArgs a;
+    std::memset(&a, 0, sizeof(a));
     a.mode = mode;
     a.n = n;
     a.k = k;
@@ -206,6 +210,7 @@ int launch_epilogue(int mode, int64_t n, int k, const float* part, int splits,
     a.st = st;
     a.XT = XT;
     a.ldxt = ldxt;
+    a.hmax_part = hmax_part;
 #define SYMNMF_EP(KE) epilogue_kernel<KE><<<nb, EP_ROWS, 0, s>>>(a)
     if (k <= 8) SYMNMF_EP(8);
     else if (k <= 16) SYMNMF_EP(16);
@@ -233,7 +238,7 @@ __global__ void __launch_bounds__(RF_THREADS)
 reduce_finalize_kernel(int mode, int nblk, int k, const double* __restrict__ tr_part,
                        const double* __restrict__ gram_part, FitState* st,
                        FinalScratch* fs, double rel_tol, int max_evals,
-                       double* history, int history_cap) {
+                       double* history, int history_cap, const float* __restrict__ hmax_part) {
     pdl_wait();
     pdl_trigger();   // the next pass's CTAs may start their setup meanwhile
     if (st->done) return;
@@ -313,13 +318,28 @@ reduce_finalize_kernel(int mode, int nblk, int k, const double* __restrict__ tr_
             __syncthreads();
         }
         if (threadIdx.x == 0) st->a_sqnorm = qs[0];
+        // the next iterate's operand scale: max |H_{t+1}| over the tiles (exact in any order)
+        if (hmax_part != nullptr) {
+            __shared__ float mw[RF_THREADS / 32];
+            float m = 0.f;
+            for (int b = threadIdx.x; b < nblk; b += RF_THREADS) m = fmaxf(m, __ldcg(&hmax_part[b]));
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+            if ((threadIdx.x & 31) == 0) mw[threadIdx.x >> 5] = m;
+            __syncthreads();
+            if (threadIdx.x == 0) {
+                float mm = 0.f;
+                for (int w = 0; w < RF_THREADS / 32; ++w) mm = fmaxf(mm, mw[w]);
+                st->xscale = pow2_scale_below_2_14((double)mm);
+            }
+        }
     }
 }
 
 int launch_finalize(int mode, int nblk, int k, const double* tr_part,
                     const double* gram_part, FitState* st, double rel_tol,
                     int max_evals, double* history, int history_cap,
-                    cudaStream_t s) {
+                    cudaStream_t s, const float* hmax_part) {
     // FinalScratch lives right after the FitState (see fit planning).
     FinalScratch* fs = reinterpret_cast<FinalScratch*>(
         reinterpret_cast<char*>(st) + ((sizeof(FitState) + 255) & ~size_t(255)));
@@ -328,7 +348,7 @@ int launch_finalize(int mode, int nblk, int k, const double* tr_part,
     const int grid = gram_blocks + 1;
     SYMNMF_CUDA_TRY(launch_pdl(reduce_finalize_kernel, dim3(grid), dim3(RF_THREADS), 0, s, mode, nblk, k,
                                tr_part, gram_part, st, fs, rel_tol, max_evals, history,
-                               history_cap));
+                               history_cap, hmax_part));
     SYMNMF_LAUNCH_CHECK();
     return SYMNMF_OK;
 }

@@ -494,10 +494,11 @@ static int tc_resident(int KP) {
 // The CTAs run in waves of `resident`; a wave takes the longer of its HBM
 // time (16 KB of S a stage at 6.5 TB/s) and one CTA's stage cadence (0.55 us
 // a stage), plus 5 us of setup and tail; each split adds 1 us to the
-// epilogue's partial sums.  Every split keeps at least 8 stages.
-static int choose_splits(int64_t tiles, int64_t steps, int64_t resident) {
-    constexpr double kBW = 6.5e12, kStageBytes = 16384.0, kCadence = 0.55e-6, kWave = 5e-6,
-                     kSplit = 1e-6;
+// epilogue's partial sums.  Every split keeps at least 8 stages.  (The fp16
+// stream passes its own stage size and cadence.)
+int choose_splits(int64_t tiles, int64_t steps, int64_t resident, double kStageBytes,
+                  double kCadence) {
+    constexpr double kBW = 6.5e12, kWave = 5e-6, kSplit = 1e-6;
     int best = 1;
     double best_t = 1e30;
     for (int s = 1; s <= 32; ++s) {
@@ -528,7 +529,7 @@ TcPlan plan_stream_tc(const Dev& d, int64_t n, int k, int64_t j0, int64_t j1) {
     p.j1 = std::min<int64_t>(n, (j1 + TC_BK - 1) / TC_BK * TC_BK);
     p.tiles = (n + TC_BM - 1) / TC_BM;
     const int64_t steps = std::max<int64_t>(1, (p.j1 - p.j0 + TC_BK - 1) / TC_BK);
-    p.splits = choose_splits(p.tiles, steps, (int64_t)d.sms * tc_resident(p.KP));
+    p.splits = choose_splits(p.tiles, steps, (int64_t)d.sms * tc_resident(p.KP), 16384.0, 0.55e-6);
     p.jspan = (steps + p.splits - 1) / p.splits * TC_BK;
     return p;
 }
@@ -540,7 +541,7 @@ TcPlan plan_stream_tc_rows(const Dev& d, int64_t rows, int64_t ncols, int k) {
     p.ncols = ncols;
     p.tiles = (rows + TC_BM - 1) / TC_BM;
     const int64_t steps = std::max<int64_t>(1, (p.j1 - p.j0 + TC_BK - 1) / TC_BK);
-    p.splits = choose_splits(p.tiles, steps, (int64_t)d.sms * tc_resident(p.KP));
+    p.splits = choose_splits(p.tiles, steps, (int64_t)d.sms * tc_resident(p.KP), 16384.0, 0.55e-6);
     p.jspan = (steps + p.splits - 1) / p.splits * TC_BK;
     return p;
 }
