@@ -491,7 +491,8 @@ SYMNMF_API int symnmf_sh_noalloc(const float* S, int64_t n, int64_t lds, const f
 
 /*
  * Test hook for failure detection (no counterpart on the pages).  on != 0:
- * the S-stream kernel's TMA producer issues no loads on the current device,
+ * the TMA producer of S in every S-stream kernel (TF32, fp16 and upper-
+ * triangle) issues no loads on the current device,
  * so every bounded pipeline wait of the next S-stream launches runs out
  * (about 2 s) and those calls return SYMNMF_ERR_TIMEOUT with the CUDA context
  * intact; on = 0 restores normal operation.  Synchronous.

@@ -181,6 +181,7 @@ int launch_tri_reduce(const TriPlan& p, const float* tpart, const float* fpart, 
 // is 2 KP rows of h16_ld(n) halves, written by launch_split16 from H and
 // st->xscale.  k <= 24, fused epilogue only.
 bool h16_supported(int k);
+int h16_set_stall(int on);   // test hook: the producer of S issues no loads
 int64_t h16_ld(int64_t n);
 size_t h16_xt_halves(int64_t n, int k);
 int launch_split16(const float* H, int64_t n, int k, const FitState* st, uint16_t* XT16,

@@ -143,11 +143,21 @@ __global__ void stats_final_kernel(const double* __restrict__ part, int nblk,
         __syncthreads();
     }
     if (threadIdx.x < 3) out3[threadIdx.x] = red[threadIdx.x][0];
-    if (amax_part != nullptr && st != nullptr && threadIdx.x == 0) {
+    if (amax_part != nullptr && st != nullptr) {
+        // max over the blocks (exact in any order): strided, then across the block
         float m = 0.f;
-        for (int b = 0; b < nblk; ++b) m = fmaxf(m, amax_part[b]);
-        st->s_absmax = m;
-        st->sscale = pow2_scale_below_2_14((double)m);
+        for (int b = threadIdx.x; b < nblk; b += blockDim.x) m = fmaxf(m, amax_part[b]);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        __shared__ float wmax[STATS_THREADS / 32];
+        if ((threadIdx.x & 31) == 0) wmax[threadIdx.x >> 5] = m;
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            float mm = 0.f;
+            for (int w = 0; w < STATS_THREADS / 32; ++w) mm = fmaxf(mm, wmax[w]);
+            st->s_absmax = mm;
+            st->sscale = pow2_scale_below_2_14((double)mm);
+        }
     }
 }
 

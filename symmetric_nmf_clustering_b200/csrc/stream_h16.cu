@@ -52,6 +52,11 @@ namespace symnmf {
 int make_map(CUtensorMap* m, const float* base, int64_t cols, int64_t rows, int64_t ld,
              uint32_t box_rows);
 
+// Test hook (symnmf_test_stall_pipeline): when set, the producer of S issues
+// no loads, so the consumers' bounded waits run out and the pass reports its
+// error word instead of a result.
+__device__ int g_h16_stall = 0;
+
 constexpr int H16_BM = 128;                    // S rows per tile = tensor-memory lanes
 constexpr int H16_BK = 64;                     // columns per stage (two 32-column S boxes)
 constexpr int H16_NSS = 3;                     // shared-memory slots of S
@@ -160,7 +165,7 @@ stream_h16_kernel(const __grid_constant__ CUtensorMap mapS, const __grid_constan
     tc_fence_after();
     const uint32_t tbase = tmem_base_sh;
 
-    if (warp == 0 && lane == 0 && ksteps > 0) {
+    if (warp == 0 && lane == 0 && ksteps > 0 && *(volatile int*)&g_h16_stall == 0) {
         // ---------------- TMA producer of S: slot s % 3, free once the split
         // warps have read stage s - 3
         int issued = 0;
@@ -389,6 +394,12 @@ __global__ void split16_kernel(const float* __restrict__ H, int64_t n, int k, in
 }
 
 bool h16_supported(int k) { return k >= 1 && k <= 24; }
+
+int h16_set_stall(int on) {
+    const int v = on ? 1 : 0;
+    SYMNMF_CUDA_TRY(cudaMemcpyToSymbol(g_h16_stall, &v, sizeof(int)));
+    return SYMNMF_OK;
+}
 
 int64_t h16_ld(int64_t n) { return (n + H16_BK - 1) / H16_BK * H16_BK; }
 

@@ -595,5 +595,6 @@ extern "C" int symnmf_test_stall_pipeline(int on) {
         symnmf::set_error("cudaMemcpyToSymbol failed: %s", cudaGetErrorString(e));
         return SYMNMF_ERR_CUDA;
     }
+    SYMNMF_TRY(symnmf::h16_set_stall(v));
     return symnmf::tri_set_stall(v);
 }

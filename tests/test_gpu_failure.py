@@ -82,3 +82,27 @@ def test_sh_upper_reports_the_timeout_and_the_context_recovers(m):
     ref = S_host.astype(np.float64) @ X.cpu().numpy().astype(np.float64)
     got = Y.cpu().numpy().astype(np.float64)
     assert np.linalg.norm(got - ref) <= 1e-4 * np.linalg.norm(ref)
+
+
+def test_fit_on_the_fp16_stream_reports_the_timeout_and_the_context_recovers(m):
+    # the fp16 S-stream (here forced at a small size) bounds its waits the same way
+    import os
+    import torch
+    from symmetric_nmf_clustering_b200 import _lib as L
+    lib = L.load()
+    _, S, _ = _problem(600, 6, 3)
+    old = os.environ.get("SYMNMF_H16_MIN_N")
+    os.environ["SYMNMF_H16_MIN_N"] = "1"
+    try:
+        _stalled(lib, lambda: m.fit(S, 6, seed=3, max_iters=20, rel_tol=0.0))
+        H1, st1 = m.fit(S, 6, seed=3, max_iters=20, rel_tol=0.0)
+        H2, st2 = m.fit(S, 6, seed=3, max_iters=20, rel_tol=0.0)
+        torch.cuda.synchronize()
+    finally:
+        if old is None:
+            os.environ.pop("SYMNMF_H16_MIN_N", None)
+        else:
+            os.environ["SYMNMF_H16_MIN_N"] = old
+    assert st1["stream_kernel"] == L.STREAM_FP16
+    assert st1["iters"] == 20 and np.isfinite(st1["loss"])
+    assert torch.equal(H1, H2) and st1["loss"] == st2["loss"]
