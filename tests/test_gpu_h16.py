@@ -1,7 +1,7 @@
 """Parity of the fp16 S-stream of the full-batch loop (stream_h16.cu).
 
 The library runs the AdaGrad solver's full-batch passes through this kernel
-from n = 32,768 up (k <= 24); SYMNMF_H16_MIN_N lowers the threshold so that
+from n = 50,000 up (k <= 24); SYMNMF_H16_MIN_N lowers the threshold so that
 it runs at sizes the oracle follows (the variable is read on every call).
 S and X enter as power-of-two scaled fp16 hi/lo pairs, so the tolerances are
 those of the TF32 path: per-step H and G 1e-4, trajectories H 1e-3 and loss
@@ -114,18 +114,22 @@ def test_h16_bitwise_reproducible_over_several_waves(m, h16_on):
 
 
 def test_h16_path_selection(m):
-    # below the threshold (and for k > 24 at any size) the TF32 path runs:
-    # two launches per pass instead of three
+    # below the threshold, for k > 24 at any size and for Block-SVRG the TF32
+    # path runs (two launches per pass instead of three)
+    from symmetric_nmf_clustering_b200 import _lib as L
     _, _, S = corr_problem(2000, 120, seed=5)
     old = os.environ.pop("SYMNMF_H16_MIN_N", None)
     try:
         _, st = _fit(m, S, 8, seed=1, max_iters=20, rel_tol=0.0)
-        assert st["kernel_launches"] < 3 * 20
+        assert st["stream_kernel"] == L.STREAM_TF32 and st["kernel_launches"] < 3 * 20
         os.environ["SYMNMF_H16_MIN_N"] = "1"
         _, st = _fit(m, S, 8, seed=1, max_iters=20, rel_tol=0.0)
-        assert st["kernel_launches"] >= 3 * 20
+        assert st["stream_kernel"] == L.STREAM_FP16 and st["kernel_launches"] >= 3 * 20
         _, st = _fit(m, S, 32, seed=1, max_iters=20, rel_tol=0.0)
-        assert st["kernel_launches"] < 3 * 20
+        assert st["stream_kernel"] == L.STREAM_TF32 and st["kernel_launches"] < 3 * 20
+        _, st = _fit(m, S, 8, seed=1, solver="block_svrg", block_rows=512, max_iters=3,
+                     rel_tol=0.0)
+        assert st["stream_kernel"] == L.STREAM_TF32
     finally:
         if old is None:
             os.environ.pop("SYMNMF_H16_MIN_N", None)
