@@ -499,6 +499,18 @@ SYMNMF_API int symnmf_sh_noalloc(const float* S, int64_t n, int64_t lds, const f
  */
 SYMNMF_API int symnmf_test_stall_pipeline(int on);
 
+/*
+ * Test hook for the fp16 S-stream's operand split (no counterpart on the
+ * pages): applies the split warps' arithmetic to the n values at x (device,
+ * n a multiple of 4, x 16-byte aligned): v = scale * x (scale a power of two),
+ * hi = v rounded to 11 significant bits by Veltkamp's splitting, lo = v - hi,
+ * both rounded to fp16; hi[i] and lo[i] (device, n / 2 words each) hold the
+ * fp16 bit patterns of values 2i (low half) and 2i + 1 (high half).
+ * Asynchronous on `stream`.
+ */
+SYMNMF_API int symnmf_test_split16(const float* x, int64_t n, float scale, uint32_t* hi,
+                                   uint32_t* lo, symnmf_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -161,6 +161,7 @@ SIGNATURES = {
                           _sz, _vp]),
     "symnmf_rolling_params_default": (None, [C.POINTER(RollingParams)]),
     "symnmf_test_stall_pipeline": (_int, [_int]),
+    "symnmf_test_split16": (_int, [_vp, _i64, C.c_float, _vp, _vp, _vp]),
     "symnmf_rolling": (_int, [_vp, _i64, _i64, _i64, _vp, _vp, _i64, C.POINTER(RollingParams),
                               C.POINTER(RollingOut), _vp, _sz, _vp]),
 }

@@ -106,6 +106,20 @@ __device__ __forceinline__ void split_11(float v, float& hi, float& lo) {
     lo = __fsub_rn(v, hi);
 }
 
+// Four values q scaled by cs (a power of two: exact), each split as above;
+// h0/l0 hold the fp16 hi/lo of q.x, q.y (low, high half), h1/l1 of q.z, q.w.
+__device__ __forceinline__ void split_scaled4(const float4 q, float cs, uint32_t& h0, uint32_t& h1,
+                                              uint32_t& l0, uint32_t& l1) {
+    const float e[4] = {q.x * cs, q.y * cs, q.z * cs, q.w * cs};
+    float h[4], l[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) split_11(e[u], h[u], l[u]);
+    h0 = pack_h2(h[0], h[1]);
+    h1 = pack_h2(h[2], h[3]);
+    l0 = pack_h2(l[0], l[1]);
+    l1 = pack_h2(l[2], l[3]);
+}
+
 template <int KP>
 __global__ void __launch_bounds__(H16_THREADS, 2)
 stream_h16_kernel(const __grid_constant__ CUtensorMap mapS, const __grid_constant__ CUtensorMap mapX,
@@ -296,15 +310,8 @@ stream_h16_kernel(const __grid_constant__ CUtensorMap mapS, const __grid_constan
 #pragma unroll
                 for (int c = 0; c < 8; ++c) {
                     const float4 q = *reinterpret_cast<const float4*>(rowp + ((c ^ (r & 7)) << 4));
-                    const float e[4] = {q.x * cs, q.y * cs, q.z * cs, q.w * cs};   // exact: cs is 2^m
-                    float h[4], l[4];
-#pragma unroll
-                    for (int u = 0; u < 4; ++u) split_11(e[u], h[u], l[u]);
                     const int w = b * 16 + c * 2;   // column pair of elements 4c..4c+3 of box b
-                    hi[w] = pack_h2(h[0], h[1]);
-                    hi[w + 1] = pack_h2(h[2], h[3]);
-                    lo[w] = pack_h2(l[0], l[1]);
-                    lo[w + 1] = pack_h2(l[2], l[3]);
+                    split_scaled4(q, cs, hi[w], hi[w + 1], lo[w], lo[w + 1]);
                 }
             }
             // the stage of S is read: release the slot.  The next fill is an
@@ -452,6 +459,25 @@ static int h16_map_x(CUtensorMap* m, const uint16_t* XT, int64_t n, int KP, int6
     return SYMNMF_OK;
 }
 
+// The split warps' arithmetic on a plain array (test hook): x[4i .. 4i+3] ->
+// hi[2i], hi[2i+1], lo[2i], lo[2i+1], as split_scaled4 produces them.
+__global__ void split_probe_kernel(const float4* __restrict__ x, int64_t quads, float cs,
+                                   uint32_t* __restrict__ hi, uint32_t* __restrict__ lo) {
+    const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (i >= quads) return;
+    split_scaled4(x[i], cs, hi[2 * i], hi[2 * i + 1], lo[2 * i], lo[2 * i + 1]);
+}
+
+int launch_split_probe(const float* x, int64_t n, float cs, uint32_t* hi, uint32_t* lo,
+                       cudaStream_t s) {
+    const int64_t quads = n / 4;
+    if (quads <= 0) return SYMNMF_OK;
+    split_probe_kernel<<<(unsigned)((quads + 255) / 256), 256, 0, s>>>(
+        reinterpret_cast<const float4*>(x), quads, cs, hi, lo);
+    SYMNMF_LAUNCH_CHECK();
+    return SYMNMF_OK;
+}
+
 TcPlan plan_stream_h16(const Dev& d, int64_t n, int k) {
     TcPlan p;
     p.n = n;
@@ -501,3 +527,15 @@ int launch_stream_h16(const TcPlan& p, const float* S, int64_t lds, const uint16
 }
 
 }  // namespace symnmf
+
+extern "C" int symnmf_test_split16(const float* x, int64_t n, float scale, uint32_t* hi, uint32_t* lo,
+                                   symnmf_stream_t stream) {
+    symnmf::clear_error();
+    if (n < 0 || n % 4 != 0 || (n > 0 && (x == nullptr || hi == nullptr || lo == nullptr)) ||
+        (reinterpret_cast<uintptr_t>(x) & 15u) != 0 || (reinterpret_cast<uintptr_t>(hi) & 3u) != 0 ||
+        (reinterpret_cast<uintptr_t>(lo) & 3u) != 0) {
+        symnmf::set_error("symnmf_test_split16: n must be a multiple of 4 and x 16-byte aligned");
+        return SYMNMF_ERR_INVALID_ARG;
+    }
+    return symnmf::launch_split_probe(x, n, scale, hi, lo, (cudaStream_t)stream);
+}

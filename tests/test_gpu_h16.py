@@ -135,3 +135,39 @@ def test_h16_path_selection(m):
             os.environ.pop("SYMNMF_H16_MIN_N", None)
         else:
             os.environ["SYMNMF_H16_MIN_N"] = old
+
+
+def test_h16_split_arithmetic_is_exact_ieee(m):
+    # the split warps' arithmetic, through its test entry point, against the same
+    # steps in IEEE float32 on the host: hi = v rounded to 11 significant bits
+    # (Veltkamp, factor 2^13 + 1), lo = v - hi, both to fp16, bit for bit.  (A
+    # split that lost lo, or rounded differently, would still pass the fit
+    # tolerances above: the tensor core's accumulation error is as large.)
+    import torch
+    from symmetric_nmf_clustering_b200 import _lib as L
+    lib = L.load()
+    rng = np.random.default_rng(21)
+    n = 1 << 16
+    x = np.concatenate([rng.random(n // 2, dtype=np.float32),
+                        (rng.random(n // 4, dtype=np.float32) * 1e-3).astype(np.float32),
+                        np.exp2(rng.uniform(-20, 0, n // 4)).astype(np.float32)])
+    for scale in (16384.0, 2.0 ** -6, 1.0):
+        xd = torch.from_numpy(x).to(DEV)
+        hi = torch.empty(n // 2, dtype=torch.int32, device=DEV)
+        lo = torch.empty(n // 2, dtype=torch.int32, device=DEV)
+        assert lib.symnmf_test_split16(xd.data_ptr(), n, scale, hi.data_ptr(), lo.data_ptr(),
+                                       torch.cuda.current_stream().cuda_stream) == 0
+        torch.cuda.synchronize()
+        v = (x * np.float32(scale)).astype(np.float32)
+        t = (v * np.float32(8193.0)).astype(np.float32)
+        h = (t - (t - v).astype(np.float32)).astype(np.float32)
+        lo_f = (v - h).astype(np.float32)
+        want_h = h.astype(np.float16).view(np.uint16).astype(np.uint32)
+        want_l = lo_f.astype(np.float16).view(np.uint16).astype(np.uint32)
+        got = hi.cpu().numpy().view(np.uint32)
+        got_l = lo.cpu().numpy().view(np.uint32)
+        assert np.array_equal(got & 0xFFFF, want_h[0::2]) and np.array_equal(got >> 16, want_h[1::2])
+        assert np.array_equal(got_l & 0xFFFF, want_l[0::2]) and np.array_equal(got_l >> 16, want_l[1::2])
+        # hi is exactly the fp16 value (no rounding left for the conversion) where it is normal
+        normal = np.abs(h) >= 2.0 ** -14
+        assert np.array_equal(h[normal].astype(np.float16).astype(np.float32), h[normal])
