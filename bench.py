@@ -218,16 +218,17 @@ def _timed(torch, fn):
 
 
 def stream_clock_bins(m, torch, dev, S, H0, n, k, peak):
-    """The S-stream's launch time against the SM clock: 60 back-to-back
-    products Y = S H (the sustained regime, where the power cap lowers the SM
-    clock) after a second idle, then 12 launches spaced by 40 ms idle, with
-    nvidia-smi clock samples every 50 ms.  Each back-to-back launch takes the
-    clock sampled nearest its midpoint; launches are grouped by that clock."""
+    """The fit's S-stream launch time against the SM clock.  After a second of
+    idle, a 60-iteration fit on S (the sustained regime, where the power cap
+    lowers the SM clock) with every stream launch timed by CUDA events; then
+    12 single-pass fits, each after 40 ms of idle (the pass follows the fit's
+    statistics read of S).  nvidia-smi samples the clock every 50 ms; each
+    back-to-back launch takes the sample nearest its midpoint, and launches
+    are grouped by that clock.  The stream is the one the fit runs
+    (`stream_kernel` in the row)."""
     import datetime
     gpu = int(os.environ.get("LOCAL_RANK", "0"))
-    ws = m.workspace(m._lib.OP_SH, n, k, device=dev)
-    X = H0.contiguous()
-    m.sh(S, X, ws=ws)
+    m.fit(S, k, seed=1000, max_iters=1, rel_tol=0.0)   # warm (workspace, attributes)
     out_f = tempfile.TemporaryFile(mode="w+")
     proc = subprocess.Popen(["nvidia-smi", "-i", str(gpu), "--query-gpu=timestamp,clocks.sm",
                              "--format=csv,noheader,nounits", "-lms", "50"],
@@ -235,23 +236,18 @@ def stream_clock_bins(m, torch, dev, S, H0, n, k, peak):
     try:
         torch.cuda.synchronize()
         time.sleep(1.0)
-        es = [torch.cuda.Event(enable_timing=True) for _ in range(61)]
-        es[0].record()
-        t_start = time.time()
-        for i in range(60):
-            m.sh(S, X, ws=ws)
-            es[i + 1].record()
+        _, st = m.fit(S, k, seed=1000, max_iters=59, rel_tol=0.0, stream_times=True)
         torch.cuda.synchronize()
-        b2b = [es[i].elapsed_time(es[i + 1]) for i in range(60)]
+        t_end = time.time()
+        b2b = st["stream_ms_each"]
+        t_start = t_end - st["loop_ms"] / 1e3   # the loop ends just before the call returns
+        kind = m._lib.STREAM_KERNEL_NAMES.get(st.get("stream_kernel", 0), "stream_tc_kernel")
         spaced = []
         for _ in range(12):
             time.sleep(0.04)
-            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            a.record()
-            m.sh(S, X, ws=ws)
-            b.record()
+            _, s1 = m.fit(S, k, seed=1000, max_iters=0, rel_tol=0.0, stream_times=True)
             torch.cuda.synchronize()
-            spaced.append(a.elapsed_time(b))
+            spaced.append(s1["stream_ms_each"][0])
         time.sleep(0.1)
     finally:
         proc.terminate()
@@ -269,8 +265,7 @@ def stream_clock_bins(m, torch, dev, S, H0, n, k, peak):
         except (ValueError, IndexError):
             continue
     gb = (4.0 * n * n + 4.0 * n * k) / 1e9
-    del ws
-    return {"spaced": _launch_row(spaced, [], gb, peak),
+    return {"stream_kernel": kind, "spaced": _launch_row(spaced, [], gb, peak),
             "back_to_back": bin_by_clock(b2b, t_start, samples, gb, peak)}
 
 

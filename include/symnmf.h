@@ -118,6 +118,9 @@ typedef struct {
     double probe_tol;        /* AUTO probe Ritz tolerance; default 1e-6 */
     int check_every;         /* host reads the stop flag every this many iterations; default 16 */
     int timing;              /* 1 = record CUDA-event time of the S-stream kernels in stats */
+    double* stream_ms_out;   /* optional host array: with timing = 1, the CUDA-event time (ms) of each
+                                S-stream launch, in launch order (at most stream_ms_len entries) */
+    int stream_ms_len;       /* capacity of stream_ms_out */
 } symnmf_fit_params;
 
 typedef struct {

@@ -50,6 +50,8 @@ class FitParams(C.Structure):
         ("probe_tol", C.c_double),
         ("check_every", C.c_int),
         ("timing", C.c_int),
+        ("stream_ms_out", C.POINTER(C.c_double)),
+        ("stream_ms_len", C.c_int),
     ]
 
 

@@ -166,13 +166,16 @@ def fit(S: torch.Tensor, k: int, *, H0: torch.Tensor | None = None, G: torch.Ten
         stall_tol: float = 1e-4, gap_threshold: float = 5.0, eigvals=None,
         probe_block: int = 16, probe_max_iter: int = 40, probe_tol: float = 1e-6,
         check_every: int = 16, timing: bool = False, history: bool = False, upper_only: bool = False,
-        out: torch.Tensor | None = None, ws: torch.Tensor | None = None):
+        stream_times: bool = False, out: torch.Tensor | None = None,
+        ws: torch.Tensor | None = None):
     """Factorise S ~ H H^T with H >= 0.  Returns (H, stats dict).
 
     H0 given: INIT_USER from a copy of H0 (or in place when ``out is H0``);
     otherwise the scale-matched seeded init.  G (n x k float32) is the AdaGrad
     accumulator, read and updated in place.  With ``history`` the per-
-    evaluation losses are returned in stats["history"].
+    evaluation losses are returned in stats["history"]; with ``stream_times``
+    (implies ``timing``) the CUDA-event time of every S-stream launch, in
+    order, in stats["stream_ms_each"].
     """
     n, _, lds = _matrix(S, "S")
     if H0 is not None:
@@ -188,7 +191,7 @@ def fit(S: torch.Tensor, k: int, *, H0: torch.Tensor | None = None, G: torch.Ten
                    rel_tol=rel_tol, block_rows=block_rows, grow=int(grow), stall_tol=stall_tol,
                    gap_threshold=gap_threshold, probe_block=probe_block,
                    probe_max_iter=probe_max_iter, probe_tol=probe_tol, check_every=check_every,
-                   timing=int(timing), upper_only=int(upper_only))
+                   timing=int(timing or stream_times), upper_only=int(upper_only))
     if G is not None:
         _dense(G, "G")
         p.G_inout = G.data_ptr()
@@ -197,6 +200,11 @@ def fit(S: torch.Tensor, k: int, *, H0: torch.Tensor | None = None, G: torch.Ten
         hist = (C.c_double * (max_iters + 1))()
         p.loss_history = C.cast(hist, C.POINTER(C.c_double))
         p.loss_history_len = max_iters + 1
+    times = None
+    if stream_times:
+        times = (C.c_double * (max_iters + 8))()
+        p.stream_ms_out = C.cast(times, C.POINTER(C.c_double))
+        p.stream_ms_len = max_iters + 8
     ev = None
     if eigvals is not None:
         ev = (C.c_double * len(eigvals))(*[float(x) for x in eigvals])
@@ -210,6 +218,8 @@ def fit(S: torch.Tensor, k: int, *, H0: torch.Tensor | None = None, G: torch.Ten
     d = st.as_dict()
     if hist is not None:
         d["history"] = np.array(hist[:st.evaluations], dtype=np.float64)
+    if times is not None:
+        d["stream_ms_each"] = [float(x) for x in times[:min(st.stream_launches, max_iters + 8)]]
     return H, d
 
 

@@ -289,6 +289,7 @@ struct Timing {
     int used = 0;
     double ms = 0.0;
     int launches = 0;
+    std::vector<float> each;      // every timed launch, in order
     int record(cudaEvent_t e, cudaStream_t s) {
         if (capturing) SYMNMF_CUDA_TRY(cudaEventRecordWithFlags(e, s, cudaEventRecordExternal));
         else SYMNMF_CUDA_TRY(cudaEventRecord(e, s));
@@ -300,6 +301,7 @@ struct Timing {
             float ms1 = 0.f;
             SYMNMF_CUDA_TRY(cudaEventElapsedTime(&ms1, ev[i], ev[i + 1]));
             ms += ms1;
+            each.push_back(ms1);
             ++launches;
         }
         return SYMNMF_OK;
@@ -329,6 +331,7 @@ struct Timing {
             float ms1 = 0.f;
             SYMNMF_CUDA_TRY(cudaEventElapsedTime(&ms1, ev[i], ev[i + 1]));
             ms += ms1;
+            each.push_back(ms1);
             ++launches;
         }
         used = 0;
@@ -836,6 +839,9 @@ static int fit_impl(const float* S, int64_t n, int64_t lds, int k, const symnmf_
         out->s_sqnorm = hs.s_sqnorm;
         out->evaluations = hs.t;
         out->stream_launches = c.tm.launches;
+        if (P.stream_ms_out != nullptr && P.stream_ms_len > 0)
+            for (int i = 0; i < std::min<int>(P.stream_ms_len, (int)c.tm.each.size()); ++i)
+                P.stream_ms_out[i] = c.tm.each[i];
         out->stream_ms = c.tm.ms;
         out->loop_ms = loop_ms;
         out->kernel_launches = launches();

@@ -171,3 +171,14 @@ def test_h16_split_arithmetic_is_exact_ieee(m):
         # hi is exactly the fp16 value (no rounding left for the conversion) where it is normal
         normal = np.abs(h) >= 2.0 ** -14
         assert np.array_equal(h[normal].astype(np.float16).astype(np.float32), h[normal])
+
+
+def test_per_launch_stream_times(m, h16_on):
+    # stream_times: every S-stream launch's CUDA-event time, in order, summing
+    # to the total the fit reports
+    _, _, S = corr_problem(3000, 150, seed=8)
+    _, st = _fit(m, S, 24, seed=1, max_iters=12, rel_tol=0.0, stream_times=True)
+    each = st["stream_ms_each"]
+    assert len(each) == st["stream_launches"] == 13
+    assert all(x > 0 for x in each)
+    assert abs(sum(each) - st["stream_ms"]) <= 1e-3 * st["stream_ms"] + 1e-3
