@@ -216,12 +216,15 @@ int launch_finalize(int mode, int nblk, int k, const double* tr_part,
 // the finite entries goes to st->s_absmax and its power-of-two scale to st->sscale
 int launch_stats(const float* S, int64_t rows, int64_t n, int64_t lds, double* part, int nblk,
                  double* out3, cudaStream_t s, float* amax_part = nullptr, FitState* st = nullptr);
-// 2^(14 - e) for m < 2^e (m > 0 finite), at most 2^127; 1 otherwise: c m < 2^14
+// 2^(14 - e) for m < 2^e (m > 0 finite), at most 2^63; 1 otherwise: c m < 2^14.
+// The cap keeps 1/c a normal float (the fp16 stream scales its products back
+// by 1/cS and 1/cX); it only matters for m below 2^-49, where c m still lands
+// in fp16's normal range for every entry above 2^-77 m.
 __host__ __device__ inline float pow2_scale_below_2_14(double m) {
     if (!(m > 0.0) || !(m <= 1.7976931348623157e308)) return 1.f;
     int e = 0;
     (void)frexp(m, &e);                 // m = f 2^e, f in [0.5, 1)
-    const int sh = 14 - e > 127 ? 127 : 14 - e;
+    const int sh = 14 - e > 63 ? 63 : 14 - e;
     return ldexpf(1.f, sh);
 }
 int stats_blocks();

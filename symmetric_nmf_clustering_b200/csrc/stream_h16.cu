@@ -263,7 +263,9 @@ stream_h16_kernel(const __grid_constant__ CUtensorMap mapS, const __grid_constan
         const int r = wl * 32 + lane;
         const uint32_t lane_off = (uint32_t)(wl * 32) << 16;
         const float cs = st->sscale;
-        const float inv = 1.f / (st->sscale * st->xscale);   // a power of two: exact
+        // powers of two: the products scale back exactly; applied one after the
+        // other, since cS cX alone could overflow for tiny S and X
+        const float inv_s = 1.f / st->sscale, inv_x = 1.f / st->xscale;
         float acc[KP];
 #pragma unroll
         for (int c = 0; c < KP; ++c) acc[c] = 0.f;
@@ -282,7 +284,8 @@ stream_h16_kernel(const __grid_constant__ CUtensorMap mapS, const __grid_constan
             tmem_wait_ld();
 #pragma unroll
             for (int c = 0; c < KP; ++c)
-                acc[c] += (__uint_as_float(v[c / 8][c % 8]) + __uint_as_float(v[(KP + c) / 8][c % 8])) * inv;
+                acc[c] += (__uint_as_float(v[c / 8][c % 8]) + __uint_as_float(v[(KP + c) / 8][c % 8])) *
+                          inv_s * inv_x;
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&bar_dempty[ts]);

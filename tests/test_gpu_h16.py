@@ -182,3 +182,23 @@ def test_per_launch_stream_times(m, h16_on):
     assert len(each) == st["stream_launches"] == 13
     assert all(x > 0 for x in each)
     assert abs(sum(each) - st["stream_ms"]) <= 1e-3 * st["stream_ms"] + 1e-3
+
+
+def test_h16_tiny_matrix_and_iterate_scales_at_their_cap(m, h16_on):
+    # S = 2^-60 |corr| and H0 near 2^-55: both operand scales reach their cap
+    # (2^63; uncapped, cS cX would overflow fp32), and the products are scaled
+    # back one scale at a time
+    import torch
+    n, k = 1000, 8
+    _, _, C = corr_problem(n, 120, seed=13)
+    S = (C.astype(np.float64) * 2.0 ** -60).astype(np.float32)
+    rng = np.random.default_rng(14)
+    H0 = (rng.random((n, k)) * 2.0 ** -55).astype(np.float32)
+    s_sum, sq, _ = oracle.stats(S)
+    H, st = m.fit(to_dev(S, DEV, pad4=True), k, H0=to_dev(H0, DEV), max_iters=5, rel_tol=0.0,
+                  history=True)
+    torch.cuda.synchronize()
+    ref = oracle.fit_adagrad(S, k, H0, max_iters=5, S_sqnorm=sq)
+    assert st["stream_kernel"] == 1   # STREAM_FP16
+    np.testing.assert_allclose(st["history"], ref.history, rtol=1e-4)
+    assert rel_fro(H.cpu().numpy(), ref.H) <= 1e-3
