@@ -506,9 +506,9 @@ SYMNMF_API int symnmf_test_stall_pipeline(int on);
  * Test hook for the fp16 S-stream's operand split (no counterpart on the
  * pages): applies the split warps' arithmetic to the n values at x (device,
  * n a multiple of 4, x 16-byte aligned): v = scale * x (scale a power of two),
- * hi = v rounded to 11 significant bits by Veltkamp's splitting, lo = v - hi,
- * both rounded to fp16; hi[i] and lo[i] (device, n / 2 words each) hold the
- * fp16 bit patterns of values 2i (low half) and 2i + 1 (high half).
+ * hi = v rounded to fp16, lo = v - hi (exact in fp32) rounded to fp16;
+ * hi[i] and lo[i] (device, n / 2 words each) hold the fp16 bit patterns of
+ * values 2i (low half) and 2i + 1 (high half).
  * Asynchronous on `stream`.
  */
 SYMNMF_API int symnmf_test_split16(const float* x, int64_t n, float scale, uint32_t* hi,

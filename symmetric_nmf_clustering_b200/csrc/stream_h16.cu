@@ -13,8 +13,8 @@
 //
 // Accuracy.  With cS = st->sscale (cS max|S| < 2^14, from the statistics
 // pass) and cX = st->xscale (the same for max|X|, from the previous pass's
-// finalise step), each value v = c s enters as hi = v rounded to 11
-// significant bits (an fp16 number in fp16's normal range) and lo = rn16(v - hi):
+// finalise step), each value v = c s enters as hi = rn16(v) (v to 11
+// significant bits in fp16's normal range) and lo = rn16(v - hi):
 // v = hi + lo to 2^-22 |v| while both parts are normal fp16 numbers, and to
 // 2^-25 in absolute terms below (entries under 2^-17 of the largest).  Then
 //     cS cX S X = S_hi X_hi + S_hi X_lo + S_lo X_hi  (+ S_lo X_lo for 8 columns)
@@ -90,34 +90,24 @@ __device__ __forceinline__ void h16_fail(int* err, volatile int* abort_flag, int
     if (err != nullptr) atomicExch(err, code);
 }
 
-// two fp32 values rounded to fp16 in one 32-bit word, a in the low half
-__device__ __forceinline__ uint32_t pack_h2(float a, float b) {
+// v = hi + lo with hi = rn16(v) and lo = rn16(v - hi), two values at a time:
+// the packed conversion's rounding does the split.  The difference is exact in
+// fp32 (v and hi are fp32 numbers less than half an fp16 ulp apart), and hi
+// carries v to 11 significant bits wherever v is in fp16's normal range.
+__device__ __forceinline__ void split_pair(float a, float b, uint32_t& hi, uint32_t& lo) {
     const __half2 h = __floats2half2_rn(a, b);
-    return *reinterpret_cast<const uint32_t*>(&h);
-}
-
-// v = hi + lo with hi = v rounded to 11 significant bits (Veltkamp's splitting
-// with the factor 2^13 + 1, rounding to nearest in every step), so that hi is an
-// fp16 number wherever v is in fp16's normal range, and lo = v - hi exactly.
-// Only |v| < 2^14 occurs here, so t cannot overflow.
-__device__ __forceinline__ void split_11(float v, float& hi, float& lo) {
-    const float t = __fmul_rn(v, 8193.f);
-    hi = __fsub_rn(t, __fsub_rn(t, v));
-    lo = __fsub_rn(v, hi);
+    const float2 f = __half22float2(h);
+    const __half2 l = __floats2half2_rn(__fsub_rn(a, f.x), __fsub_rn(b, f.y));
+    hi = *reinterpret_cast<const uint32_t*>(&h);
+    lo = *reinterpret_cast<const uint32_t*>(&l);
 }
 
 // Four values q scaled by cs (a power of two: exact), each split as above;
 // h0/l0 hold the fp16 hi/lo of q.x, q.y (low, high half), h1/l1 of q.z, q.w.
 __device__ __forceinline__ void split_scaled4(const float4 q, float cs, uint32_t& h0, uint32_t& h1,
                                               uint32_t& l0, uint32_t& l1) {
-    const float e[4] = {q.x * cs, q.y * cs, q.z * cs, q.w * cs};
-    float h[4], l[4];
-#pragma unroll
-    for (int u = 0; u < 4; ++u) split_11(e[u], h[u], l[u]);
-    h0 = pack_h2(h[0], h[1]);
-    h1 = pack_h2(h[2], h[3]);
-    l0 = pack_h2(l[0], l[1]);
-    l1 = pack_h2(l[2], l[3]);
+    split_pair(q.x * cs, q.y * cs, h0, l0);
+    split_pair(q.z * cs, q.w * cs, h1, l1);
 }
 
 template <int KP>

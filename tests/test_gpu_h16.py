@@ -139,10 +139,10 @@ def test_h16_path_selection(m):
 
 def test_h16_split_arithmetic_is_exact_ieee(m):
     # the split warps' arithmetic, through its test entry point, against the same
-    # steps in IEEE float32 on the host: hi = v rounded to 11 significant bits
-    # (Veltkamp, factor 2^13 + 1), lo = v - hi, both to fp16, bit for bit.  (A
-    # split that lost lo, or rounded differently, would still pass the fit
-    # tolerances above: the tensor core's accumulation error is as large.)
+    # steps in IEEE arithmetic on the host: v = x scale in float32, hi = rn16(v),
+    # lo = rn16(v - hi) (the difference exact in float32), bit for bit.  (A split
+    # that lost lo, or rounded differently, would still pass the fit tolerances
+    # above: the tensor core's accumulation error is as large.)
     import torch
     from symmetric_nmf_clustering_b200 import _lib as L
     lib = L.load()
@@ -159,18 +159,25 @@ def test_h16_split_arithmetic_is_exact_ieee(m):
                                        torch.cuda.current_stream().cuda_stream) == 0
         torch.cuda.synchronize()
         v = (x * np.float32(scale)).astype(np.float32)
-        t = (v * np.float32(8193.0)).astype(np.float32)
-        h = (t - (t - v).astype(np.float32)).astype(np.float32)
+        h16 = v.astype(np.float16)
+        h = h16.astype(np.float32)
         lo_f = (v - h).astype(np.float32)
-        want_h = h.astype(np.float16).view(np.uint16).astype(np.uint32)
+        # the difference is exact: hi and v are float32 numbers less than half an
+        # fp16 ulp apart (computed in float64 as well)
+        assert np.array_equal(lo_f.astype(np.float64), v.astype(np.float64) - h.astype(np.float64))
+        want_h = h16.view(np.uint16).astype(np.uint32)
         want_l = lo_f.astype(np.float16).view(np.uint16).astype(np.uint32)
         got = hi.cpu().numpy().view(np.uint32)
         got_l = lo.cpu().numpy().view(np.uint32)
         assert np.array_equal(got & 0xFFFF, want_h[0::2]) and np.array_equal(got >> 16, want_h[1::2])
         assert np.array_equal(got_l & 0xFFFF, want_l[0::2]) and np.array_equal(got_l >> 16, want_l[1::2])
-        # hi is exactly the fp16 value (no rounding left for the conversion) where it is normal
-        normal = np.abs(h) >= 2.0 ** -14
-        assert np.array_equal(h[normal].astype(np.float16).astype(np.float32), h[normal])
+        # where v is in fp16's normal range, hi + lo carries v to 2^-22 relative,
+        # plus 2^-25 absolute where lo falls below fp16's normal range
+        normal = np.abs(v) >= 2.0 ** -14
+        got_sum = (np.asarray(want_h, np.uint16).view(np.float16).astype(np.float64) +
+                   np.asarray(want_l, np.uint16).view(np.float16).astype(np.float64))
+        err = np.abs(got_sum - v)[normal]
+        assert np.all(err <= 2.0 ** -22 * np.abs(v[normal]) + 2.0 ** -25)
 
 
 def test_per_launch_stream_times(m, h16_on):
