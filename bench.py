@@ -50,7 +50,6 @@ SAMPLE_ROWS = 8192   # oracle sample: leading principal r x r block of the same 
 # its kernel changes.
 STREAM_TRAFFIC_RATIO = {
     "stream_tc_kernel": (1.618906e9 + 13.768704e6) / (4.0 * 20000 ** 2 + 4.0 * 20000 * 24),
-    "stream_h16_kernel": (1.611688e9 + 6.660096e6) / (4.0 * 20000 ** 2 + 4.0 * 20000 * 24),
 }
 STREAM_TRAFFIC_SOURCE = ("ncu dram__bytes_read.sum + dram__bytes_write.sum of one launch at "
                          "n = 20,000, k = 24, scaled to this launch by algorithmic bytes")

@@ -18,8 +18,9 @@
 // v = hi + lo to 2^-22 |v| while both parts are normal fp16 numbers, and to
 // 2^-25 in absolute terms below (entries under 2^-17 of the largest).  Then
 //     cS cX S X = S_hi X_hi + S_hi X_lo + S_lo X_hi  (+ S_lo X_lo for 8 columns)
-// accumulated in fp32 in tensor memory and scaled back by 1 / (cS cX), a
-// power of two, when the split warps fold each finished accumulator.
+// accumulated in fp32 in tensor memory over each pair of stages, folded into
+// registers with round-to-nearest fp32 adds, and scaled back by 1 / cS and
+// 1 / cX (powers of two: exact) once the split's range is done.
 //
 // Per CTA (256 threads, two CTAs per SM): a 128-row tile of S times the
 // contraction range of its split, in stages of 64 columns:
@@ -34,7 +35,7 @@
 //   warp 2      tensor-memory allocator
 //   warps 4-7   split warps: thread r reads row r of the stage from shared
 //               memory, scales and splits it, stores hi and lo into tensor
-//               memory lane r, folds the previous stage's accumulator
+//               memory lane r, folds each pair of stages' accumulator
 //   all warps   in the last split CTA of the tile, the epilogue (epilogue.cuh)
 #include <cuda_fp16.h>
 #include <cudaTypedefs.h>
@@ -61,7 +62,7 @@ constexpr int H16_BM = 128;                    // S rows per tile = tensor-memor
 constexpr int H16_BK = 64;                     // columns per stage (two 32-column S boxes)
 constexpr int H16_NSS = 3;                     // shared-memory slots of S
 constexpr int H16_NSX = 2;                     // shared-memory slots of X
-constexpr int H16_NT = 2;                      // tensor-memory stages (= accumulator sets)
+constexpr int H16_NT = 2;                      // A stages in tensor memory = accumulator sets (a pair each)
 constexpr int H16_NDONE = 4;                   // stage-completion barriers: > both rings, a multiple of each
 constexpr int H16_THREADS = 256;
 constexpr uint32_t H16_BOX = H16_BM * 32 * 4;  // 16 KB: one 128 x 32 fp32 box of S
@@ -216,16 +217,22 @@ stream_h16_kernel(const __grid_constant__ CUtensorMap mapS, const __grid_constan
                 mbar_wait(&bar_xfull[s % H16_NSX], (uint32_t)(s / H16_NSX) & 1u);
         }
     } else if (warp == 1 && lane == 0 && ksteps > 0) {
-        // ---------------- MMA issuer: stage s accumulates into D[s % 2]
+        // ---------------- MMA issuer: stage s accumulates into D[(s / 2) % 2]
         constexpr uint32_t id1 = idesc_f16(H16_BM, Cfg::N1);
         constexpr uint32_t id2 = idesc_f16(H16_BM, Cfg::N2);
         for (int s = 0; s < ksteps; ++s) {
             if (abort_sh) break;
             const int slot = s % H16_NSX;
             const int ts = s % H16_NT;
+            // stages 2g and 2g + 1 accumulate into set g % 2, which the split
+            // warps must have folded for pair g - 2 first
+            const int g = s / 2;
+            const int dset = g % H16_NT;
+            const bool first = (s % 2) == 0;
             bool ok = mbar_wait(&bar_tfull[ts], (uint32_t)(s / H16_NT) & 1u) &&
                       mbar_wait(&bar_xfull[slot], (uint32_t)(s / H16_NSX) & 1u);
-            if (ok && s >= H16_NT) ok = mbar_wait(&bar_dempty[ts], (uint32_t)((s / H16_NT) - 1) & 1u);
+            if (ok && first && g >= H16_NT)
+                ok = mbar_wait(&bar_dempty[dset], (uint32_t)((g / H16_NT) - 1) & 1u);
             if (!ok) {
                 h16_fail(err, &abort_sh, 2);
                 break;
@@ -234,11 +241,11 @@ stream_h16_kernel(const __grid_constant__ CUtensorMap mapS, const __grid_constan
             const uint32_t b_base = smem_u32(smemB + slot * Cfg::B_BYTES);
             const uint32_t a_hi = tbase + Cfg::COL_A + (uint32_t)ts * Cfg::TSTAGE;
             const uint32_t a_lo = a_hi + 32u;
-            const uint32_t d = tbase + (uint32_t)ts * Cfg::DSTRIDE;
+            const uint32_t d = tbase + (uint32_t)dset * Cfg::DSTRIDE;
 #pragma unroll
             for (int kk = 0; kk < H16_BK / 16; ++kk) {
                 const uint64_t bd = umma_desc_sw128(b_base + (uint32_t)kk * 32u);
-                umma_f16_ts(d, a_hi + (uint32_t)kk * 8u, bd, id1, kk == 0 ? 0u : 1u);
+                umma_f16_ts(d, a_hi + (uint32_t)kk * 8u, bd, id1, (kk == 0 && first) ? 0u : 1u);
                 umma_f16_ts(d, a_lo + (uint32_t)kk * 8u, bd, id2, 1u);
             }
             umma_commit(&bar_done[s % H16_NDONE]);
@@ -261,24 +268,23 @@ stream_h16_kernel(const __grid_constant__ CUtensorMap mapS, const __grid_constan
         for (int c = 0; c < KP; ++c) acc[c] = 0.f;
         bool alive = true;
 
-        // fold accumulator D[s % 2] of stage s into acc (round-to-nearest fp32 adds)
-        auto drain = [&](int s) -> bool {
-            const int ts = s % H16_NT;
-            if (!__all_sync(0xffffffffu, mbar_wait(&bar_done[s % H16_NDONE], (uint32_t)(s / H16_NDONE) & 1u)))
+        // fold accumulator set dset, complete once the MMAs of stage s_last are
+        // done, into acc (round-to-nearest fp32 adds)
+        auto drain = [&](int s_last, int dset) -> bool {
+            if (!__all_sync(0xffffffffu, mbar_wait(&bar_done[s_last % H16_NDONE], (uint32_t)(s_last / H16_NDONE) & 1u)))
                 return false;
             tc_fence_after();
-            const uint32_t dcol = tbase + lane_off + (uint32_t)ts * Cfg::DSTRIDE;
+            const uint32_t dcol = tbase + lane_off + (uint32_t)dset * Cfg::DSTRIDE;
             uint32_t v[2 * KP / 8][8];
 #pragma unroll
             for (int g = 0; g < 2 * KP / 8; ++g) tmem_ld_32x32b_x8(dcol + (uint32_t)g * 8u, v[g]);
             tmem_wait_ld();
 #pragma unroll
             for (int c = 0; c < KP; ++c)
-                acc[c] += (__uint_as_float(v[c / 8][c % 8]) + __uint_as_float(v[(KP + c) / 8][c % 8])) *
-                          inv_s * inv_x;
+                acc[c] += __uint_as_float(v[c / 8][c % 8]) + __uint_as_float(v[(KP + c) / 8][c % 8]);
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&bar_dempty[ts]);
+            if (lane == 0) mbar_arrive(&bar_dempty[dset]);
             return true;
         };
 
@@ -329,14 +335,15 @@ stream_h16_kernel(const __grid_constant__ CUtensorMap mapS, const __grid_constan
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&bar_tfull[ts]);
-            // the previous stage's MMAs are done by now: fold its accumulator
-            if (s >= 1 && !drain(s - 1)) {
+            // at the start of a pair, the previous pair's MMAs are done by now:
+            // fold its accumulator set
+            if (s >= 2 && s % 2 == 0 && !drain(s - 1, ((s - 1) / 2) % H16_NT)) {
                 if (lane == 0) h16_fail(err, &abort_sh, 4);
                 alive = false;
                 break;
             }
         }
-        if (alive && ksteps > 0 && !drain(ksteps - 1)) {
+        if (alive && ksteps > 0 && !drain(ksteps - 1, ((ksteps - 1) / 2) % H16_NT)) {
             if (lane == 0) h16_fail(err, &abort_sh, 5);
             alive = false;
         }
@@ -350,7 +357,7 @@ stream_h16_kernel(const __grid_constant__ CUtensorMap mapS, const __grid_constan
             float* out = part + (int64_t)split * n * k + i * (int64_t)k;
 #pragma unroll
             for (int c = 0; c < KP; ++c)
-                if (c < k) out[c] = acc[c];
+                if (c < k) out[c] = acc[c] * inv_s * inv_x;
         }
         if (go && counters != nullptr) {
             // the last split CTA of this row tile runs the epilogue for it
