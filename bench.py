@@ -73,7 +73,7 @@ def parse():
                     help="time the upper-triangle S-stream (upper_only = 1) in the main loop")
     ap.add_argument("--h16-min-n", type=int, default=None,
                     help="size from which full-batch fits run the fp16 S-stream "
-                         "(sets SYMNMF_H16_MIN_N; the library's default is 50000, 0 = never)")
+                         "(sets SYMNMF_H16_MIN_N; the library's default is 20000, 0 = never)")
     args = ap.parse_args()
     if args.h16_min_n is not None:
         os.environ["SYMNMF_H16_MIN_N"] = str(args.h16_min_n)

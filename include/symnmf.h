@@ -144,9 +144,9 @@ typedef struct {
 
 /* Which S-stream ran the full-batch passes of a fit (symnmf_fit_stats.stream_kernel):
  * TF32: the tensor-core stream with S and X as exact TF32 splits (the default
- *       below n = 50,000, for k > 24, and for Block-SVRG);
+ *       below n = 20,000, for k > 24, and for Block-SVRG);
  * FP16: the tensor-core stream with S and X as power-of-two scaled fp16 hi/lo
- *       pairs (the AdaGrad solver from n = 50,000 up, k <= 24; the environment
+ *       pairs (the AdaGrad solver from n = 20,000 up, k <= 24; the environment
  *       variable SYMNMF_H16_MIN_N moves the threshold, 0 turns it off);
  * UPPER: the upper-triangle stream (upper_only = 1);
  * CUDA_CORE: the CUDA-core stream (SYMNMF_STREAM=cuda_core). */

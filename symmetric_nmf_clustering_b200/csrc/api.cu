@@ -247,13 +247,14 @@ static int plan_fit(const Dev& d, Arena& a, int64_t n, int k, const symnmf_fit_p
 }
 
 // The full-batch loop of the AdaGrad solver streams S through the fp16
-// tensor-core kernel (stream_h16.cu) from n = 50,000 up (k <= 24, tensor-core
-// path, full matrix); below that the TF32 kernel, which measured as fast or
-// faster there (its passes need no extra launch for the operand split).  SYMNMF_H16_MIN_N overrides the size (0: never).
+// tensor-core kernel (stream_h16.cu) from n = 20,000 up (k <= 24, tensor-core
+// path, full matrix); below that the TF32 kernel, which measured about as fast
+// there (its passes need no extra launch for the operand split).
+// SYMNMF_H16_MIN_N overrides the size (0: never).
 static int64_t h16_min_n() {
     const char* e = getenv("SYMNMF_H16_MIN_N");   // read per call: tests switch it
     if (e != nullptr && *e != 0) return std::strtoll(e, nullptr, 10);
-    return 50000;
+    return 20000;
 }
 static bool h16_path(int64_t n, int k, const symnmf_fit_params& P) {
     const int64_t m = h16_min_n();

@@ -1,7 +1,7 @@
 """Parity of the fp16 S-stream of the full-batch loop (stream_h16.cu).
 
 The library runs the AdaGrad solver's full-batch passes through this kernel
-from n = 50,000 up (k <= 24); SYMNMF_H16_MIN_N lowers the threshold so that
+from n = 20,000 up (k <= 24); SYMNMF_H16_MIN_N lowers the threshold so that
 it runs at sizes the oracle follows (the variable is read on every call).
 S and X enter as power-of-two scaled fp16 hi/lo pairs, so the tolerances are
 those of the TF32 path: per-step H and G 1e-4, trajectories H 1e-3 and loss
