@@ -15,9 +15,13 @@
 // pass) and cX = st->xscale (the same for max|X|, from the previous pass's
 // finalise step), each value v = c s enters as hi = rn16(v) (v to 11
 // significant bits in fp16's normal range) and lo = rn16(v - hi):
-// v = hi + lo to 2^-22 |v| while both parts are normal fp16 numbers, and to
-// 2^-25 in absolute terms below (entries under 2^-17 of the largest).  Then
-//     cS cX S X = S_hi X_hi + S_hi X_lo + S_lo X_hi  (+ S_lo X_lo for 8 columns)
+// v = hi + lo to 2^-22 |v| where lo is a normal fp16 number, and to 2^-25 in
+// absolute terms where it is not (more than 2^-22 |v| only for v below 2^-3,
+// about 2^-16 of the largest).
+// Then
+//     cS cX S X = S_hi X_hi + S_hi X_lo + S_lo X_hi
+// (+ S_lo X_lo on the columns c < N2 - KP), each entry to first order within
+// 3 * 2^-22 sum_j |s_ij| |x_jc| + 2^-25 sum_j (|s_ij| + |x_jc|) in scaled units,
 // accumulated in fp32 in tensor memory over each pair of stages, folded into
 // registers with round-to-nearest fp32 adds, and scaled back by 1 / cS and
 // 1 / cX (powers of two: exact) once the split's range is done.
