@@ -3,9 +3,13 @@
 //
 //  - cyclic Jacobi with eigenvectors (Golub & Van Loan, "Matrix
 //    Computations", section 8.5) for the b x b Gram matrices of a block;
-//  - Householder reduction to tridiagonal form (section 8.3.1) followed by
-//    Sturm-sequence bisection (section 8.4.1) for the leading eigenvalues of
-//    the block-tridiagonal Lanczos matrix.
+//  - reduction to tridiagonal form followed by Sturm-sequence bisection
+//    (section 8.4.1) for the leading eigenvalues of the block-tridiagonal
+//    Lanczos matrix: for a band matrix (the Lanczos matrix has half-bandwidth
+//    b) by Givens rotations with bulge chasing (H. R. Schwarz,
+//    "Tridiagonalization of a symmetric band matrix", Numerische Mathematik
+//    12, 1968), O(m^2 b) instead of O(m^3); for a full matrix by Householder
+//    reflections (section 8.3.1).
 #include "hostla.h"
 
 #include <algorithm>
@@ -116,6 +120,85 @@ static void householder_tridiag(int m, std::vector<double>& A, std::vector<doubl
     d[m - 1] = a(m - 1, m - 1);
 }
 
+// Largest |i - j| over the nonzero entries of an m x m matrix (row-major).
+static int half_bandwidth(int m, const std::vector<double>& A) {
+    int w = 0;
+    for (int i = 0; i < m; ++i) {
+        const double* ai = &A[(size_t)i * m];
+        for (int j = m - 1; j > i + w; --j)
+            if (ai[j] != 0.0 || A[(size_t)j * m + i] != 0.0) {
+                w = j - i;
+                break;
+            }
+    }
+    return w;
+}
+
+// Tridiagonal form of a symmetric band matrix of half-bandwidth w (dense
+// row-major A; only its lower band is read): the entries at distance
+// dd = w, w - 1, ..., 2 below the diagonal are zeroed one width at a time,
+// column by column, each by a rotation in the plane (c - 1, c) of its row c.
+// Such a rotation mixes columns c - 1 and c, which fills entry (c + dd, c - 1)
+// just outside the band; the next rotation, in plane (c + dd - 1, c + dd),
+// zeroes that and moves the fill dd further down, until it leaves the matrix.
+// The rotations are orthogonal similarities, so the eigenvalues are kept to
+// rounding.  The lower band is held compactly, row i's entries at distances
+// 0 .. w + 1 (the last for the fill) side by side, so that a rotation's
+// updates stay within a few cache lines.
+static void band_tridiag(int m, int w, const std::vector<double>& A, std::vector<double>& d,
+                         std::vector<double>& e) {
+    const int W = w + 2;
+    std::vector<double> band((size_t)m * W, 0.0);
+    // entry (i, j), j <= i <= j + w + 1
+    auto a = [&](int i, int j) -> double& { return band[(size_t)i * W + (i - j)]; };
+    for (int i = 0; i < m; ++i)
+        for (int j = std::max(0, i - w); j <= i; ++j) a(i, j) = A[(size_t)i * m + j];
+    for (int dd = w; dd >= 2; --dd) {
+        for (int k = 0; k + dd < m; ++k) {
+            int r = k, c = k + dd;   // the entry (c, r) to zero
+            while (c < m) {
+                const int p = c - 1;
+                const double x = a(p, r), y = a(c, r);
+                if (y == 0.0) break;   // nothing to zero: no fill either
+                double h = std::sqrt(x * x + y * y);
+                if (!(h > 0.0) || !std::isfinite(h)) h = std::hypot(x, y);   // under/overflow
+                const double cs = x / h, sn = y / h;
+                // rows p and c left of the 2 x 2 diagonal block: their nonzeros
+                // start at column p - dd (row p's band edge)
+                for (int j = std::max(0, p - dd); j < p; ++j) {
+                    double& u = a(p, j);
+                    double& v = a(c, j);
+                    const double u0 = u, v0 = v;
+                    u = cs * u0 + sn * v0;
+                    v = cs * v0 - sn * u0;
+                }
+                // the diagonal block
+                const double app = a(p, p), acp = a(c, p), acc = a(c, c);
+                a(p, p) = cs * cs * app + 2.0 * cs * sn * acp + sn * sn * acc;
+                a(c, c) = sn * sn * app - 2.0 * cs * sn * acp + cs * cs * acc;
+                a(c, p) = cs * sn * (acc - app) + (cs * cs - sn * sn) * acp;
+                // columns p and c below it: nonzeros down to row c + dd (column
+                // c's band edge), where the fill appears in column p
+                const int ihi = std::min(m - 1, c + dd);
+                for (int i = c + 1; i <= ihi; ++i) {
+                    double& u = a(i, p);
+                    double& v = a(i, c);
+                    const double u0 = u, v0 = v;
+                    u = cs * u0 + sn * v0;
+                    v = cs * v0 - sn * u0;
+                }
+                a(c, r) = 0.0;
+                r = p;        // the fill entry (c + dd, c - 1)
+                c += dd;
+            }
+        }
+    }
+    d.assign(m, 0.0);
+    e.assign(m > 1 ? m - 1 : 0, 0.0);
+    for (int i = 0; i < m; ++i) d[i] = a(i, i);
+    for (int i = 0; i + 1 < m; ++i) e[i] = a(i + 1, i);
+}
+
 // Number of eigenvalues of the tridiagonal (d, e) below each of four shifts
 // x[r] (Sturm counts through the pivots of the LDL^T factorisations of
 // T - x[r] I), as four independent recurrences so that their divisions overlap.
@@ -138,8 +221,18 @@ static void sturm_below4(const std::vector<double>& d, const std::vector<double>
 }
 
 void sym_top_eigvals(int m, std::vector<double> A, int count, std::vector<double>& out) {
+    // scale by a power of two (exact) so that the largest entry is about 1:
+    // the rotations' squares and the Sturm recurrence's e^2 then neither
+    // overflow nor underflow for any finite input scale
+    double amax = 0.0;
+    for (double v : A) amax = std::max(amax, std::fabs(v));
+    const int ex = amax > 0.0 && std::isfinite(amax) ? std::ilogb(amax) : 0;
+    if (ex != 0)
+        for (double& v : A) v = std::ldexp(v, -ex);
     std::vector<double> d, e;
-    householder_tridiag(m, A, d, e);
+    const int w = half_bandwidth(m, A);
+    if (w <= m / 8) band_tridiag(m, w, A, d, e);   // also w <= 1: read off d and e
+    else householder_tridiag(m, A, d, e);
     // Gershgorin interval
     double lo = 0.0, hi = 0.0;
     for (int i = 0; i < m; ++i) {
@@ -186,6 +279,8 @@ void sym_top_eigvals(int m, std::vector<double> A, int count, std::vector<double
         }
         for (int q = 0; q < g; ++q) out[j0 + q] = 0.5 * (blo[j0 + q] + bhi[j0 + q]);
     }
+    if (ex != 0)
+        for (double& v : out) v = std::ldexp(v, ex);
 }
 
 bool cholesky_upper(int m, const std::vector<double>& M, std::vector<double>& R) {

@@ -1,8 +1,9 @@
 """The spectral probe's host eigen-solvers against LAPACK (numpy).
 
 The block Lanczos probe reduces S to a block tridiagonal matrix T of at most a
-few hundred rows and takes its leading eigenvalues on the host (Householder
-tridiagonalisation and Sturm bisection); Cholesky and cyclic Jacobi
+few hundred rows and takes its leading eigenvalues on the host (reduction to
+tridiagonal form: by bulge-chasing Givens rotations for a band matrix, by
+Householder reflections otherwise; then Sturm bisection); Cholesky and cyclic Jacobi
 orthonormalise each new block.  These run without a GPU: the test compiles
 them with a small C shim and checks them against numpy.linalg.
 """
@@ -78,6 +79,44 @@ def test_top_eigenvalues_block_tridiagonal(hl, blocks, b):
     T = block_tridiagonal(np.random.default_rng(blocks * b), blocks, b)
     ref = np.sort(np.linalg.eigvalsh(T))[::-1][:26]
     got = top(hl, T, 26)
+    assert np.max(np.abs(got - ref)) <= 1e-11 * np.max(np.abs(ref))
+
+
+@pytest.mark.parametrize("blocks,b,count", [(41, 16, 64), (30, 8, 26), (70, 4, 40)])
+def test_top_eigenvalues_band_path_at_the_probe_sizes(hl, blocks, b, count):
+    # m >= 8 b: the band reduction (Givens rotations with bulge chasing) runs;
+    # (41, 16) is the 64-eigenvalue probe's final Rayleigh-Ritz matrix
+    T = block_tridiagonal(np.random.default_rng(blocks + b), blocks, b)
+    ref = np.sort(np.linalg.eigvalsh(T))[::-1][:count]
+    got = top(hl, T, count)
+    assert np.max(np.abs(got - ref)) <= 1e-11 * np.max(np.abs(ref))
+
+
+@pytest.mark.parametrize("w", [1, 2, 3, 7])
+def test_top_eigenvalues_random_band_matrices(hl, w):
+    # general band matrices (full bands, not triangular coupling blocks), zero
+    # entries inside the band, a decoupled block and an indefinite spectrum
+    rng = np.random.default_rng(w + 40)
+    m = 120
+    A = np.zeros((m, m))
+    for dd in range(w + 1):
+        v = rng.standard_normal(m - dd)
+        v[rng.random(m - dd) < 0.2] = 0.0
+        A += np.diag(v, -dd) + (np.diag(v, dd) if dd else 0)
+    A[60:, :60] = 0.0
+    A[:60, 60:] = 0.0
+    ref = np.sort(np.linalg.eigvalsh(A))[::-1][:30]
+    got = top(hl, A, 30)
+    assert np.max(np.abs(got - ref)) <= 1e-11 * np.max(np.abs(ref))
+
+
+@pytest.mark.parametrize("scale", [1e-200, 1e-150, 1e150, 1e200])
+def test_top_eigenvalues_band_path_far_from_unit_scale(hl, scale):
+    # rotations whose squared entries under- or overflow fall back to hypot
+    T = block_tridiagonal(np.random.default_rng(9), 20, 4) * scale
+    ref = np.sort(np.linalg.eigvalsh(T / scale))[::-1][:10] * scale
+    got = top(hl, T, 10)
+    assert np.all(np.isfinite(got))
     assert np.max(np.abs(got - ref)) <= 1e-11 * np.max(np.abs(ref))
 
 
