@@ -740,7 +740,8 @@ def run_ours(args):
             "config": bench_config(args.workload, world),
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak, "traffic": traffic,
-                         "traffic_source": STREAM_TRAFFIC_SOURCE if traffic is not None else None,
+                         "traffic_source": (STREAM_TRAFFIC_SOURCE if traffic is not None else
+                                            "null: no ncu capture of this kernel since its last change"),
                          "kernel": kname,
                          "peak_source": peak_src,
                          "alg_bytes_per_launch": alg_bytes, "launch_ms": stream_ms,
