@@ -741,7 +741,9 @@ def run_ours(args):
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak, "traffic": traffic,
                          "traffic_source": (STREAM_TRAFFIC_SOURCE if traffic is not None else
-                                            "null: no ncu capture of this kernel since its last change"),
+                                            "null: no ncu capture of this kernel since its last change"
+                                            if ratio is None else
+                                            "null: the capture's ratio applies to the n = 100,000, k = 24 launch only"),
                          "kernel": kname,
                          "peak_source": peak_src,
                          "alg_bytes_per_launch": alg_bytes, "launch_ms": stream_ms,
