@@ -175,7 +175,11 @@ def fit(S: torch.Tensor, k: int, *, H0: torch.Tensor | None = None, G: torch.Ten
     accumulator, read and updated in place.  With ``history`` the per-
     evaluation losses are returned in stats["history"]; with ``stream_times``
     (implies ``timing``) the CUDA-event time of every S-stream launch, in
-    order, in stats["stream_ms_each"].
+    order, in stats["stream_ms_each"].  stats["stream_kernel"] names the
+    S-stream that ran the full-batch passes (``_lib.STREAM_KERNEL_NAMES``):
+    the fp16 stream for the AdaGrad solver from n = 20,000 (k <= 24; the
+    environment variable SYMNMF_H16_MIN_N moves the threshold, 0 turns it
+    off), the TF32 stream otherwise.
     """
     n, _, lds = _matrix(S, "S")
     if H0 is not None:
